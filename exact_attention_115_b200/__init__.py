@@ -1,0 +1,200 @@
+"""B200 (sm_100a) fused exact attention: thin Python binding of the C ABI.
+
+Every computation happens in the CUDA kernels of ``libfa_b200.so`` (built by
+``python -m exact_attention_115_b200.build``); this module only checks
+tensors and marshals pointers, sizes and the current CUDA stream.  There is no
+CPU or PyTorch fallback: if the library is missing or a tensor is not on a
+CUDA device, the call raises.
+
+Layouts follow ``include/fa.h``: Q/O/dO [B, H, Nq, d], K/V [B, H, Nk, d],
+L [B, H, Nq] float32 natural-log logsumexp.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
+
+FA_FP32, FA_BF16, FA_FP16 = 0, 1, 2
+FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = (
+    0, -1, -2, -3, -4, -5)
+STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED",
+                -3: "FA_ERR_WORKSPACE", -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT"}
+
+# Every symbol include/fa.h declares: name -> (restype, argtypes)
+_VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+SIGNATURES = {
+    "fa_fwd": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
+    "fa_bwd_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
+    "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I,
+                    _VP, _SZ, _VP]),
+    "fa_set_bwd_dq_mode": (_I, [_I]),
+    "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
+    "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
+    "fa_status": (_I, [_VP]),
+    "fa_version": (ctypes.c_char_p, []),
+}
+
+_lib = None
+
+
+class FAError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
+        self.code = code
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfa_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m exact_attention_115_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in SIGNATURES.items():
+            f = getattr(h, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = h
+    return _lib
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return FA_BF16
+    if t.dtype == torch.float16:
+        return FA_FP16
+    if t.dtype == torch.float32:
+        return FA_FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _check(name, t, shape=None, dtype=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _raise(fn, code):
+    if code != FA_OK:
+        raise FAError(fn, code)
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+    """O, L = attention(q, k, v).  Returns (O [B,H,Nq,d] q.dtype, L [B,H,Nq] fp32)."""
+    _check("q", q)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    _check("k", k, (B, H, Nk, d), q.dtype)
+    _check("v", v, (B, H, Nk, d), q.dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    _check("out", out, q.shape, q.dtype)
+    _check("lse", lse, (B, H, Nq), torch.float32)
+    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                      B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
+                      _stream(q.device))
+    _raise("fa_fwd", rc)
+    return out, lse
+
+
+def bwd_workspace_bytes(B, H, Nq, Nk, d, dtype=torch.bfloat16) -> int:
+    code = {torch.bfloat16: FA_BF16, torch.float16: FA_FP16, torch.float32: FA_FP32}[dtype]
+    return int(lib().fa_bwd_workspace_bytes(B, H, Nq, Nk, d, code))
+
+
+def set_bwd_dq_mode(mode: int) -> int:
+    """0 auto, 1 reduce-add into one fp32 buffer, 2 per-K/V-block partials."""
+    rc = lib().fa_set_bwd_dq_mode(int(mode))
+    if rc < 0:
+        raise FAError("fa_set_bwd_dq_mode", rc)
+    return rc
+
+
+def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
+             dq=None, dk=None, dv=None, workspace=None):
+    """dQ, dK, dV of attention given the forward's O and L and the upstream dO."""
+    _check("q", q)
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    for name, t, n in (("k", k, Nk), ("v", v, Nk), ("o", o, Nq), ("do", do, Nq)):
+        _check(name, t, (B, H, n, d), q.dtype)
+    _check("lse", lse, (B, H, Nq), torch.float32)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
+        _check(name, t, ref.shape, q.dtype)
+    need = bwd_workspace_bytes(B, H, Nq, Nk, d, q.dtype)
+    if workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    _check("workspace", workspace)
+    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                      B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
+                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                      _stream(q.device))
+    _raise("fa_bwd", rc)
+    return dq, dk, dv
+
+
+def decode_workspace_bytes(B, H, Nk, d, num_splits=0) -> int:
+    return int(lib().fa_decode_workspace_bytes(B, H, Nk, d, num_splits))
+
+
+def decode(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
+           workspace=None):
+    """Split-KV decode: q [B,H,1,d], k/v [B,H,Nk,d] -> (O [B,H,1,d], L [B,H,1])."""
+    _check("q", q)
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes exactly one query row per (batch, head)")
+    Nk = k.shape[2]
+    _check("k", k, (B, H, Nk, d), q.dtype)
+    _check("v", v, (B, H, Nk, d), q.dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    out = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device) if lse is None else lse
+    need = decode_workspace_bytes(B, H, Nk, d, num_splits)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    rc = lib().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         B, H, Nk, d, float(scale), _dtype_code(q), int(num_splits),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream(q.device))
+    _raise("fa_decode", rc)
+    return out, lse
+
+
+def status(device=None) -> int:
+    """Synchronise the current stream and return (and clear) the kernel
+    error status: FA_OK, FA_ERR_TIMEOUT or FA_ERR_CUDA."""
+    return int(lib().fa_status(_stream(device)))
+
+
+def version() -> str:
+    return lib().fa_version().decode()

@@ -1,0 +1,278 @@
+// C ABI of the attention library: argument checks, TMA descriptor set-up,
+// workspace layout and kernel launches.  No device memory is allocated here
+// and nothing synchronises except fa_status.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fa.h"
+#include "launch.h"
+
+namespace fa {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+int g_dq_mode = 0;  // 0 auto, 1 reduce-add, 2 partial buffers
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+int elem_size(int dtype) { return dtype == FA_FP32 ? 4 : 2; }
+
+CUtensorMapDataType tma_type(int dtype) {
+  switch (dtype) {
+    case FA_BF16: return CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    case FA_FP16: return CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+    default: return CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  }
+}
+
+// 3-D map over a contiguous [BH, N, d] tensor: x = d (innermost), y = row,
+// z = batch·head.  The box is one 128-byte swizzled column block of
+// `box_rows` rows; rows past N read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int BH, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const int es = elem_size(dtype);
+  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
+  cuuint64_t strides[2] = {cuuint64_t(d) * es, cuuint64_t(N) * d * es};
+  cuuint32_t box[3] = {cuuint32_t(128 / es), cuuint32_t(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, tma_type(dtype), 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int check_common(int B, int H, int Nq, int Nk, int d, float scale, int dtype) {
+  if (B <= 0 || H <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return FA_ERR_INVALID;
+  if (!std::isfinite(scale) || scale <= 0.f) return FA_ERR_INVALID;
+  if (dtype != FA_FP32 && dtype != FA_BF16 && dtype != FA_FP16) return FA_ERR_INVALID;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return FA_ERR_UNSUPPORTED;
+  if (int64_t(B) * H > (int64_t(1) << 31) - 1) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+int bwd_pad_rows(int Nq) { return int(round_up(size_t(Nq), 128)); }
+
+int effective_dq_mode(int B, int H, int Nq, int Nk, int d) {
+  if (g_dq_mode != 0) return g_dq_mode;
+  (void)B; (void)H; (void)Nq; (void)Nk; (void)d;
+  return 1;  // reduce-add: measured faster (partials cost nkv× the dQ traffic)
+}
+
+struct BwdWorkspace {
+  size_t d_off, dq_off, total;
+};
+
+BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
+  const size_t BH = size_t(B) * H;
+  const size_t rows = size_t(bwd_pad_rows(Nq));
+  const size_t nkv = (size_t(Nk) + 127) / 128;
+  BwdWorkspace w;
+  w.d_off = 0;
+  w.dq_off = round_up(BH * rows * sizeof(float), 256);
+  const size_t dq = BH * rows * size_t(d) * sizeof(float) * (mode == 2 ? nkv : 1);
+  w.total = w.dq_off + round_up(dq, 256);
+  return w;
+}
+
+int decode_auto_splits(int BH, int Nk) {
+  // Enough CTAs for many waves over 148 SMs (so the ragged last wave costs
+  // little), but parts of at least 256 keys.
+  const int target = 148 * 8 * 16;
+  int s = (target + BH - 1) / BH;
+  s = std::max(1, std::min(s, 128));
+  const int max_by_len = std::max(1, Nk / 256);
+  return std::min(s, max_by_len);
+}
+
+int decode_keys_per_split(int Nk, int splits) {
+  int kps = (Nk + splits - 1) / splits;
+  return int(round_up(size_t(kps), 64));
+}
+
+}  // namespace
+
+cudaError_t set_smem_once(const void* kernel, int bytes) {
+  static std::mutex mu;
+  static int done_n[kMaxDevices] = {0};
+  static const void* done_k[kMaxDevices][64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lk(mu);
+  const bool track = dev >= 0 && dev < kMaxDevices;
+  if (track)
+    for (int i = 0; i < done_n[dev]; ++i)
+      if (done_k[dev][i] == kernel) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && track && done_n[dev] < 64) done_k[dev][done_n[dev]++] = kernel;
+  return e;
+}
+
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
+           int Nk, int d, int causal, float scale, int dtype, void* stream) {
+  int st = check_common(B, H, Nq, Nk, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L))
+    return FA_ERR_INVALID;
+  if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
+  if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
+  const int BH = B * H;
+  FwdLaunch a;
+  std::memset(&a, 0, sizeof(a));
+  if (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, 128) || !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) ||
+      !make_map(&a.tmV, V, dtype, d, Nk, BH, 128))
+    return FA_ERR_CUDA;
+  a.params.Q = Q;
+  a.params.K = K;
+  a.params.V = V;
+  a.params.O = O;
+  a.params.L = L;
+  a.params.B = B;
+  a.params.H = H;
+  a.params.Nq = Nq;
+  a.params.Nk = Nk;
+  a.params.scale_log2 = scale * 1.4426950408889634f;
+  a.params.n_qblocks = (Nq + 255) / 256;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_fwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
+  if (check_common(B, H, Nq, Nk, d, 1.0f, dtype) != FA_OK) return 0;
+  return bwd_layout(B, H, Nq, Nk, d, effective_dq_mode(B, H, Nq, Nk, d)).total;
+}
+
+int fa_set_bwd_dq_mode(int mode) {
+  if (mode < 0 || mode > 2) return FA_ERR_INVALID;
+  const int prev = g_dq_mode;
+  g_dq_mode = mode;
+  return prev;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+           const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
+           int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  int st = check_common(B, H, Nq, Nk, d, scale, dtype);
+  if (st != FA_OK) return st;
+  const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return FA_ERR_INVALID;
+  if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
+  if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
+  const int mode = effective_dq_mode(B, H, Nq, Nk, d);
+  const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
+    return FA_ERR_WORKSPACE;
+  const int BH = B * H;
+  BwdLaunch a;
+  std::memset(&a, 0, sizeof(a));
+  if (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, 64) || !make_map(&a.tmdO, dO, dtype, d, Nq, BH, 64) ||
+      !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128))
+    return FA_ERR_CUDA;
+  BwdParams& p = a.params;
+  p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;
+  p.dQ = dQ; p.dK = dK; p.dV = dV;
+  p.Dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
+  p.dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dq_off);
+  p.B = B; p.H = H; p.Nq = Nq; p.Nk = Nk;
+  p.Nq_pad = bwd_pad_rows(Nq);
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_kblocks = (Nk + 127) / 128;
+  p.dq_mode = mode;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return launch_bwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {
+  if (B <= 0 || H <= 0 || Nk <= 0 || (d != 64 && d != 128) || num_splits < 0) return 0;
+  const int BH = B * H;
+  int s = num_splits > 0 ? num_splits : decode_auto_splits(BH, Nk);
+  s = std::min(s, Nk);
+  const int kps = decode_keys_per_split(Nk, s);
+  s = (Nk + kps - 1) / kps;
+  return round_up(size_t(BH) * s * d * sizeof(float), 256) + round_up(size_t(BH) * s * 4, 256);
+}
+
+int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nk,
+              int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
+              void* stream) {
+  int st = check_common(B, H, 1, Nk, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (num_splits < 0) return FA_ERR_INVALID;
+  const void* ptrs[] = {Q, K, V, O, L};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return FA_ERR_INVALID;
+  const int BH = B * H;
+  int s = num_splits > 0 ? num_splits : decode_auto_splits(BH, Nk);
+  s = std::min(s, Nk);
+  if (s > 65535) return FA_ERR_UNSUPPORTED;
+  const int kps = decode_keys_per_split(Nk, s);
+  s = (Nk + kps - 1) / kps;
+  const size_t need = fa_decode_workspace_bytes(B, H, Nk, d, num_splits);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < need)
+    return FA_ERR_WORKSPACE;
+  DecodeParams p;
+  p.Q = Q; p.K = K; p.V = V; p.O = O; p.L = L;
+  p.Opart = static_cast<float*>(workspace);
+  p.Lpart = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                     round_up(size_t(BH) * s * d * sizeof(float), 256));
+  p.BH = BH;
+  p.Nk = Nk;
+  p.splits = s;
+  p.keys_per_split = kps;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
+int fa_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  int word = 0;
+  if (take_error_fwd(&word) != cudaSuccess) return FA_ERR_CUDA;
+  if (take_error_bwd(&word) != cudaSuccess) return FA_ERR_CUDA;
+  if (take_error_decode(&word) != cudaSuccess) return FA_ERR_CUDA;
+  if (word != 0) return FA_ERR_TIMEOUT;
+  return FA_OK;
+}
+
+const char* fa_version(void) { return "fa-b200 0.1 (sm_100a)"; }
+
+}  // extern "C"

@@ -1,0 +1,515 @@
+// Forward attention kernel for sm_100a.
+//
+// FlashAttention1 post (CSDN), section "具体算法", and the FlashAttention
+// V1/V2 study notes (51CTO), sections "Thread Block Level 并行" and "算法的改进":
+// the query rows are cut into tiles, one group of tiles per CTA; the K/V
+// sequence streams through shared memory tile by tile; each row keeps a
+// running maximum m, a running denominator ℓ and an unnormalised output
+// accumulator that is rescaled when m grows; O and the row logsumexp L are
+// written once at the end.  Causal: K/V tiles wholly above the diagonal are
+// never loaded, and only tiles that cross the diagonal (or the ragged end of
+// K) are masked.  The notes' instruction-level section: the softmax uses
+// exp2 with scale·log2(e) folded into one FFMA per score.
+//
+// B200 design (not the pages'): one CTA owns two 128-row Q tiles and
+// ping-pongs them so the tensor core works on one tile while the softmax
+// warps work on the other.  Roles per CTA (384 threads, 3 warpgroups):
+//   warpgroup 0 (warps 0-3)  softmax + correction + epilogue, Q tile 0
+//                            (thread = row), 200 registers
+//   warpgroup 1 (warps 4-7)  the same for Q tile 1, 200 registers
+//   warpgroup 2: warp 8 tcgen05.mma issuer (one thread) and TMEM owner,
+//                warp 9 TMA producer, warps 10-11 idle; 80 registers
+// TMEM (512 columns): S0 | S1 | O0 | O1.  P overwrites S in place (bf16 pairs
+// or tf32) and is read by the P·V MMA straight from TMEM.  The running max is
+// only moved when it grows by more than kRescaleThreshold (log2 units), so
+// the O accumulator is rescaled rarely; the result is exact either way
+// because O and ℓ always share the same reference maximum.
+#include "common.cuh"
+#include "launch.h"
+
+namespace fa {
+
+namespace {
+
+#ifndef FA_RESCALE_THRESHOLD
+#define FA_RESCALE_THRESHOLD 8.0f
+#endif
+constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entries stay <= 2^8
+
+template <typename T, int D>
+struct FwdTraits {
+  static constexpr int ES = sizeof(T);
+  static constexpr int BN = 128;                 // keys of a K/V tile
+  static constexpr int AW = 128 / ES;            // elements per 128-byte swizzled row
+  static constexpr int DC = D / AW;              // 128-byte column blocks in a row
+  static constexpr int CHUNK = 128 * 128;        // bytes of one column block (128 rows)
+  static constexpr int TILE = 128 * D * ES;      // bytes of one 128-row tile
+  static constexpr int KSTEP = 32 / ES;          // K extent of one MMA instruction
+  static constexpr int NS_RAW = (200 * 1024 - 2 * TILE) / TILE;
+  static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
+  static constexpr int SMEM_BAR = 2 * TILE + NS * TILE;
+  static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers + alignment slack
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_SOFTMAX = 200;  // per thread, warpgroups 0-1
+  static constexpr int REGS_OTHER = 80;     // per thread, warpgroup 2
+  static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
+  static constexpr uint32_t IDESC_PV =
+      make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
+  static_assert(NS >= 2, "need at least two K/V slots");
+  static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
+};
+
+struct FwdBarriers {
+  uint64_t q_full[2];
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full[2];
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ float round_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+
+// fp32 inputs (TF32 tensor-core products).  The tensor core reads only the
+// top 19 bits of each fp32 operand, i.e. it truncates; to keep the products
+// unbiased every operand is rounded to nearest TF32 first, so the producer
+// warp stages fp32 tiles itself instead of with TMA.  Rows past N are zero.
+//
+// K-major copy of rows [row0, row0+128) of a [N, D] fp32 matrix: row r,
+// element n at column block n/32 (blocks 128*128 bytes apart), 128-byte
+// swizzled rows.
+template <int D>
+__device__ __forceinline__ void stage_rows_tf32(const float* X, int bh, int N, int row0,
+                                                uint8_t* dst, int lane) {
+  const float* Xh = X + size_t(bh) * N * D;
+  for (int idx = lane; idx < 128 * (D / 4); idx += 32) {
+    const int r = idx / (D / 4), n4 = (idx % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row0 + r < N) v = *reinterpret_cast<const float4*>(Xh + size_t(row0 + r) * D + n4);
+    v = make_float4(round_tf32(v.x), round_tf32(v.y), round_tf32(v.z), round_tf32(v.w));
+    const uint32_t byte = (n4 & 31) * 4;
+    const uint32_t o = (n4 >> 5) * (128 * 128) + r * 128 + (((byte >> 4) ^ (r & 7)) << 4);
+    *reinterpret_cast<float4*>(dst + o) = v;
+  }
+}
+
+// V transposed for the P·V product: row n = d index, the 128 keys along the
+// row (32 keys per 128-byte column block, blocks D*128 bytes apart).
+template <int D>
+__device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, int Nk, int key0,
+                                                        uint8_t* dst, int lane) {
+  const float* Vh = V + size_t(bh) * Nk * D;
+  for (int idx = lane; idx < 128 * (D / 4); idx += 32) {
+    const int kk = idx / (D / 4), n4 = (idx % (D / 4)) * 4;
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (key0 + kk < Nk) v = *reinterpret_cast<const float4*>(Vh + size_t(key0 + kk) * D + n4);
+    const float vals[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const int n = n4 + e;
+      const uint32_t byte = (kk & 31) * 4;
+      const uint32_t o = (kk >> 5) * (D * 128) + n * 128 + ((((byte >> 4) ^ (n & 7)) << 4) | (byte & 15));
+      *reinterpret_cast<float*>(dst + o) = round_tf32(vals[e]);
+    }
+  }
+}
+
+template <typename T, int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+               const __grid_constant__ CUtensorMap tmV, FwdParams p) {
+  using Tr = FwdTraits<T, D>;
+  constexpr bool TF32 = ElemTraits<T>::tf32;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + Tr::SMEM_BAR);
+  volatile int* abort_flag = &bars->abort_flag;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  const int n_qb = p.n_qblocks;
+  const int qb = CAUSAL ? (n_qb - 1 - int(blockIdx.x)) : int(blockIdx.x);  // heavy blocks first
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int q_row0 = qb * 256;
+  const int off = p.Nk - p.Nq;  // bottom-right causal alignment
+
+  int kv_end = p.Nk;
+  if (CAUSAL) {
+    const int q_last = min(q_row0 + 255, p.Nq - 1);
+    kv_end = min(p.Nk, q_last + off + 1);
+  }
+  const int n_kv = (kv_end + Tr::BN - 1) / Tr::BN;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&bars->q_full[i], 1);
+      mbar_init(&bars->s_full[i], 1);
+      mbar_init(&bars->p_full[i], 128);
+      mbar_init(&bars->o_full[i], 1);
+    }
+    for (int i = 0; i < Tr::NS; ++i) {
+      mbar_init(&bars->kv_full[i], 1);
+      mbar_init(&bars->kv_empty[i], 1);
+    }
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  uint8_t* sQ[2] = {smem, smem + Tr::TILE};
+  uint8_t* sKV = smem + 2 * Tr::TILE;
+
+  if (warp >= 10) {
+    // idle warps of the producer/MMA warpgroup
+    regs_dec<Tr::REGS_OTHER>();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    regs_dec<Tr::REGS_OTHER>();
+    // Lane 0 issues the TMA loads (16-bit types).  fp32 tiles are staged by
+    // the whole warp instead (see stage_rows_tf32).
+    auto load_tile = [&](int which, uint8_t* dst, uint64_t* bar, int row) {
+      // which: 0 = Q, 1 = K, 2 = V
+      if constexpr (TF32) {
+        const float* src = reinterpret_cast<const float*>(which == 0 ? p.Q : which == 1 ? p.K : p.V);
+        if (which == 2)
+          stage_v_transposed_tf32<D>(src, bh, p.Nk, row, dst, lane);
+        else
+          stage_rows_tf32<D>(src, bh, which == 0 ? p.Nq : p.Nk, row, dst, lane);
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar);
+      } else if (lane == 0) {
+        const CUtensorMap* map = which == 0 ? &tmQ : which == 1 ? &tmK : &tmV;
+        mbar_arrive_expect_tx(bar, Tr::TILE);
+#pragma unroll
+        for (int c = 0; c < Tr::DC; ++c)
+          tma_load_3d(dst + c * Tr::CHUNK, map, bar, c * Tr::AW, row, bh);
+      }
+    };
+    auto load_kv = [&](int i) {  // i-th K/V tile in consumption order: K0 V0 K1 V1 ...
+      const int slot = i % Tr::NS;
+      bool ok = true;
+      if (i >= Tr::NS)
+        ok = mbar_wait(&bars->kv_empty[slot], ((i / Tr::NS) - 1) & 1, abort_flag);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) return false;
+      load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
+      return true;
+    };
+    load_tile(0, sQ[0], &bars->q_full[0], q_row0);
+    load_kv(0);
+    load_tile(0, sQ[1], &bars->q_full[1], q_row0 + 128);
+    for (int i = 1; i < 2 * n_kv; ++i)
+      if (!load_kv(i)) break;
+    if (lane == 0) {
+      // Drain: wait until every issued load has landed before the CTA may exit.
+      for (int i = max(0, 2 * n_kv - Tr::NS); i < 2 * n_kv; ++i)
+        mbar_wait(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
+      mbar_wait(&bars->q_full[0], 0, abort_flag);
+      mbar_wait(&bars->q_full[1], 0, abort_flag);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<Tr::REGS_OTHER>();
+    if (lane == 0) {
+      const uint32_t tS[2] = {tmem, tmem + 128};
+      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
+      const uint32_t aKV = smem_u32(sKV);
+
+      auto issue_qk = [&](int t, int slot) {
+        const uint32_t kb = aKV + slot * Tr::TILE;
+#pragma unroll
+        for (int ks = 0; ks < D / Tr::KSTEP; ++ks) {
+          const uint32_t o = (ks >> 2) * Tr::CHUNK + (ks & 3) * 32;
+          mma_ss<TF32>(tS[t], sw128_desc(aQ[t] + o, 16, 1024), sw128_desc(kb + o, 16, 1024),
+                       Tr::IDESC_QK, ks > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int slot, bool acc) {
+        const uint32_t vb = aKV + slot * Tr::TILE;
+#pragma unroll
+        for (int ks = 0; ks < Tr::BN / Tr::KSTEP; ++ks) {
+          // 16-bit: V tile [key][d] is an MN-major B operand; step = KSTEP key rows.
+          // TF32: V tile was stored transposed ([d][key], K-major); step = 32 bytes.
+          const uint64_t bdesc =
+              TF32 ? sw128_desc(vb + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024)
+                   : sw128_desc(vb + ks * Tr::KSTEP * 128, Tr::CHUNK, 1024);
+          mma_ts<TF32>(tO[t], tS[t] + ks * 8, bdesc, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
+        }
+      };
+      auto kv_wait = [&](int i) {
+        return mbar_wait(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
+      };
+
+      bool ok = mbar_wait(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+      tc_fence_after();
+      if (ok) issue_qk(0, 0);
+      tc_commit(&bars->s_full[0]);
+      ok = ok && mbar_wait(&bars->q_full[1], 0, abort_flag);
+      tc_fence_after();
+      if (ok) issue_qk(1, 0);
+      tc_commit(&bars->s_full[1]);
+      tc_commit(&bars->kv_empty[0]);
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int iv = 2 * j + 1, ik = 2 * j + 2;
+        const int sv = iv % Tr::NS, sk = ik % Tr::NS;
+        ok = kv_wait(iv) && mbar_wait(&bars->p_full[0], j & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        issue_pv(0, sv, j > 0);
+        tc_commit(&bars->o_full[0]);
+        const bool more = j + 1 < n_kv;
+        if (more) {
+          ok = kv_wait(ik);
+          tc_fence_after();
+          if (!ok) break;
+          issue_qk(0, sk);
+          tc_commit(&bars->s_full[0]);
+        }
+        ok = mbar_wait(&bars->p_full[1], j & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        issue_pv(1, sv, j > 0);
+        tc_commit(&bars->o_full[1]);
+        tc_commit(&bars->kv_empty[sv]);
+        if (more) {
+          issue_qk(1, sk);
+          tc_commit(&bars->s_full[1]);
+          tc_commit(&bars->kv_empty[sk]);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    regs_inc<Tr::REGS_SOFTMAX>();
+    const int t = warp >> 2;         // which Q tile
+    const int quad = warp & 3;       // TMEM lane quadrant of this warp
+    const int r = quad * 32 + lane;  // row in the tile = TMEM lane
+    const int qi = q_row0 + t * 128 + r;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tS = tmem + lane_off + t * 128;
+    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const float sl2 = p.scale_log2;
+    const int tile_first_row = q_row0 + t * 128;
+
+    float m_ref = -INFINITY;  // reference maximum, scaled log2 units
+    float row_sum = 0.f;      // Σ exp2 of the scores: gives the logsumexp L
+    float row_sum_p = 0.f;    // Σ of P as rounded for the P·V product: normalises O
+    bool ok = true;
+
+    for (int j = 0; j < n_kv; ++j) {
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, abort_flag));
+      tc_fence_after();
+      if (!ok) break;
+      float s[Tr::BN];
+#pragma unroll
+      for (int c = 0; c < Tr::BN; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tS + c, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(u[e]);
+      }
+      const int k0 = j * Tr::BN;
+      const bool tail = k0 + Tr::BN > p.Nk;
+      const bool diag = CAUSAL && (k0 + Tr::BN - 1 > tile_first_row + off);
+      if (tail || diag) {
+        int lim = p.Nk - k0;
+        if (CAUSAL) lim = min(lim, qi + off + 1 - k0);
+#pragma unroll
+        for (int c = 0; c < Tr::BN; ++c)
+          if (c >= lim) s[c] = -INFINITY;
+      }
+      float mx = fmax3(s[0], s[1], s[2]);
+#pragma unroll
+      for (int c = 3; c + 1 < Tr::BN; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
+      if constexpr ((Tr::BN - 3) % 2 == 1) mx = fmaxf(mx, s[Tr::BN - 1]);
+      const float m_tile = mx * sl2;
+      const bool upd = m_tile > m_ref + kRescaleThreshold;
+      float alpha = 1.f;
+      if (upd) {
+        alpha = ex2(m_ref - m_tile);  // 0 when m_ref is -inf
+        row_sum *= alpha;
+        row_sum_p *= alpha;
+        m_ref = m_tile;
+      }
+      if (j > 0 && __any_sync(0xffffffffu, upd)) {
+        // Correction: O (which holds tiles < j) moves onto the new maximum.
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], (j - 1) & 1, abort_flag));
+        tc_fence_after();
+        if (!ok) break;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tO + c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+          tmem_st32(tO + c, u);
+        }
+      }
+      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+      const uint64_t c2 = pk2(sl2, sl2), negm2 = pk2(-m_use, -m_use);
+      uint64_t sum2 = pk2(0.f, 0.f), sum2_p = pk2(0.f, 0.f);
+      if constexpr (TF32) {
+#pragma unroll
+        for (int c = 0; c < Tr::BN; c += 32) {
+          uint32_t u[32];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 x = upk2(ffma2(pk2(s[c + e], s[c + e + 1]), c2, negm2));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
+            const float r0 = round_tf32(p0), r1 = round_tf32(p1);
+            sum2 = fadd2(sum2, pk2(p0, p1));
+            sum2_p = fadd2(sum2_p, pk2(r0, r1));
+            u[e] = __float_as_uint(r0);
+            u[e + 1] = __float_as_uint(r1);
+          }
+          tmem_st32(tS + c, u);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < Tr::BN; c += 64) {
+          uint32_t u[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float2 x = upk2(ffma2(pk2(s[c + 2 * e], s[c + 2 * e + 1]), c2, negm2));
+            const float p0 = ex2(x.x), p1 = ex2(x.y);
+            u[e] = ElemTraits<T>::pack2(p0, p1);
+            // O is normalised by the sum of the same rounded P the P·V
+            // product uses, so a row's weights add up to one exactly; L keeps
+            // the unrounded sum (the exact logsumexp).
+            const float2 pr = ElemTraits<T>::unpack2(u[e]);
+            sum2 = fadd2(sum2, pk2(p0, p1));
+            sum2_p = fadd2(sum2_p, pk2(pr.x, pr.y));
+          }
+          tmem_st32(tS + c / 2, u);
+        }
+      }
+      {
+        const float2 a = upk2(sum2), b = upk2(sum2_p);
+        row_sum += a.x + a.y;
+        row_sum_p += b.x + b.y;
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_full[t]);
+    }
+
+    // ------------------------------------------------------------ epilogue
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
+    tc_fence_after();
+    if (ok) {
+      const float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;
+      const bool live = qi < p.Nq;
+      T* orow = reinterpret_cast<T*>(p.O) + (size_t(bh) * p.Nq + (live ? qi : 0)) * D;
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tO + c, u);
+        tmem_ld_wait();
+        if (live) {
+          if constexpr (TF32) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float4 v = make_float4(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv,
+                                     __uint_as_float(u[e + 2]) * inv,
+                                     __uint_as_float(u[e + 3]) * inv);
+              *reinterpret_cast<float4*>(orow + c + e) = v;
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv);
+              v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]) * inv,
+                                         __uint_as_float(u[e + 3]) * inv);
+              v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]) * inv,
+                                         __uint_as_float(u[e + 5]) * inv);
+              v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]) * inv,
+                                         __uint_as_float(u[e + 7]) * inv);
+              *reinterpret_cast<uint4*>(orow + c + e) = v;
+            }
+          }
+        }
+      }
+      if (live)
+        p.L[size_t(bh) * p.Nq + qi] =
+            row_sum > 0.f ? (m_ref + lg2(row_sum)) * kLn2 : -INFINITY;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace
+
+template <typename T, int D, bool CAUSAL>
+static cudaError_t launch_fwd_t(const FwdLaunch& a) {
+  using Tr = FwdTraits<T, D>;
+  auto kern = fwd_kernel<T, D, CAUSAL>;
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  // setmaxnreg redistributes the registers the CTA was launched with; refuse
+  // to launch if the compiled register count cannot cover the split.
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
+    if (e != cudaSuccess) return e;
+    regs_ok = attr.numRegs * Tr::THREADS >= 256 * Tr::REGS_SOFTMAX + 128 * Tr::REGS_OTHER;
+  }
+  if (!regs_ok) return cudaErrorInvalidConfiguration;
+  dim3 grid(a.params.n_qblocks, a.params.H, a.params.B);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.params);
+  return cudaGetLastError();
+}
+
+int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
+
+cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
+#define FA_FWD_CASE(TY, DD)                                                      \
+  return causal ? launch_fwd_t<TY, DD, true>(a) : launch_fwd_t<TY, DD, false>(a);
+  if (dtype == FA_BF16) {
+    if (d == 64) FA_FWD_CASE(__nv_bfloat16, 64)
+    if (d == 128) FA_FWD_CASE(__nv_bfloat16, 128)
+  } else if (dtype == FA_FP16) {
+    if (d == 64) FA_FWD_CASE(__half, 64)
+    if (d == 128) FA_FWD_CASE(__half, 128)
+  } else if (dtype == FA_FP32) {
+    if (d == 64) FA_FWD_CASE(float, 64)
+  }
+#undef FA_FWD_CASE
+  return cudaErrorInvalidValue;
+}
+
+FA_ERROR_ACCESSOR(take_error_fwd)
+
+}  // namespace fa

@@ -1,0 +1,80 @@
+// Host-side launch interface between the C ABI (api.cu) and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fa {
+
+struct FwdParams {
+  const void* Q;  // raw inputs (read directly only by the fp32 path)
+  const void* K;
+  const void* V;
+  void* O;
+  float* L;
+  int B, H, Nq, Nk;
+  float scale_log2;  // scale * log2(e)
+  int n_qblocks;     // ceil(Nq / 256): one CTA per 256 query rows
+};
+
+struct FwdLaunch {
+  CUtensorMap tmQ, tmK, tmV;
+  FwdParams params;
+  cudaStream_t stream;
+};
+
+// Elements in one 128-byte swizzled row for the dtype (the TMA box width).
+int fwd_tile_elems(int dtype);
+cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a);
+
+struct BwdParams {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const void* O;
+  const void* dO;
+  const float* L;
+  void* dQ;
+  void* dK;
+  void* dV;
+  float* Dsum;    // [B*H, Nq_pad] rowsum(dO * O), padded rows zero
+  float* dQacc;   // [B*H, Nq_pad, d] fp32 (mode 1) or [nkv, B*H, Nq_pad, d] (mode 2)
+  int B, H, Nq, Nk, Nq_pad;
+  float scale;        // softmax scale
+  float scale_log2;   // scale * log2(e)
+  int n_kblocks;      // ceil(Nk / 128)
+  int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials
+};
+
+struct BwdLaunch {
+  CUtensorMap tmQ, tmK, tmV, tmdO;
+  BwdParams params;
+  cudaStream_t stream;
+};
+
+cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a);
+
+struct DecodeParams {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  float* L;
+  float* Opart;  // [B*H, S, d] normalised partial outputs
+  float* Lpart;  // [B*H, S] natural-log logsumexp of each part (-inf if empty)
+  int BH, Nk, splits, keys_per_split;
+  float scale_log2;
+};
+
+cudaError_t launch_decode(int dtype, int d, const DecodeParams& p, cudaStream_t s);
+
+// Read-and-clear accessors of each kernel file's device error word.
+cudaError_t take_error_fwd(int* word);
+cudaError_t take_error_bwd(int* word);
+cudaError_t take_error_decode(int* word);
+
+// Sets the dynamic shared-memory limit of `kernel` on the current device once.
+cudaError_t set_smem_once(const void* kernel, int bytes);
+
+}  // namespace fa

@@ -1,0 +1,115 @@
+/*
+ * fa.h — C ABI of the B200 (sm_100a) fused exact-attention library.
+ *
+ * The library computes exact scaled-dot-product attention
+ *     O = softmax(scale · Q Kᵀ [+ causal mask]) V
+ * fused into tiled kernels with an online softmax, and its gradient.
+ *
+ *   FlashAttention1 post (CSDN), section "具体算法": S = Q Kᵀ, P = softmax(S),
+ *     O = P V, computed block by block with a running row maximum and a
+ *     running denominator so that S and P never reach device memory.
+ *   FlashAttention V1/V2 study notes (51CTO), section "算法的改进": the
+ *     forward writes the row logsumexp L once; the backward rebuilds P from
+ *     L instead of storing it.  Causal: blocks wholly above the diagonal are
+ *     skipped, only the diagonal block is masked.
+ *   Same notes, section "Sequence Parallel": the backward runs one K/V block
+ *     per CTA and reduces dQ across CTAs; Flash-Decoding splits K/V of a
+ *     single query across CTAs and combines the parts by their logsumexp.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor arguments are DEVICE pointers to contiguous row-major arrays
+ *    allocated and owned by the caller.  The library never allocates device
+ *    memory on these paths and never synchronises (except fa_status).
+ *  - Q, O, dO, dQ: [B, H, Nq, d];  K, V, dK, dV: [B, H, Nk, d];  L, D: [B, H, Nq]
+ *    (d fastest).  Element type of Q/K/V/O/dO/dQ/dK/dV is `dtype`; L is
+ *    always float32 and holds the NATURAL-log logsumexp of the scaled,
+ *    masked scores of each query row.
+ *  - Every pointer must be 16-byte aligned.
+ *  - causal != 0 uses bottom-right alignment: key j is visible to query i iff
+ *    j <= i + (Nk - Nq).  Causal requires Nq <= Nk, so no row is empty.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Work is
+ *    enqueued on it and the call returns without waiting.
+ *  - Supported: d in {64, 128}; dtype FA_BF16 or FA_FP16 for every d, FA_FP32
+ *    (computed with TF32 tensor-core products and fp32 softmax) for d = 64.
+ *  - Return value: FA_OK, or a negative fa_status_t detected synchronously
+ *    before anything is enqueued (invalid arguments, unsupported shape,
+ *    workspace too small) or at launch (FA_ERR_CUDA).  Faults and bounded-
+ *    wait timeouts inside kernels are reported later by fa_status().
+ */
+#ifndef FA_B200_H_
+#define FA_B200_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FA_FP32 = 0, FA_BF16 = 1, FA_FP16 = 2 } fa_dtype;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID = -1,     /* null pointer, size <= 0, non-finite scale, misaligned pointer */
+  FA_ERR_UNSUPPORTED = -2, /* d not in {64,128}, fp32 with d=128, causal with Nq > Nk */
+  FA_ERR_WORKSPACE = -3,   /* workspace pointer null or smaller than the query says */
+  FA_ERR_CUDA = -4,        /* a CUDA runtime error at launch or in fa_status */
+  FA_ERR_TIMEOUT = -5      /* a kernel's bounded wait expired (reported by fa_status) */
+} fa_status_t;
+
+/* Forward.  Writes O [B,H,Nq,d] (dtype) and L [B,H,Nq] (float32, natural
+ * log).  FlashAttention V1/V2 study notes (51CTO), sections "算法的改进" and
+ * "Thread Block Level 并行": one CTA per block of query rows, the K/V
+ * sequence streamed through shared memory, O and L written once. */
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
+           int Nk, int d, int causal, float scale, int dtype, void* stream);
+
+/* Bytes of device workspace fa_bwd needs for this problem (0 on invalid
+ * arguments).  The workspace holds D = rowsum(dO ∘ O) [B,H,Nq] and the fp32
+ * dQ accumulator; its contents on entry do not matter. */
+size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype);
+
+/* Backward.  Given the forward's inputs, its O and L, and dO, writes dQ, dK,
+ * dV (dtype, shapes of Q, K, V).  Recomputes P = exp(scale·S − L) block by
+ * block (the N×N matrix is never stored), D = rowsum(dO ∘ O) first.  The
+ * 51CTO notes, sections "算法的改进" and "Sequence Parallel".  `workspace`
+ * must hold fa_bwd_workspace_bytes(...) bytes, 256-byte aligned. */
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+           const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
+           int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* How fa_bwd reduces the dQ contributions of the different K/V blocks:
+ *   0 = automatic (the measured faster strategy for the shape),
+ *   1 = fp32 bulk reductions (red.add) into one accumulator,
+ *   2 = one fp32 partial buffer per K/V block, then a reduction kernel.
+ * The 51CTO notes, section "Sequence Parallel", describe both.  Returns the
+ * previous mode, or FA_ERR_INVALID for an unknown mode.  Process-wide. */
+int fa_set_bwd_dq_mode(int mode);
+
+/* Bytes of workspace fa_decode needs for `num_splits` parts (0 = the count
+ * fa_decode would choose itself). */
+size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits);
+
+/* Split-KV decode forward for one query row per (batch, head):
+ * Q [B,H,1,d], K,V [B,H,Nk,d] -> O [B,H,1,d] (dtype), L [B,H,1] (float32).
+ * No mask.  Each of `num_splits` parts (0 = automatic) runs the online
+ * softmax over its slice of K/V and writes a normalised partial output and
+ * its logsumexp; a combine kernel then rescales and adds them
+ * (the 51CTO notes, Flash-Decoding paragraph of "Sequence Parallel"). */
+int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nk,
+              int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
+              void* stream);
+
+/* Synchronises `stream`, then returns and clears the device error word:
+ * FA_OK, FA_ERR_TIMEOUT if a kernel's bounded wait expired, FA_ERR_CUDA if
+ * the stream reports a CUDA error. */
+int fa_status(void* stream);
+
+/* Library version string (static storage). */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H_ */

@@ -1,0 +1,56 @@
+"""Shared helpers for the GPU parity tests: tolerance checks against the
+fp64 oracle.  Tolerances (bf16/fp16 inputs, fp32 accumulation):
+O max-abs <= 1e-2 and mean-abs <= 1e-3; L max-abs <= 1e-3;
+dQ/dK/dV max-abs <= 2e-2 * max|grad_ref| (each).
+
+O is stored in the input dtype, and the final cast alone moves a value by
+up to half a unit in the last place of that dtype (0.0156 for bf16 values in
+[4, 8)), more than 1e-2 for any |O| > 2.56.  The element-wise O bound is
+therefore 1e-2 plus half an ulp of the output dtype at the reference value;
+the mean-abs bound and the L bound are applied as stated.  ``check_fwd``
+also returns the plain max-abs error so callers can report it."""
+import numpy as np
+import torch
+
+O_MAX, O_MEAN, L_MAX, G_REL = 1e-2, 1e-3, 1e-3, 2e-2
+
+
+def f64(t):
+    if isinstance(t, torch.Tensor):
+        return t.detach().float().cpu().double().numpy()
+    return np.asarray(t, dtype=np.float64)
+
+
+MANTISSA_BITS = {torch.bfloat16: 7, torch.float16: 10, torch.float32: 23}
+
+
+def half_ulp(x, dtype):
+    """Half a unit in the last place of ``dtype`` at |x| (normal range)."""
+    mb = MANTISSA_BITS[dtype]
+    ax = np.maximum(np.abs(x), 2.0 ** -14)
+    return np.ldexp(1.0, np.floor(np.log2(ax)).astype(int) - mb - 1)
+
+
+def check_fwd(O, L, O_ref, L_ref, what=""):
+    dtype = O.dtype if isinstance(O, torch.Tensor) else torch.float32
+    O, L = f64(O), f64(L)
+    assert np.all(np.isfinite(O)), f"{what}: non-finite O"
+    assert np.all(np.isfinite(L)), f"{what}: non-finite L"
+    e = np.abs(O - O_ref)
+    el = np.abs(L - L_ref)
+    bound = O_MAX + half_ulp(O_ref, dtype)
+    worst = np.argmax(e - bound)
+    assert np.all(e <= bound), (f"{what}: O error {e.flat[worst]:.3e} at ref {O_ref.flat[worst]:.4f} "
+                                f"exceeds 1e-2 + half-ulp; plain max-abs {e.max():.3e}")
+    assert e.mean() <= O_MEAN, f"{what}: O mean-abs {e.mean():.3e}"
+    assert el.max() <= L_MAX, f"{what}: L max-abs {el.max():.3e}"
+    return e.max(), e.mean(), el.max()
+
+
+def check_grad(G, G_ref, name, what="", scale_ref=None):
+    G = f64(G)
+    assert np.all(np.isfinite(G)), f"{what}: non-finite {name}"
+    ref_max = np.abs(G_ref).max() if scale_ref is None else scale_ref
+    e = np.abs(G - G_ref).max()
+    assert e <= G_REL * ref_max, f"{what}: {name} max-abs {e:.3e} > {G_REL} * {ref_max:.3e}"
+    return e / max(ref_max, 1e-30)

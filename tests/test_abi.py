@@ -1,0 +1,136 @@
+"""Host-side tests of the C ABI (no GPU needed): the library loads, exports
+every function include/fa.h declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_attention_115_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+FAKE = 0x10000  # a 16-byte aligned non-null value; never dereferenced on these paths
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from exact_attention_115_b200 import build
+    build.build()
+    return fa.lib()
+
+
+def test_exports_every_declared_symbol(lib):
+    names = declared_functions()
+    assert "fa_fwd" in names and "fa_bwd" in names and "fa_decode" in names
+    for n in names:
+        assert hasattr(lib, n), f"{n} not exported"
+        assert n in fa.SIGNATURES, f"{n} has no ctypes signature in the binding"
+
+
+def test_version(lib):
+    assert "sm_100a" in fa.version()
+
+
+def fwd(lib, **kw):
+    a = dict(Q=FAKE, K=FAKE, V=FAKE, O=FAKE, L=FAKE, B=1, H=1, Nq=128, Nk=128, d=64, causal=0,
+             scale=0.125, dtype=fa.FA_BF16, stream=None)
+    a.update(kw)
+    return lib.fa_fwd(a["Q"], a["K"], a["V"], a["O"], a["L"], a["B"], a["H"], a["Nq"], a["Nk"],
+                      a["d"], a["causal"], a["scale"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Q=None), fa.FA_ERR_INVALID),
+    (dict(L=None), fa.FA_ERR_INVALID),
+    (dict(K=FAKE + 2), fa.FA_ERR_INVALID),
+    (dict(B=0), fa.FA_ERR_INVALID),
+    (dict(Nq=0), fa.FA_ERR_INVALID),
+    (dict(Nk=-1), fa.FA_ERR_INVALID),
+    (dict(scale=float("nan")), fa.FA_ERR_INVALID),
+    (dict(scale=float("inf")), fa.FA_ERR_INVALID),
+    (dict(scale=0.0), fa.FA_ERR_INVALID),
+    (dict(dtype=7), fa.FA_ERR_INVALID),
+    (dict(d=96), fa.FA_ERR_UNSUPPORTED),
+    (dict(d=256), fa.FA_ERR_UNSUPPORTED),
+    (dict(dtype=fa.FA_FP32, d=128), fa.FA_ERR_UNSUPPORTED),
+    (dict(causal=1, Nq=200, Nk=100), fa.FA_ERR_UNSUPPORTED),
+    (dict(H=70000), fa.FA_ERR_UNSUPPORTED),
+])
+def test_fwd_rejects(lib, kw, code):
+    assert fwd(lib, **kw) == code
+
+
+def test_bwd_workspace_query(lib):
+    n = lib.fa_bwd_workspace_bytes(2, 3, 100, 200, 64, fa.FA_BF16)
+    # D (fp32 per padded row) + fp32 dQ accumulator (padded rows × d), 256-aligned pieces
+    rows = 128
+    assert n >= 2 * 3 * rows * 4 + 2 * 3 * rows * 64 * 4
+    assert lib.fa_bwd_workspace_bytes(0, 3, 100, 200, 64, fa.FA_BF16) == 0
+    assert lib.fa_bwd_workspace_bytes(1, 1, 100, 200, 96, fa.FA_BF16) == 0
+
+
+def test_bwd_dq_modes_change_workspace(lib):
+    prev = lib.fa_set_bwd_dq_mode(2)
+    try:
+        n2 = lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16)
+        lib.fa_set_bwd_dq_mode(1)
+        n1 = lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16)
+        assert n2 > n1 * 4  # 8 K/V blocks of partial buffers vs one accumulator
+        assert lib.fa_set_bwd_dq_mode(3) == fa.FA_ERR_INVALID
+        assert lib.fa_set_bwd_dq_mode(-1) == fa.FA_ERR_INVALID
+    finally:
+        lib.fa_set_bwd_dq_mode(prev)
+
+
+def bwd(lib, ws=FAKE, ws_bytes=1 << 40, **kw):
+    a = dict(B=1, H=1, Nq=128, Nk=128, d=64, causal=0, scale=0.125, dtype=fa.FA_BF16)
+    a.update(kw)
+    return lib.fa_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, a["B"], a["H"],
+                      a["Nq"], a["Nk"], a["d"], a["causal"], a["scale"], a["dtype"], ws, ws_bytes,
+                      None)
+
+
+def test_bwd_rejects(lib):
+    assert bwd(lib, d=80) == fa.FA_ERR_UNSUPPORTED
+    assert bwd(lib, Nq=0) == fa.FA_ERR_INVALID
+    assert bwd(lib, causal=1, Nq=256, Nk=128) == fa.FA_ERR_UNSUPPORTED
+    assert bwd(lib, ws=None) == fa.FA_ERR_WORKSPACE
+    assert bwd(lib, ws=FAKE + 16) == fa.FA_ERR_WORKSPACE  # not 256-aligned
+    need = lib.fa_bwd_workspace_bytes(1, 1, 128, 128, 64, fa.FA_BF16)
+    assert bwd(lib, ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+
+
+def test_decode_rejects(lib):
+    def dec(ws=FAKE, ws_bytes=1 << 40, **kw):
+        a = dict(B=2, H=2, Nk=1000, d=128, scale=0.1, dtype=fa.FA_BF16, splits=0)
+        a.update(kw)
+        return lib.fa_decode(FAKE, FAKE, FAKE, FAKE, FAKE, a["B"], a["H"], a["Nk"], a["d"],
+                             a["scale"], a["dtype"], a["splits"], ws, ws_bytes, None)
+    assert dec(Nk=0) == fa.FA_ERR_INVALID
+    assert dec(d=32) == fa.FA_ERR_UNSUPPORTED
+    assert dec(dtype=fa.FA_FP32) == fa.FA_ERR_UNSUPPORTED
+    assert dec(splits=-2) == fa.FA_ERR_INVALID
+    assert dec(ws=None) == fa.FA_ERR_WORKSPACE
+    need = lib.fa_decode_workspace_bytes(2, 2, 1000, 128, 0)
+    assert need > 0
+    assert dec(ws_bytes=need - 1) == fa.FA_ERR_WORKSPACE
+    # explicit split counts are clamped to the number of keys
+    assert lib.fa_decode_workspace_bytes(1, 1, 5, 64, 100) <= lib.fa_decode_workspace_bytes(1, 1, 5000, 64, 100)
+
+
+def test_python_binding_refuses_cpu_tensors(lib):
+    import torch
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)
+    with pytest.raises(ValueError):
+        fa.decode(q[:, :, :1], q, q)

@@ -1,0 +1,113 @@
+"""GPU parity of the forward kernel against the fp64 oracle (call path:
+Python binding -> fa_fwd C ABI -> sm_100a kernel)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from tests._parity import check_fwd, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def fa():
+    import exact_attention_115_b200 as fa
+    fa.lib()
+    return fa
+
+
+def run_full(fa, B, H, Nq, Nk, d, causal, dtype="bf16", seed=0, q_mult=1.0):
+    q, k, v, _ = W.make_tensors(B, H, Nq, Nk, d, dtype, seed=seed, q_mult=q_mult,
+                                device="cuda", with_grad=False)
+    scale = 1 / math.sqrt(d)
+    O, L = fa.forward(q, k, v, causal=causal, scale=scale)
+    assert fa.status() == fa.FA_OK
+    O_ref, L_ref = oracle.attention_forward(f64(q), f64(k), f64(v), scale, causal)
+    return check_fwd(O, L, O_ref, L_ref, f"B{B} H{H} Nq{Nq} Nk{Nk} d{d} {dtype} causal={causal}")
+
+
+@pytest.mark.parametrize("w", [W.TINY_BF16, W.TINY_FP32], ids=lambda w: w.name)
+def test_tiny_workloads(fa, w):
+    run_full(fa, w.B, w.H, w.Nq, w.Nk, w.d, w.causal, w.dtype)
+
+
+def test_medium_workload(fa):
+    w = W.MEDIUM
+    run_full(fa, w.B, w.H, w.Nq, w.Nk, w.d, w.causal, w.dtype)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("N", [1, 17, 127, 128, 129, 255, 256, 257, 1000])
+def test_odd_lengths(fa, N, d, causal):
+    run_full(fa, 2, 3, N, N, d, causal, seed=N)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(1, 300), (100, 1000), (257, 513), (700, 129)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rectangular(fa, Nq, Nk, causal):
+    if causal and Nq > Nk:
+        pytest.skip("causal requires Nq <= Nk")
+    run_full(fa, 1, 2, Nq, Nk, 128, causal, seed=Nq + Nk)
+
+
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_fp16_and_bf16(fa, dtype):
+    run_full(fa, 2, 4, 384, 384, 128, True, dtype)
+    run_full(fa, 2, 4, 384, 512, 64, False, dtype)
+
+
+def test_fp32_tf32(fa):
+    run_full(fa, 1, 2, 300, 300, 64, True, "fp32")
+
+
+def test_peaky_rescaling(fa):
+    """Q scaled ×8: row maxima grow across many K/V tiles, exercising the
+    correction of the O accumulator."""
+    run_full(fa, 1, 4, 1024, 1024, 128, False, q_mult=8.0, seed=3)
+    run_full(fa, 1, 4, 1024, 1024, 128, True, q_mult=8.0, seed=4)
+
+
+def test_keys_sorted_ascending_force_rescales(fa):
+    """Scores that grow along the key axis: every tile raises the maximum."""
+    B, H, N, d = 1, 1, 1024, 64
+    q = torch.ones(B, H, N, d, device="cuda", dtype=torch.bfloat16)
+    ramp = torch.linspace(-4, 4, N, device="cuda").view(1, 1, N, 1)
+    k = (ramp * torch.ones(1, 1, 1, d, device="cuda")).to(torch.bfloat16).contiguous()
+    v = torch.randn(B, H, N, d, device="cuda", generator=torch.Generator("cuda").manual_seed(1)).to(torch.bfloat16)
+    O, L = fa.forward(q, k, v, causal=False, scale=1.0)
+    O_ref, L_ref = oracle.attention_forward(f64(q), f64(k), f64(v), 1.0, False)
+    check_fwd(O, L, O_ref, L_ref, "ascending scores")
+
+
+def _sampled(fa, w, heads, rows_per_head=96, seed=0):
+    q, k, v, _ = W.make_inputs(w, device="cuda", with_grad=False)
+    O, L = fa.forward(q, k, v, causal=w.causal, scale=w.scale)
+    assert fa.status() == fa.FA_OK
+    rng = np.random.default_rng(seed)
+    for (b, h) in heads:
+        rows = np.unique(np.concatenate([[0, 1, 127, 128, w.Nq - 1],
+                                         rng.integers(0, w.Nq, rows_per_head)]))
+        qh = f64(q[b, h])
+        O_ref, L_ref = oracle.head_forward(qh[rows], f64(k[b, h]), f64(v[b, h]), w.scale,
+                                           w.causal, rows=rows, nq_total=w.Nq)
+        check_fwd(O[b, h][torch.as_tensor(rows, device="cuda")],
+                  L[b, h][torch.as_tensor(rows, device="cuda")], O_ref, L_ref,
+                  f"{w.name} head ({b},{h})")
+    # properties at every output: finite, |O| bounded by max|V| of the head
+    assert torch.isfinite(O.float()).all() and torch.isfinite(L).all()
+    assert (O.float().abs().amax(dim=(2, 3)) <= v.float().abs().amax(dim=(2, 3)) * 1.01 + 1e-3).all()
+
+
+def test_causal_2k_sampled(fa):
+    w = W.CAUSAL_2K
+    _sampled(fa, w, [(0, 0), (3, 7), (7, 15)])
+
+
+def test_long_16k_sampled(fa):
+    w = W.LONG_16K
+    _sampled(fa, w, [(0, 0), (0, 13), (0, 31)], rows_per_head=64)
