@@ -86,7 +86,7 @@ int effective_dq_mode(int B, int H, int Nq, int Nk, int d) {
 }
 
 struct BwdWorkspace {
-  size_t d_off, dq_off, total;
+  size_t d_off, l_off, dq_off, total;
 };
 
 BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
@@ -95,7 +95,8 @@ BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
   const size_t nkv = (size_t(Nk) + 127) / 128;
   BwdWorkspace w;
   w.d_off = 0;
-  w.dq_off = round_up(BH * rows * sizeof(float), 256);
+  w.l_off = round_up(BH * rows * sizeof(float), 256);
+  w.dq_off = w.l_off + round_up(BH * rows * sizeof(float), 256);
   const size_t dq = BH * rows * size_t(d) * sizeof(float) * (mode == 2 ? nkv : 1);
   w.total = w.dq_off + round_up(dq, 256);
   return w;
@@ -200,13 +201,17 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   const int BH = B * H;
   BwdLaunch a;
   std::memset(&a, 0, sizeof(a));
-  if (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, 64) || !make_map(&a.tmdO, dO, dtype, d, Nq, BH, 64) ||
-      !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128))
+  const int bm = bwd_block_rows(d);
+  // (the fp32 path stages its operands without TMA)
+  if (dtype != FA_FP32 &&
+      (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, bm) || !make_map(&a.tmdO, dO, dtype, d, Nq, BH, bm) ||
+       !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128)))
     return FA_ERR_CUDA;
   BwdParams& p = a.params;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;
   p.dQ = dQ; p.dK = dK; p.dV = dV;
   p.Dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
+  p.Lsc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.l_off);
   p.dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dq_off);
   p.B = B; p.H = H; p.Nq = Nq; p.Nk = Nk;
   p.Nq_pad = bwd_pad_rows(Nq);

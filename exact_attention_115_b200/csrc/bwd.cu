@@ -1,11 +1,784 @@
-// Backward kernels (placeholder until the tcgen05 backward lands).
+// Backward attention kernels for sm_100a.
+//
+// FlashAttention V1/V2 study notes (51CTO):
+//   section "算法的改进": the backward needs only the row logsumexp L from
+//     the forward; P is rebuilt block by block as exp(scale·S − L) instead of
+//     being stored.
+//   section "Thread Block Level 并行": the backward is parallel along the K/V
+//     sequence ("vertical slices"): one CTA per K/V block, looping over the
+//     query blocks, so dK and dV stay on chip and are written once.
+//   section "Warp Level 并行": dV = Pᵀ dO, dP = dO Vᵀ, dS = P ∘ (dP − D),
+//     dQ = dS K, dK = dSᵀ Q (with the scale on dQ and dK and
+//     D = rowsum(dO ∘ O), the exact softmax gradient).
+//   section "Sequence Parallel": dQ receives a contribution from every K/V
+//     block, so it is reduced across CTAs, either by atomic adds into one
+//     buffer or by one buffer per K/V block and a separate reduction kernel.
+//     Both are implemented (dq_mode 1 and 2).  Mode 1 uses bulk reductions
+//     (cp.reduce.async.bulk .add.f32): a whole [BM × d] fp32 tile per
+//     instruction, performed in L2, instead of one atomic per element.
+//
+// Kernels: bwd_preprocess (D = rowsum(dO ∘ O), L·log2e into a padded buffer,
+// dQ accumulator cleared), bwd_main (below), bwd_dq_finalise (sum/convert).
+//
+// bwd_main, B200 design.  The two score-like products are computed
+// transposed (keys on TMEM lanes): Sᵀ = K Qᵀ and dPᵀ = V dOᵀ, so that the
+// thread owning key row k holds Pᵀ[k, :] and dSᵀ[k, :] and writes them back
+// to TMEM as the A operand of dV += Pᵀ dO and dK += dSᵀ Q (no shared-memory
+// round trip).  dSᵀ also goes to shared memory for the dQ product:
+//   d = 128: BM = 64 query rows per step, dQᵀ = Kᵀ dSᵀ (M = d = 128);
+//   d = 64:  BM = 128, dQ = dS K (M = BM = 128).
+// Roles (384 threads):
+//   warpgroup 0: thread = key row: P, dS, and the final dK/dV store;
+//   warpgroup 1: reads dQ from TMEM, stages it in shared memory, issues the
+//                bulk reduction (or partial store);
+//   warp 8: tcgen05.mma issuer, TMEM owner; warp 9: TMA producer.
+// TMEM (512 columns), d = 128: Sᵀ[2] | dPᵀ[2] | dV | dK (64,64,64,64,128,128);
+//                    d = 64:  Sᵀ[2] | dPᵀ | dV | dK (128,128,128,64,64).
+// Sᵀ is double buffered so the next step's Sᵀ MMA runs while the current
+// step is still in the softmax warps; dQ of step i reuses Sᵀ[i % 2] once
+// Pᵀ has been consumed by the dV product.
 #include "common.cuh"
 #include "launch.h"
 
 namespace fa {
 
+namespace {
+
+// ------------------------------------------------------------------ bulk copies
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
+               "r"(smem_u32(src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+// Named barrier that also ANDs a predicate over the participating threads,
+// so a go/no-go decision is uniform across them.
+__device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"(uint32_t(pred)), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <typename T, int D>
+struct BwdTraits {
+  static constexpr int ES = 2;
+  static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
+  static constexpr int BM = D == 128 ? 64 : 128;     // query rows per step
+  static constexpr bool DQ_T = D == 128;             // dQᵀ = Kᵀ dSᵀ (else dQ = dS K)
+  static constexpr int NSTG = 2;                     // Q/dO pipeline stages
+  static constexpr int KV_TILE = BN * D * ES;        // bytes of the K (or V) tile
+  static constexpr int KV_CHUNK = BN * 128;          // one 128-byte column block of it
+  static constexpr int Q_TILE = BM * D * ES;         // bytes of a Q (or dO) tile
+  static constexpr int Q_CHUNK = BM * 128;
+  static constexpr int DS_TILE = BN * BM * ES;       // dSᵀ, rows = keys, q contiguous
+  static constexpr int DQ_STAGE = BM * D * 4;        // fp32 dQ tile staging
+  // shared-memory offsets (all 1024-aligned)
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + KV_TILE;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;
+  static constexpr int OFF_DO = OFF_Q + NSTG * Q_TILE;
+  static constexpr int OFF_DS = OFF_DO + NSTG * Q_TILE;
+  static constexpr int OFF_DQ = OFF_DS + DS_TILE;
+  static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;        // L·log2e and D per stage
+  static constexpr int OFF_BAR = OFF_LD + NSTG * 2 * BM * 4;
+  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+  // TMEM columns
+  static constexpr int COL_S0 = 0;
+  static constexpr int COL_S1 = BM;
+  static constexpr int COL_DP0 = 2 * BM;
+  static constexpr int COL_DP1 = D == 128 ? 3 * BM : 2 * BM;  // single dPᵀ buffer for d = 64
+  static constexpr int COL_DV = D == 128 ? 4 * BM : 3 * BM;
+  static constexpr int COL_DK = COL_DV + D;
+  static_assert(COL_DK + D <= 512, "TMEM budget");
+  static constexpr int THREADS = 384;
+  static constexpr int REGS_COMPUTE = 232;
+  static constexpr int REGS_DQ = 120;
+  static constexpr int REGS_OTHER = 56;
+  static constexpr uint32_t F = ElemTraits<T>::fmt;
+  static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
+  static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV, dK (A in TMEM)
+  static constexpr uint32_t IDESC_DQ = make_idesc(F, 128, DQ_T ? BM : D, 1, 1);
+};
+
+struct BwdBarriers {
+  uint64_t kv_full;
+  uint64_t qdo_full[2];
+  uint64_t qdo_empty[2];
+  uint64_t s_full[2];
+  uint64_t dp_full[2];
+  uint64_t p_ready;
+  uint64_t ds_ready;
+  uint64_t dq_full;
+  uint64_t dq_empty;
+  uint64_t ds_free;
+  uint64_t dkv_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Query-tile range of K/V block `kb`: with bottom-right causal alignment the
+// first query that sees key kb*BN is kb*BN - (Nk - Nq).
+template <int BM, bool CAUSAL>
+__device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, int& n) {
+  int first = 0;
+  if (CAUSAL) first = max(0, kb * 128 - (Nk - Nq));
+  i0 = first / BM;
+  const int nt = (Nq + BM - 1) / BM;
+  n = max(0, nt - i0);
+}
+
+template <typename T, int D, bool CAUSAL>
+__global__ void __launch_bounds__(384, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    BwdParams p) {
+  using Tr = BwdTraits<T, D>;
+  constexpr int BM = Tr::BM;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Tr::OFF_BAR);
+  volatile int* abort_flag = &bars->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int key0 = kb * Tr::BN;
+  const int off = p.Nk - p.Nq;
+  int i0, n_q;
+  q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->kv_full, 1);
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->qdo_full[s], 1);
+      mbar_init(&bars->qdo_empty[s], 1);
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->dp_full[s], 1);
+    }
+    mbar_init(&bars->p_ready, 128);
+    mbar_init(&bars->ds_ready, 128);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->dkv_done, 1);
+    bars->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(&bars->tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    tma_prefetch_desc(&tmQ);
+    tma_prefetch_desc(&tmK);
+    tma_prefetch_desc(&tmV);
+    tma_prefetch_desc(&tmdO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  uint8_t* sK = smem + Tr::OFF_K;
+  uint8_t* sV = smem + Tr::OFF_V;
+  uint8_t* sQ = smem + Tr::OFF_Q;
+  uint8_t* sdO = smem + Tr::OFF_DO;
+  uint8_t* sdS = smem + Tr::OFF_DS;
+  float* sdQ = reinterpret_cast<float*>(smem + Tr::OFF_DQ);
+  float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
+
+  if (warp >= 10) {
+    regs_dec<Tr::REGS_OTHER>();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ producer
+    regs_dec<Tr::REGS_OTHER>();
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&bars->kv_full, 2 * Tr::KV_TILE);
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c) {
+        tma_load_3d(sK + c * Tr::KV_CHUNK, &tmK, &bars->kv_full, c * 64, key0, bh);
+        tma_load_3d(sV + c * Tr::KV_CHUNK, &tmV, &bars->kv_full, c * 64, key0, bh);
+      }
+      for (int i = 0; i < n_q; ++i) {
+        const int s = i % Tr::NSTG;
+        if (i >= Tr::NSTG &&
+            !mbar_wait(&bars->qdo_empty[s], ((i / Tr::NSTG) - 1) & 1, abort_flag))
+          break;
+        const int q0 = (i0 + i) * BM;
+        uint64_t* bar = &bars->qdo_full[s];
+        mbar_arrive_expect_tx(bar, 2 * Tr::Q_TILE + 2 * BM * 4);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c) {
+          tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
+          tma_load_3d(sdO + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmdO, bar, c * 64, q0, bh);
+        }
+        const size_t row = size_t(bh) * p.Nq_pad + q0;
+        bulk_load(sLD + (s * 2 + 0) * BM, p.Lsc + row, BM * 4, bar);
+        bulk_load(sLD + (s * 2 + 1) * BM, p.Dsum + row, BM * 4, bar);
+      }
+      // Drain every issued load before the CTA may exit.
+      for (int i = max(0, n_q - Tr::NSTG); i < n_q; ++i)
+        mbar_wait(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
+      mbar_wait(&bars->kv_full, 0, abort_flag);
+    }
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    regs_dec<Tr::REGS_OTHER>();
+    if (lane == 0) {
+      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      const uint32_t adS = smem_u32(sdS);
+      const uint32_t colS[2] = {tmem + Tr::COL_S0, tmem + Tr::COL_S1};
+      const uint32_t colDP[2] = {tmem + Tr::COL_DP0, tmem + Tr::COL_DP1};
+      const uint32_t colDV = tmem + Tr::COL_DV, colDK = tmem + Tr::COL_DK;
+
+      // Sᵀ (or dPᵀ) = X[128 keys × D] · Y[BM × D]ᵀ, both K-major.
+      auto mma_st = [&](uint32_t dcol, uint32_t aX, uint32_t aY) {
+#pragma unroll
+        for (int ks = 0; ks < D / 16; ++ks) {
+          const uint32_t oa = (ks >> 2) * Tr::KV_CHUNK + (ks & 3) * 32;
+          const uint32_t ob = (ks >> 2) * Tr::Q_CHUNK + (ks & 3) * 32;
+          mma_ss<false>(dcol, sw128_desc(aX + oa, 16, 1024), sw128_desc(aY + ob, 16, 1024),
+                        Tr::IDESC_ST, ks > 0);
+        }
+      };
+      // dV or dK [128 × D] += A[128 × BM] (TMEM) · Y[BM × D] (MN-major).
+      auto mma_grad = [&](uint32_t dcol, uint32_t acol, uint32_t aY, bool acc) {
+#pragma unroll
+        for (int ks = 0; ks < BM / 16; ++ks)
+          mma_ts<false>(dcol, acol + ks * 8, sw128_desc(aY + ks * 2048, Tr::Q_CHUNK, 1024),
+                        Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
+      };
+      // dQᵀ [D × BM] = Kᵀ · dSᵀ  (d = 128), or dQ [BM × D] = dS · K (d = 64);
+      // both operands MN-major, K dimension = the 128 keys.
+      auto mma_dq = [&](uint32_t dcol) {
+#pragma unroll
+        for (int ks = 0; ks < Tr::BN / 16; ++ks) {
+          uint64_t da, db;
+          if constexpr (Tr::DQ_T) {
+            da = sw128_desc(aK + ks * 2048, Tr::KV_CHUNK, 1024);
+            db = sw128_desc(adS + ks * 2048, Tr::BN * 128, 1024);
+          } else {
+            da = sw128_desc(adS + ks * 2048, Tr::BN * 128, 1024);
+            db = sw128_desc(aK + ks * 2048, Tr::KV_CHUNK, 1024);
+          }
+          mma_ss<false>(dcol, da, db, Tr::IDESC_DQ, ks > 0);
+        }
+      };
+      auto qwait = [&](int i) {
+        return mbar_wait(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
+      };
+
+      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag) && (n_q == 0 || qwait(0));
+      tc_fence_after();
+      if (ok && n_q > 0) {
+        mma_st(colS[0], aK, aQ);
+        tc_commit(&bars->s_full[0]);
+        mma_st(colDP[0], aV, adO);
+        tc_commit(&bars->dp_full[0]);
+      }
+      for (int i = 0; i < n_q && ok; ++i) {
+        const int s = i % Tr::NSTG, b2 = i & 1;
+        const uint32_t aQs = aQ + s * Tr::Q_TILE, adOs = adO + s * Tr::Q_TILE;
+        const bool more = i + 1 < n_q;
+        // Next step's Sᵀ into the other buffer (its previous dQ must have
+        // been read by the dQ warpgroup).
+        if (more) {
+          ok = qwait(i + 1) && (i < 1 || mbar_wait(&bars->dq_empty, (i - 1) & 1, abort_flag));
+          tc_fence_after();
+          if (!ok) break;
+          const int s1 = (i + 1) % Tr::NSTG;
+          mma_st(colS[b2 ^ 1], aK, aQ + s1 * Tr::Q_TILE);
+          tc_commit(&bars->s_full[b2 ^ 1]);
+          if constexpr (D == 128) {
+            mma_st(colDP[b2 ^ 1], aV, adO + s1 * Tr::Q_TILE);
+            tc_commit(&bars->dp_full[b2 ^ 1]);
+          }
+        }
+        ok = mbar_wait(&bars->p_ready, i & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        mma_grad(colDV, colS[b2], adOs, i > 0);
+        ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        mma_grad(colDK, colDP[D == 128 ? b2 : 0], aQs, i > 0);
+        tc_commit(&bars->qdo_empty[s]);
+        if (!more) tc_commit(&bars->dkv_done);
+        mma_dq(colS[b2]);
+        tc_commit(&bars->dq_full);
+        tc_commit(&bars->ds_free);
+        if constexpr (D == 64) {
+          if (more) {
+            mma_st(colDP[0], aV, adO + ((i + 1) % Tr::NSTG) * Tr::Q_TILE);
+            tc_commit(&bars->dp_full[0]);
+          }
+        }
+      }
+      if (n_q == 0) tc_commit(&bars->dkv_done);
+    }
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P / dS (thread = key)
+    regs_inc<Tr::REGS_COMPUTE>();
+    const int quad = warp;
+    const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
+    const int key = key0 + kr;
+    const bool key_live = key < p.Nk;
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const float sl2 = p.scale_log2;
+    const float scale = p.scale;
+    bool ok = true;
+    for (int i = 0; i < n_q; ++i) {
+      const int s = i % Tr::NSTG, b2 = i & 1;
+      const int q0 = (i0 + i) * BM;
+      const float* sL = sLD + (s * 2 + 0) * BM;
+      const float* sDv = sLD + (s * 2 + 1) * BM;
+      // ---- P = exp2(S·c − L·log2e), causal / ragged masking
+      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b2], (i >> 1) & 1, abort_flag));
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tS = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
+      // A key sees query q iff key <= q + off; keys past Nk contribute nothing.
+      const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
+      const int qmin = key - off;  // first query row that sees this key
+      float P[BM];
+      const uint64_t c2 = pk2(sl2, sl2);
+      // Processed 64 columns at a time: Pᵀ is packed to bf16 pairs and stored
+      // straight back to TMEM; the fp32 P stays in registers for dS.
+#pragma unroll
+      for (int c = 0; c < BM; c += 64) {
+        uint32_t w[32];
+#pragma unroll
+        for (int h = 0; h < 64; h += 32) {
+          uint32_t u[32];
+          tmem_ld32(tS + c + h, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = c + h + e;
+            const float2 x = upk2(ffma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
+                                        pk2(-sL[q], -sL[q + 1])));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
+            if (need_mask) {
+              if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
+              if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
+            }
+            P[q] = p0;
+            P[q + 1] = p1;
+            w[(h + e) / 2] = ElemTraits<T>::pack2(p0, p1);
+          }
+        }
+        tmem_st32(tS + c / 2, w);
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->p_ready);
+
+      // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
+      // and to shared memory for the dQ product (row = key, BM query values
+      // contiguous, 128-byte swizzled, 64 values per column block).
+      ok = __all_sync(0xffffffffu,
+                      mbar_wait(&bars->dp_full[D == 128 ? b2 : 0], (D == 128 ? (i >> 1) : i) & 1,
+                                abort_flag));
+      if (ok && i > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(&bars->ds_free, (i - 1) & 1, abort_flag));
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tDP = tmem + lane_off + (D == 128 && b2 ? Tr::COL_DP1 : Tr::COL_DP0);
+#pragma unroll
+      for (int c = 0; c < BM; c += 64) {
+        uint32_t w[32];
+#pragma unroll
+        for (int h = 0; h < 64; h += 32) {
+          uint32_t u[32];
+          tmem_ld32(tDP + c + h, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int q = c + h + e;
+            const uint64_t t = fadd2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])),
+                                     pk2(-sDv[q], -sDv[q + 1]));
+            const float2 ds = upk2(fmul2(t, pk2(P[q] * scale, P[q + 1] * scale)));
+            w[(h + e) / 2] = ElemTraits<T>::pack2(ds.x, ds.y);
+          }
+        }
+        tmem_st32(tDP + c / 2, w);
+        uint8_t* rowp = sdS + (c / 64) * (Tr::BN * 128) + kr * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch)
+          *reinterpret_cast<uint4*>(rowp + ((ch ^ (kr & 7)) << 4)) =
+              make_uint4(w[ch * 4], w[ch * 4 + 1], w[ch * 4 + 2], w[ch * 4 + 3]);
+      }
+      fence_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      mbar_arrive(&bars->ds_ready);
+    }
+    // ---- dK, dV out (once per CTA)
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkv_done, 0, abort_flag));
+    tc_fence_after();
+    if (ok) {
+      T* dKrow = reinterpret_cast<T*>(p.dK) + (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
+      T* dVrow = reinterpret_cast<T*>(p.dV) + (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
+#pragma unroll 1
+      for (int which = 0; which < 2; ++which) {
+        const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV);
+        T* out = which ? dKrow : dVrow;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tcol + c, u);
+          tmem_ld_wait();
+          if (key_live && n_q > 0) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8) {
+              uint4 v;
+              v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+              v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
+              v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]), __uint_as_float(u[e + 5]));
+              v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]), __uint_as_float(u[e + 7]));
+              *reinterpret_cast<uint4*>(out + c + e) = v;
+            }
+          } else if (key_live) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 8)
+              *reinterpret_cast<uint4*>(out + c + e) = make_uint4(0, 0, 0, 0);
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ (warpgroup 1)
+    regs_dec<Tr::REGS_DQ>();
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;  // TMEM lane: d index (dQᵀ) or query row (dQ)
+    const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const bool leader = (warp == 4 && lane == 0);
+    bool ok = true;
+    for (int i = 0; i < n_q; ++i) {
+      const int b2 = i & 1;
+      const int q0 = (i0 + i) * BM;
+      ok = named_bar_and(1, 128, mbar_wait(&bars->dq_full, i & 1, abort_flag));
+      tc_fence_after();
+      if (!ok) break;
+      const uint32_t tQ = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
+      constexpr int NV = Tr::DQ_T ? BM : D;  // values per thread
+      float v[NV];
+#pragma unroll
+      for (int c = 0; c < NV; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tQ + c, u);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[c + e] = __uint_as_float(u[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars->dq_empty);
+      // The previous bulk operation must have finished reading the staging buffer.
+      if (leader) bulk_wait_read0();
+      named_bar(1, 128);
+      if constexpr (Tr::DQ_T) {
+        // thread = d index r; staging is [BM][D] row-major fp32
+#pragma unroll
+        for (int q = 0; q < BM; ++q) sdQ[q * D + r] = v[q];
+      } else {
+        // thread = query row r; write its D values, rotating the 16-byte
+        // chunk order by lane to spread shared-memory banks
+#pragma unroll
+        for (int cc = 0; cc < D / 4; ++cc) {
+          const int c4 = (cc + lane) % (D / 4);
+          float4 x;
+          x.x = v[c4 * 4 + 0];
+          x.y = v[c4 * 4 + 1];
+          x.z = v[c4 * 4 + 2];
+          x.w = v[c4 * 4 + 3];
+          *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
+        }
+      }
+      fence_async_smem();
+      named_bar(1, 128);
+      if (leader) {
+        if (p.dq_mode == 2) {
+          float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
+          bulk_store(dst, sdQ, Tr::DQ_STAGE);
+        } else {
+          float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
+          bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+        }
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// D = rowsum(dO ∘ O); L·log2e copied into a padded buffer (+inf on padding
+// rows, so their P is 0); in mode 1 the fp32 dQ accumulator is cleared.
+// A group of D/8 lanes handles one row (8 elements per lane).
+template <typename T, int D>
+__global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
+  constexpr int LPR = D / 8;
+  constexpr int RPB = 256 / LPR;  // rows per block
+  const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
+  const int bh = blockIdx.y;
+  const int q = blockIdx.x * RPB + g;
+  if (q >= p.Nq_pad) return;
+  float dsum = 0.f;
+  float lsc = INFINITY;
+  if (q < p.Nq) {
+    const size_t off = (size_t(bh) * p.Nq + q) * D + sl * 8;
+    const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.O) + off);
+    const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dO) + off);
+    const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float2 x = ElemTraits<T>::unpack2(aw[k]), y = ElemTraits<T>::unpack2(cw[k]);
+      dsum = fmaf(x.x, y.x, dsum);
+      dsum = fmaf(x.y, y.y, dsum);
+    }
+    lsc = p.L[size_t(bh) * p.Nq + q] * kLog2e;
+  }
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
+  const size_t row = size_t(bh) * p.Nq_pad + q;
+  if (sl == 0) {
+    p.Dsum[row] = q < p.Nq ? dsum : 0.f;
+    p.Lsc[row] = lsc;
+  }
+  if (p.dq_mode == 1) {
+    float4* z = reinterpret_cast<float4*>(p.dQacc + row * D + sl * 8);
+    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// dQ = Σ (dQ accumulator or per-K/V-block partials), cast to the dtype.
+template <typename T, int D, bool CAUSAL>
+__global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
+  constexpr int LPR = D / 8;
+  constexpr int RPB = 256 / LPR;
+  const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
+  const int bh = blockIdx.y;
+  const int q = blockIdx.x * RPB + g;
+  if (q >= p.Nq) return;
+  float acc[8];
+  const size_t row = size_t(bh) * p.Nq_pad + q;
+  if (p.dq_mode == 2) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+    int last = p.n_kblocks - 1;
+    if (CAUSAL) last = min(last, (q + p.Nk - p.Nq) / 128);
+    const size_t stride = size_t(p.B) * p.H * p.Nq_pad * D;
+    for (int j = 0; j <= last; ++j) {
+      const float4* src = reinterpret_cast<const float4*>(p.dQacc + j * stride + row * D + sl * 8);
+      const float4 x = src[0], y = src[1];
+      acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;
+      acc[4] += y.x; acc[5] += y.y; acc[6] += y.z; acc[7] += y.w;
+    }
+  } else {
+    const float4* src = reinterpret_cast<const float4*>(p.dQacc + row * D + sl * 8);
+    const float4 x = src[0], y = src[1];
+    acc[0] = x.x; acc[1] = x.y; acc[2] = x.z; acc[3] = x.w;
+    acc[4] = y.x; acc[5] = y.y; acc[6] = y.z; acc[7] = y.w;
+  }
+  uint4 o;
+  o.x = ElemTraits<T>::pack2(acc[0], acc[1]);
+  o.y = ElemTraits<T>::pack2(acc[2], acc[3]);
+  o.z = ElemTraits<T>::pack2(acc[4], acc[5]);
+  o.w = ElemTraits<T>::pack2(acc[6], acc[7]);
+  *reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dQ) + (size_t(bh) * p.Nq + q) * D + sl * 8) = o;
+}
+
+// fp32 backward on the CUDA cores (fp32 inputs only; a parity path, not a
+// fast one).  Same structure as the tensor-core kernel: one CTA per block of
+// 64 keys, query rows visited one at a time, P rebuilt from L, D = dO·O per
+// row, dK/dV accumulated in shared memory and written once, dQ added with
+// fp32 atomics into the (zeroed) output.
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(256) bwd_fp32_simt_kernel(BwdParams p) {
+  constexpr int BK = 64;
+  extern __shared__ float fsm[];
+  float* sK = fsm;               // [BK][D]
+  float* sV = sK + BK * D;       // [BK][D]
+  float* sdK = sV + BK * D;      // [BK][D]
+  float* sdV = sdK + BK * D;     // [BK][D]
+  float* sq = sdV + BK * D;      // [D]
+  float* sdo = sq + D;           // [D]
+  float* sp = sdo + D;           // [BK]
+  float* sds = sp + BK;          // [BK]
+  __shared__ float sred[2];
+  const int tid = threadIdx.x;
+  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int bh = b * p.H + h;
+  const int key0 = kb * BK;
+  const int off = p.Nk - p.Nq;
+  const float* Q = reinterpret_cast<const float*>(p.Q) + size_t(bh) * p.Nq * D;
+  const float* K = reinterpret_cast<const float*>(p.K) + size_t(bh) * p.Nk * D;
+  const float* V = reinterpret_cast<const float*>(p.V) + size_t(bh) * p.Nk * D;
+  const float* O = reinterpret_cast<const float*>(p.O) + size_t(bh) * p.Nq * D;
+  const float* dO = reinterpret_cast<const float*>(p.dO) + size_t(bh) * p.Nq * D;
+  float* dQ = reinterpret_cast<float*>(p.dQ) + size_t(bh) * p.Nq * D;
+  for (int i = tid; i < BK * D; i += 256) {
+    const int k = i / D;
+    const bool live = key0 + k < p.Nk;
+    sK[i] = live ? K[size_t(key0) * D + i] : 0.f;
+    sV[i] = live ? V[size_t(key0) * D + i] : 0.f;
+    sdK[i] = 0.f;
+    sdV[i] = 0.f;
+  }
+  __syncthreads();
+  const int q_first = CAUSAL ? max(0, key0 - off) : 0;
+  const int k_sub = tid >> 2, part = tid & 3;  // 4 threads per key
+  for (int q = q_first; q < p.Nq; ++q) {
+    for (int c = tid; c < D; c += 256) {
+      sq[c] = Q[size_t(q) * D + c];
+      sdo[c] = dO[size_t(q) * D + c];
+    }
+    if (tid < 32) {  // D_q = dO_q · O_q
+      float acc = 0.f;
+      for (int c = tid; c < D; c += 32) acc = fmaf(dO[size_t(q) * D + c], O[size_t(q) * D + c], acc);
+      for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+      if (tid == 0) sred[0] = acc;
+    }
+    __syncthreads();
+    {
+      const int key = key0 + k_sub;
+      float s = 0.f, dp = 0.f;
+      for (int c = part; c < D; c += 4) {
+        s = fmaf(sq[c], sK[k_sub * D + c], s);
+        dp = fmaf(sdo[c], sV[k_sub * D + c], dp);
+      }
+      s += __shfl_xor_sync(0xffffffffu, s, 1);
+      s += __shfl_xor_sync(0xffffffffu, s, 2);
+      dp += __shfl_xor_sync(0xffffffffu, dp, 1);
+      dp += __shfl_xor_sync(0xffffffffu, dp, 2);
+      const bool vis = key < p.Nk && (!CAUSAL || key <= q + off);
+      const float L = p.L[size_t(bh) * p.Nq + q];
+      const float pr = vis ? expf(s * p.scale - L) : 0.f;
+      if (part == 0) {
+        sp[k_sub] = pr;
+        sds[k_sub] = pr * (dp - sred[0]) * p.scale;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < BK * D; i += 256) {
+      const int k = i / D, c = i % D;
+      sdV[i] = fmaf(sp[k], sdo[c], sdV[i]);
+      sdK[i] = fmaf(sds[k], sq[c], sdK[i]);
+    }
+    for (int c = tid; c < D; c += 256) {
+      float acc = 0.f;
+      for (int k = 0; k < BK; ++k) acc = fmaf(sds[k], sK[k * D + c], acc);
+      atomicAdd(&dQ[size_t(q) * D + c], acc);
+    }
+    __syncthreads();
+  }
+  float* dK = reinterpret_cast<float*>(p.dK) + size_t(bh) * p.Nk * D;
+  float* dV = reinterpret_cast<float*>(p.dV) + size_t(bh) * p.Nk * D;
+  for (int i = tid; i < BK * D; i += 256) {
+    if (key0 + i / D < p.Nk) {
+      dK[size_t(key0) * D + i] = sdK[i];
+      dV[size_t(key0) * D + i] = sdV[i];
+    }
+  }
+}
+
+template <int D, bool CAUSAL>
+static cudaError_t launch_bwd_fp32(const BwdLaunch& a) {
+  const BwdParams& p = a.params;
+  cudaError_t e = cudaMemsetAsync(p.dQ, 0, size_t(p.B) * p.H * p.Nq * D * sizeof(float), a.stream);
+  if (e != cudaSuccess) return e;
+  const int smem = (4 * 64 * D + 2 * D + 2 * 64) * sizeof(float);
+  auto kern = bwd_fp32_simt_kernel<D, CAUSAL>;
+  e = set_smem_once(reinterpret_cast<const void*>(kern), smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3((p.Nk + 63) / 64, p.H, p.B), 256, smem, a.stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+template <typename T, int D, bool CAUSAL>
+static cudaError_t launch_bwd_t(const BwdLaunch& a) {
+  using Tr = BwdTraits<T, D>;
+  const BwdParams& p = a.params;
+  constexpr int RPB = 256 / (D / 8);
+  const int BH = p.B * p.H;
+  bwd_preprocess_kernel<T, D><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  auto kern = bwd_main_kernel<T, D, CAUSAL>;
+  e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
+    if (e != cudaSuccess) return e;
+    regs_ok = attr.numRegs * Tr::THREADS >=
+              128 * (Tr::REGS_COMPUTE + Tr::REGS_DQ + Tr::REGS_OTHER);
+  }
+  if (!regs_ok) return cudaErrorInvalidConfiguration;
+  kern<<<dim3(p.n_kblocks, p.H, p.B), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV,
+                                                                               a.tmdO, p);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  bwd_dq_finalise_kernel<T, D, CAUSAL><<<dim3((p.Nq + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  return cudaGetLastError();
+}
+
+int bwd_block_rows(int d) { return d == 128 ? 64 : 128; }
+
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
-  (void)dtype; (void)d; (void)causal; (void)a;
+#define FA_BWD_CASE(TY, DD) \
+  return causal ? launch_bwd_t<TY, DD, true>(a) : launch_bwd_t<TY, DD, false>(a);
+  if (dtype == FA_BF16) {
+    if (d == 64) FA_BWD_CASE(__nv_bfloat16, 64)
+    if (d == 128) FA_BWD_CASE(__nv_bfloat16, 128)
+  } else if (dtype == FA_FP16) {
+    if (d == 64) FA_BWD_CASE(__half, 64)
+    if (d == 128) FA_BWD_CASE(__half, 128)
+  } else if (dtype == FA_FP32) {
+    if (d == 64) return causal ? launch_bwd_fp32<64, true>(a) : launch_bwd_fp32<64, false>(a);
+    if (d == 128) return causal ? launch_bwd_fp32<128, true>(a) : launch_bwd_fp32<128, false>(a);
+  }
+#undef FA_BWD_CASE
   return cudaErrorNotSupported;
 }
 

@@ -39,6 +39,7 @@ struct BwdParams {
   void* dK;
   void* dV;
   float* Dsum;    // [B*H, Nq_pad] rowsum(dO * O), padded rows zero
+  float* Lsc;     // [B*H, Nq_pad] L * log2(e), padded rows +inf
   float* dQacc;   // [B*H, Nq_pad, d] fp32 (mode 1) or [nkv, B*H, Nq_pad, d] (mode 2)
   int B, H, Nq, Nk, Nq_pad;
   float scale;        // softmax scale
@@ -54,6 +55,8 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a);
+// Query rows per backward step (the TMA box height of Q and dO).
+int bwd_block_rows(int d);
 
 struct DecodeParams {
   const void* Q;
