@@ -1,0 +1,367 @@
+"""Benchmark: fused exact attention on B200 (forward + backward step, plus
+the split-KV decode).
+
+One step = the whole training hot path on one batch of the causal workload
+B=8, H=16, N=2048, d=128, bf16: fa_fwd (forward kernel), then fa_bwd
+(D = rowsum(dO∘O) preprocessing, the backward kernel, the dQ finalise).
+``value`` is fwd+bwd TFLOPS over all ranks, counting 4·B·H·N²·d/2 for the
+forward and 2.5× that for the backward (causal halves both).  Inputs live in
+HBM before the timed region; each step touches ~0.4 GB, larger than the
+126 MB L2, so no flush is inserted.  The decode workload (B=32, H=32,
+Nk=32768, d=128) is timed separately and reported under "decode".
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Under torchrun each rank runs its own copy of the workload (attention heads
+are independent: no collective on the data path; weak scaling); times are
+the max over ranks.  ``--impl reference`` times the fp64 CPU oracle instead
+(a bounded sample of the same workload, rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention fwd+bwd TFLOPS (bf16, 1xB200 per rank)"
+UNIT = "TFLOP/s"
+PEAKS_PATH = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_PATH) as f:
+            return json.load(f), "measured"
+    except OSError:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dist_info():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        under_load = [x for x in sm if smax and x > 0.3 * smax] or sm
+        return {"sm_mhz": statistics.median(under_load) if under_load else None,
+                "sm_max_mhz": smax, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def time_oracle_sample(w, budget_s=12.0):
+    """fp64 oracle fwd+bwd on whole heads of the workload until ~budget_s of
+    CPU time; returns (TFLOP/s, heads, seconds, cores)."""
+    import numpy as np
+
+    import oracle
+
+    q, k, v, do = W.make_tensors(1, 1, w.Nq, w.Nk, w.d, w.dtype, seed=w.seed, q_mult=w.q_mult)
+    f = lambda t: t[0, 0].float().double().numpy()
+    qh, kh, vh, doh = f(q), f(k), f(v), f(do)
+    heads, t0 = 0, time.perf_counter()
+    while True:
+        oracle.head_forward(qh, kh, vh, w.scale, w.causal)
+        oracle.head_backward(qh, kh, vh, doh, w.scale, w.causal)
+        heads += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or heads >= w.B * w.H:
+            break
+    flops_per_head = (w.fwd_flops + w.bwd_flops) / (w.B * w.H)
+    cores = len(os.sched_getaffinity(0))
+    return flops_per_head * heads / el / 1e12, heads, el, cores
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_info()
+    if rank != 0:
+        return
+    per_step, heads_total, el_total = [], 0, 0.0
+    for i in range(args.warmup + args.steps):
+        tf, heads, el, cores = time_oracle_sample(w, budget_s=max(2.0, 60.0 / (args.warmup + args.steps)))
+        if i >= args.warmup:
+            per_step.append(el)
+            heads_total += heads
+            el_total += el
+    flops = (w.fwd_flops + w.bwd_flops) / (w.B * w.H) * heads_total
+    value = flops / el_total / 1e12
+    sample = f"{heads_total} of {w.B * w.H} heads per {args.steps} steps, fp64 numpy fwd+bwd"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * el_total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "shape": w.describe(), "global_batch": w.B, "seq_len": w.Nq,
+                   "parallelism": f"replicas{world}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    w = W.CAUSAL_2K
+    if args.impl == "reference":
+        run_reference(args, w)
+        return
+
+    world, rank, local = dist_info()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    import exact_attention_115_b200 as fa
+
+    fa.lib()
+    peaks, peak_kind = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+
+    q, k, v, do = W.make_inputs(W.Workload(**{**w.__dict__, "seed": w.seed + rank}), device=dev)
+    O, L = fa.forward(q, k, v, causal=True)
+    dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+    ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d), dtype=torch.uint8,
+                     device=dev)
+
+    def step():
+        fa.forward(q, k, v, causal=True, out=O, lse=L)
+        fa.backward(q, k, v, O, do, L, causal=True, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    st = fa.status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"kernel status after warm-up: {fa.STATUS_NAMES.get(st, st)}, "
+                           f"first timed-out wait {fa.lib().fa_last_timeout_site()}")
+
+    # Per-step events: whole step, forward kernel, main backward kernel.
+    K = args.steps
+    ev = {n: [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+          for n in ("s0", "f1", "b0", "b1", "s1")}
+    for lst in ev.values():
+        for e in lst:
+            e.record(stream)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(K):
+        ev["s0"][i].record(stream)
+        fa.forward(q, k, v, causal=True, out=O, lse=L)
+        ev["f1"][i].record(stream)
+        fa.set_bwd_timing_events(ev["b0"][i], ev["b1"][i])
+        fa.backward(q, k, v, O, do, L, causal=True, dq=dq, dk=dk, dv=dv, workspace=ws)
+        ev["s1"][i].record(stream)
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    fa.set_bwd_timing_events(None, None)
+    if pg:
+        pg.barrier()
+    clocks = sampler.stop()
+    st = fa.status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"kernel status {fa.STATUS_NAMES.get(st, st)}, "
+                           f"first timed-out wait {fa.lib().fa_last_timeout_site()}")
+
+    total_ms = t_start.elapsed_time(t_stop)
+    fwd_ms = [ev["s0"][i].elapsed_time(ev["f1"][i]) for i in range(K)]
+    bwd_main_ms = [ev["b0"][i].elapsed_time(ev["b1"][i]) for i in range(K)]
+    bwd_ms = [ev["f1"][i].elapsed_time(ev["s1"][i]) for i in range(K)]
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if pg:
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    flops_step = w.fwd_flops + w.bwd_flops
+    value = flops_step * K * world / (total_ms * 1e-3) / 1e12
+
+    fwd_avg = statistics.mean(fwd_ms)
+    bwd_main_avg = statistics.mean(bwd_main_ms)
+    bwd_avg = statistics.mean(bwd_ms)
+    peak_burst = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    achieved_bwd = w.bwd_flops / (bwd_main_avg * 1e-3) / 1e12
+    achieved_fwd = w.fwd_flops / (fwd_avg * 1e-3) / 1e12
+
+    # End to end through the same public API: pinned host inputs copied in,
+    # outputs (O, L, dQ, dK, dV) copied back, every step inside the region.
+    e2e = None
+    if rank == 0 or world > 1:
+        hq, hk, hv, hdo = (x.cpu().pin_memory() for x in (q, k, v, do))
+        ho, hl = torch.empty_like(hq).pin_memory(), torch.empty(L.shape, dtype=L.dtype).pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(x).pin_memory() for x in (hq, hk, hv))
+        h2d = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hdo))
+        d2h = sum(x.numel() * x.element_size() for x in (ho, hl, hdq, hdk, hdv))
+        ksteps = max(3, min(K, 10))
+
+        def e2e_step():
+            for hsrc, dst in ((hq, q), (hk, k), (hv, v), (hdo, do)):
+                dst.copy_(hsrc, non_blocking=True)
+            fa.forward(q, k, v, causal=True, out=O, lse=L)
+            fa.backward(q, k, v, O, do, L, causal=True, dq=dq, dk=dk, dv=dv, workspace=ws)
+            for src, hdst in ((O, ho), (L, hl), (dq, hdq), (dk, hdk), (dv, hdv)):
+                hdst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ksteps):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        et = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
+        if pg:
+            pg.all_reduce(et, op=pg.ReduceOp.MAX)
+        e2e = {"value": flops_step * ksteps * world / (float(et.item()) * 1e-3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": ksteps}
+
+    # Decode (split-KV + combine), timed on its own.
+    decode = None
+    del dq, dk, dv, ws
+    if not args.no_decode:
+        wd = W.DECODE_32K
+        del q, k, v, do, O, L
+        torch.cuda.empty_cache()
+        dq_, dk_, dv_, _ = W.make_inputs(wd, device=dev, with_grad=False)
+        Od, Ld = fa.decode(dq_, dk_, dv_)
+        wsd = torch.empty(fa.decode_workspace_bytes(wd.B, wd.H, wd.Nk, wd.d), dtype=torch.uint8,
+                          device=dev)
+        for _ in range(3):
+            fa.decode(dq_, dk_, dv_, out=Od, lse=Ld, workspace=wsd)
+        torch.cuda.synchronize()
+        nd = 10
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(nd):
+            fa.decode(dq_, dk_, dv_, out=Od, lse=Ld, workspace=wsd)
+        b.record(stream)
+        torch.cuda.synchronize()
+        dms = a.elapsed_time(b) / nd
+        kv_bytes = 2 * wd.B * wd.H * wd.Nk * wd.d * 2
+        gbs = kv_bytes / (dms * 1e-3) / 1e9
+        hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+        decode = {"workload": wd.name, "shape": wd.describe(), "ms": dms, "value": gbs,
+                  "unit": "GB/s", "l2": "17.2 GB of K/V per call, far larger than L2",
+                  "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                               "frac": gbs / hbm, "peak_kind": peak_kind,
+                               "traffic": None}}
+        assert fa.status() == fa.FA_OK
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tf, heads, el, cores = time_oracle_sample(w)
+        cpu = {"value": tf, "unit": UNIT, "cores": cores, "kind": "oracle",
+               "sample": f"{heads} of {w.B * w.H} heads fwd+bwd in fp64 numpy ({el:.1f} s)"}
+
+    if rank != 0:
+        if pg:
+            pg.destroy_process_group()
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "shape": w.describe(), "global_batch": w.B * world,
+                   "seq_len": w.Nq, "heads": w.H, "head_dim": w.d, "causal": True,
+                   "parallelism": f"replicas{world}",
+                   "l2": "inputs ~0.4 GB per step > 126 MB L2; no flush"},
+        "fwd": {"ms": fwd_avg, "tflops": achieved_fwd},
+        "bwd": {"ms": bwd_avg, "tflops": w.bwd_flops / (bwd_avg * 1e-3) / 1e12,
+                "main_kernel_ms": bwd_main_avg},
+        "pct_of_peak": value / world / peak_burst,
+        "roofline": {"bound": "tensor", "kernel": "bwd_main_kernel", "achieved": achieved_bwd,
+                     "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved_bwd / peak_burst,
+                     "peak_kind": f"{peak_kind} burst bf16", "traffic": None},
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+        "decode": decode,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    if pg:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -37,6 +37,8 @@ SIGNATURES = {
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
     "fa_status": (_I, [_VP]),
+    "fa_bwd_set_timing_events": (_I, [_VP, _VP]),
+    "fa_last_timeout_site": (_I, []),
     "fa_version": (ctypes.c_char_p, []),
 }
 
@@ -194,6 +196,16 @@ def status(device=None) -> int:
     """Synchronise the current stream and return (and clear) the kernel
     error status: FA_OK, FA_ERR_TIMEOUT or FA_ERR_CUDA."""
     return int(lib().fa_status(_stream(device)))
+
+
+def set_bwd_timing_events(start=None, stop=None) -> None:
+    """Record torch.cuda.Event ``start``/``stop`` around the main backward
+    kernel of every later backward() call (None, None switches it off).  The
+    events must already exist on the device (record them once first)."""
+    if start is None or stop is None:
+        lib().fa_bwd_set_timing_events(None, None)
+    else:
+        lib().fa_bwd_set_timing_events(start.cuda_event, stop.cuda_event)
 
 
 def version() -> str:

@@ -16,6 +16,8 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 int g_dq_mode = 0;  // 0 auto, 1 reduce-add, 2 partial buffers
+cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_bwd_set_timing_events
+int g_last_site = 0;  // fa_last_timeout_site
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -220,6 +222,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   p.n_kblocks = (Nk + 127) / 128;
   p.dq_mode = mode;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.ev_start = g_ev_start;
+  a.ev_stop = g_ev_stop;
   return launch_bwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -270,13 +274,26 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
 int fa_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return FA_ERR_CUDA;
-  int word = 0;
-  if (take_error_fwd(&word) != cudaSuccess) return FA_ERR_CUDA;
-  if (take_error_bwd(&word) != cudaSuccess) return FA_ERR_CUDA;
-  if (take_error_decode(&word) != cudaSuccess) return FA_ERR_CUDA;
+  int word = 0, site = 0;
+  if (take_error_fwd(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
+  if (take_error_bwd(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
+  if (take_error_decode(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
+  if (site != 0) g_last_site = site;
   if (word != 0) return FA_ERR_TIMEOUT;
   return FA_OK;
 }
+
+int fa_bwd_set_timing_events(void* start, void* stop) {
+  if (start && stop) {
+    g_ev_start = static_cast<cudaEvent_t>(start);
+    g_ev_stop = static_cast<cudaEvent_t>(stop);
+  } else {
+    g_ev_start = g_ev_stop = nullptr;
+  }
+  return FA_OK;
+}
+
+int fa_last_timeout_site(void) { return g_last_site; }
 
 const char* fa_version(void) { return "fa-b200 0.1 (sm_100a)"; }
 

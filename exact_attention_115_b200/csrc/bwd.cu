@@ -37,6 +37,7 @@
 // Sᵀ is double buffered so the next step's Sᵀ MMA runs while the current
 // step is still in the softmax warps; dQ of step i reuses Sᵀ[i % 2] once
 // Pᵀ has been consumed by the dV product.
+#define FA_SITE_BASE 20000
 #include "common.cuh"
 #include "launch.h"
 
@@ -135,9 +136,12 @@ struct BwdBarriers {
   uint64_t qdo_empty[2];
   uint64_t s_full[2];
   uint64_t dp_full[2];
-  uint64_t p_ready;
+  // One barrier per Sᵀ buffer for the signals whose producer can otherwise
+  // run two phases ahead of a parity wait (the next step's Sᵀ is already
+  // there, or the last step skips the back-pressure wait).
+  uint64_t p_ready[2];
   uint64_t ds_ready;
-  uint64_t dq_full;
+  uint64_t dq_full[2];
   uint64_t dq_empty;
   uint64_t ds_free;
   uint64_t dkv_done;
@@ -185,9 +189,11 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->dp_full[s], 1);
     }
-    mbar_init(&bars->p_ready, 128);
+    mbar_init(&bars->p_ready[0], 128);
+    mbar_init(&bars->p_ready[1], 128);
     mbar_init(&bars->ds_ready, 128);
-    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_full[0], 1);
+    mbar_init(&bars->dq_full[1], 1);
     mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dkv_done, 1);
@@ -232,7 +238,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int i = 0; i < n_q; ++i) {
         const int s = i % Tr::NSTG;
         if (i >= Tr::NSTG &&
-            !mbar_wait(&bars->qdo_empty[s], ((i / Tr::NSTG) - 1) & 1, abort_flag))
+            !MBAR_WAIT(&bars->qdo_empty[s], ((i / Tr::NSTG) - 1) & 1, abort_flag))
           break;
         const int q0 = (i0 + i) * BM;
         uint64_t* bar = &bars->qdo_full[s];
@@ -248,8 +254,8 @@ __global__ void __launch_bounds__(384, 1)
       }
       // Drain every issued load before the CTA may exit.
       for (int i = max(0, n_q - Tr::NSTG); i < n_q; ++i)
-        mbar_wait(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
-      mbar_wait(&bars->kv_full, 0, abort_flag);
+        MBAR_WAIT(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
+      MBAR_WAIT(&bars->kv_full, 0, abort_flag);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -295,10 +301,10 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
       auto qwait = [&](int i) {
-        return mbar_wait(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
+        return MBAR_WAIT(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
       };
 
-      bool ok = mbar_wait(&bars->kv_full, 0, abort_flag) && (n_q == 0 || qwait(0));
+      bool ok = MBAR_WAIT(&bars->kv_full, 0, abort_flag) && (n_q == 0 || qwait(0));
       tc_fence_after();
       if (ok && n_q > 0) {
         mma_st(colS[0], aK, aQ);
@@ -313,7 +319,7 @@ __global__ void __launch_bounds__(384, 1)
         // Next step's Sᵀ into the other buffer (its previous dQ must have
         // been read by the dQ warpgroup).
         if (more) {
-          ok = qwait(i + 1) && (i < 1 || mbar_wait(&bars->dq_empty, (i - 1) & 1, abort_flag));
+          ok = qwait(i + 1) && (i < 1 || MBAR_WAIT(&bars->dq_empty, (i - 1) & 1, abort_flag));
           tc_fence_after();
           if (!ok) break;
           const int s1 = (i + 1) % Tr::NSTG;
@@ -324,18 +330,18 @@ __global__ void __launch_bounds__(384, 1)
             tc_commit(&bars->dp_full[b2 ^ 1]);
           }
         }
-        ok = mbar_wait(&bars->p_ready, i & 1, abort_flag);
+        ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         mma_grad(colDV, colS[b2], adOs, i > 0);
-        ok = mbar_wait(&bars->ds_ready, i & 1, abort_flag);
+        ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         mma_grad(colDK, colDP[D == 128 ? b2 : 0], aQs, i > 0);
         tc_commit(&bars->qdo_empty[s]);
         if (!more) tc_commit(&bars->dkv_done);
         mma_dq(colS[b2]);
-        tc_commit(&bars->dq_full);
+        tc_commit(&bars->dq_full[b2]);
         tc_commit(&bars->ds_free);
         if constexpr (D == 64) {
           if (more) {
@@ -363,7 +369,7 @@ __global__ void __launch_bounds__(384, 1)
       const float* sL = sLD + (s * 2 + 0) * BM;
       const float* sDv = sLD + (s * 2 + 1) * BM;
       // ---- P = exp2(S·c − L·log2e), causal / ragged masking
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[b2], (i >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[b2], (i >> 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
       const uint32_t tS = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
@@ -401,16 +407,16 @@ __global__ void __launch_bounds__(384, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_ready);
+      mbar_arrive(&bars->p_ready[b2]);
 
       // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
       // and to shared memory for the dQ product (row = key, BM query values
       // contiguous, 128-byte swizzled, 64 values per column block).
       ok = __all_sync(0xffffffffu,
-                      mbar_wait(&bars->dp_full[D == 128 ? b2 : 0], (D == 128 ? (i >> 1) : i) & 1,
+                      MBAR_WAIT(&bars->dp_full[D == 128 ? b2 : 0], (D == 128 ? (i >> 1) : i) & 1,
                                 abort_flag));
       if (ok && i > 0)
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->ds_free, (i - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (i - 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
       const uint32_t tDP = tmem + lane_off + (D == 128 && b2 ? Tr::COL_DP1 : Tr::COL_DP0);
@@ -444,7 +450,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_arrive(&bars->ds_ready);
     }
     // ---- dK, dV out (once per CTA)
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->dkv_done, 0, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dkv_done, 0, abort_flag));
     tc_fence_after();
     if (ok) {
       T* dKrow = reinterpret_cast<T*>(p.dK) + (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
@@ -487,7 +493,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int i = 0; i < n_q; ++i) {
       const int b2 = i & 1;
       const int q0 = (i0 + i) * BM;
-      ok = named_bar_and(1, 128, mbar_wait(&bars->dq_full, i & 1, abort_flag));
+      ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full[b2], (i >> 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
       const uint32_t tQ = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
@@ -755,10 +761,18 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
               128 * (Tr::REGS_COMPUTE + Tr::REGS_DQ + Tr::REGS_OTHER);
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
+  if (a.ev_start) {
+    e = cudaEventRecord(a.ev_start, a.stream);
+    if (e != cudaSuccess) return e;
+  }
   kern<<<dim3(p.n_kblocks, p.H, p.B), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV,
                                                                                a.tmdO, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.ev_stop) {
+    e = cudaEventRecord(a.ev_stop, a.stream);
+    if (e != cudaSuccess) return e;
+  }
   bwd_dq_finalise_kernel<T, D, CAUSAL><<<dim3((p.Nq + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
   return cudaGetLastError();
 }

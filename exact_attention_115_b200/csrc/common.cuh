@@ -23,16 +23,22 @@ namespace fa {
 // code is needed); each kernel file exports a host accessor made with
 // FA_ERROR_ACCESSOR that reads and clears it for fa_status.
 static __device__ int g_fa_error = 0;
+// Code of the first wait that timed out (file base + source line), 0 if none.
+static __device__ int g_fa_site = 0;
 
 #define FA_ERROR_ACCESSOR(name)                                                 \
-  cudaError_t name(int* word) {                                                 \
-    int w = 0;                                                                  \
+  cudaError_t name(int* word, int* site) {                                      \
+    int w = 0, st = 0;                                                          \
     cudaError_t e = cudaMemcpyFromSymbol(&w, g_fa_error, sizeof(int));          \
     if (e != cudaSuccess) return e;                                             \
+    e = cudaMemcpyFromSymbol(&st, g_fa_site, sizeof(int));                      \
+    if (e != cudaSuccess) return e;                                             \
     *word |= w;                                                                 \
-    if (w != 0) {                                                               \
+    if (st != 0 && *site == 0) *site = st;                                      \
+    if (w != 0 || st != 0) {                                                    \
       const int z = 0;                                                          \
       e = cudaMemcpyToSymbol(g_fa_error, &z, sizeof(int));                      \
+      if (e == cudaSuccess) e = cudaMemcpyToSymbol(g_fa_site, &z, sizeof(int)); \
     }                                                                           \
     return e;                                                                   \
   }
@@ -88,7 +94,8 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Wait until the phase of `bar` with the given parity has completed.
 // Returns false (and leaves the CTA aborted) on timeout or if the CTA was
 // already aborted by another thread.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          int site = 0) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (uint32_t it = 1;; ++it) {
@@ -98,11 +105,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
       if (globaltimer_ns() - t0 > kWaitLimitNs) {
         *abort_flag = 1;
         atomicOr(&g_fa_error, kErrTimeout);
+        atomicCAS(&g_fa_site, 0, site);
         return false;
       }
     }
   }
 }
+// mbar_wait tagged with the call's source line (plus a per-file base set by
+// FA_SITE_BASE) so a timeout can be traced to its wait.
+#define MBAR_WAIT(bar, parity, abort_flag) mbar_wait(bar, parity, abort_flag, FA_SITE_BASE + __LINE__)
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

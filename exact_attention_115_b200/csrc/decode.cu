@@ -12,6 +12,7 @@
 // of K/V), so it runs on the CUDA cores and is bound by HBM bandwidth: every
 // K/V byte is read exactly once with 16-byte non-allocating loads, several
 // rows in flight per warp.
+#define FA_SITE_BASE 30000
 #include "common.cuh"
 #include "launch.h"
 

@@ -24,6 +24,7 @@
 // only moved when it grows by more than kRescaleThreshold (log2 units), so
 // the O accumulator is rescaled rarely; the result is exact either way
 // because O and ℓ always share the same reference maximum.
+#define FA_SITE_BASE 10000
 #include "common.cuh"
 #include "launch.h"
 
@@ -211,7 +212,7 @@ __global__ void __launch_bounds__(384, 1)
       const int slot = i % Tr::NS;
       bool ok = true;
       if (i >= Tr::NS)
-        ok = mbar_wait(&bars->kv_empty[slot], ((i / Tr::NS) - 1) & 1, abort_flag);
+        ok = MBAR_WAIT(&bars->kv_empty[slot], ((i / Tr::NS) - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
       load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
@@ -225,9 +226,9 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       // Drain: wait until every issued load has landed before the CTA may exit.
       for (int i = max(0, 2 * n_kv - Tr::NS); i < 2 * n_kv; ++i)
-        mbar_wait(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
-      mbar_wait(&bars->q_full[0], 0, abort_flag);
-      mbar_wait(&bars->q_full[1], 0, abort_flag);
+        MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
+      MBAR_WAIT(&bars->q_full[0], 0, abort_flag);
+      MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
@@ -260,14 +261,14 @@ __global__ void __launch_bounds__(384, 1)
         }
       };
       auto kv_wait = [&](int i) {
-        return mbar_wait(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
+        return MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       };
 
-      bool ok = mbar_wait(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+      bool ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
       tc_fence_after();
       if (ok) issue_qk(0, 0);
       tc_commit(&bars->s_full[0]);
-      ok = ok && mbar_wait(&bars->q_full[1], 0, abort_flag);
+      ok = ok && MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
       tc_fence_after();
       if (ok) issue_qk(1, 0);
       tc_commit(&bars->s_full[1]);
@@ -275,7 +276,7 @@ __global__ void __launch_bounds__(384, 1)
       for (int j = 0; j < n_kv && ok; ++j) {
         const int iv = 2 * j + 1, ik = 2 * j + 2;
         const int sv = iv % Tr::NS, sk = ik % Tr::NS;
-        ok = kv_wait(iv) && mbar_wait(&bars->p_full[0], j & 1, abort_flag);
+        ok = kv_wait(iv) && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         issue_pv(0, sv, j > 0);
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(384, 1)
           issue_qk(0, sk);
           tc_commit(&bars->s_full[0]);
         }
-        ok = mbar_wait(&bars->p_full[1], j & 1, abort_flag);
+        ok = MBAR_WAIT(&bars->p_full[1], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         issue_pv(1, sv, j > 0);
@@ -320,7 +321,7 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
 
     for (int j = 0; j < n_kv; ++j) {
-      ok = __all_sync(0xffffffffu, mbar_wait(&bars->s_full[t], j & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
       float s[Tr::BN];
@@ -357,7 +358,7 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (j > 0 && __any_sync(0xffffffffu, upd)) {
         // Correction: O (which holds tiles < j) moves onto the new maximum.
-        ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], (j - 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->o_full[t], (j - 1) & 1, abort_flag));
         tc_fence_after();
         if (!ok) break;
 #pragma unroll 1
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(384, 1)
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
+    if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
     tc_fence_after();
     if (ok) {
       const float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;

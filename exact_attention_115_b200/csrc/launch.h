@@ -52,6 +52,7 @@ struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmdO;
   BwdParams params;
   cudaStream_t stream;
+  cudaEvent_t ev_start, ev_stop;  // optional timing events around the main kernel
 };
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a);
@@ -73,9 +74,9 @@ struct DecodeParams {
 cudaError_t launch_decode(int dtype, int d, const DecodeParams& p, cudaStream_t s);
 
 // Read-and-clear accessors of each kernel file's device error word.
-cudaError_t take_error_fwd(int* word);
-cudaError_t take_error_bwd(int* word);
-cudaError_t take_error_decode(int* word);
+cudaError_t take_error_fwd(int* word, int* site);
+cudaError_t take_error_bwd(int* word, int* site);
+cudaError_t take_error_decode(int* word, int* site);
 
 // Sets the dynamic shared-memory limit of `kernel` on the current device once.
 cudaError_t set_smem_once(const void* kernel, int bytes);

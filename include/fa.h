@@ -105,6 +105,20 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
  * the stream reports a CUDA error. */
 int fa_status(void* stream);
 
+/* Diagnostic: identifies the first kernel wait that timed out among those
+ * fa_status has reported (10000 + line in the forward kernel file, 20000 +
+ * line in the backward file); 0 if none has.  No counterpart on the pages. */
+int fa_last_timeout_site(void);
+
+/* Measurement hook (no counterpart on the pages, which only say to profile
+ * kernels with Nsight Compute, 51CTO notes, section "FlashAttention V2相比V1有
+ * 哪些改进").  When both are non-NULL, every later fa_bwd call records the
+ * cudaEvent_t `start` on its stream just before the main backward kernel and
+ * `stop` just after it, so callers can time that kernel alone with
+ * cudaEventElapsedTime.  The events are created and owned by the caller.
+ * Pass NULLs to switch it off.  Process-wide; returns FA_OK. */
+int fa_bwd_set_timing_events(void* start, void* stop);
+
 /* Library version string (static storage). */
 const char* fa_version(void);
 
