@@ -49,6 +49,37 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def kernel_traffic(kernel: str, sources):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since that capture (hash mismatch)."""
+    import hashlib
+
+    try:
+        with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
+            rec = json.load(f)[kernel]
+    except (OSError, KeyError, ValueError):
+        return None
+    m = hashlib.sha256()
+    for p in sources:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            m.update(f.read())
+    return rec["bytes_per_launch"] if m.hexdigest() == rec["source_sha256"] else None
+
+
+def reduce_max(x: float, pg, device) -> float:
+    """Max of a per-rank float over all ranks (identity without a group)."""
+    if pg is None:
+        return float(x)
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_workload(w, rank: int):
+    """Each rank runs its own replica of the workload, drawn from its own seed."""
+    return W.Workload(**{**w.__dict__, "seed": w.seed + rank})
+
+
 def dist_info():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -188,7 +219,7 @@ def main():
     peaks, peak_kind = load_peaks()
     stream = torch.cuda.current_stream(dev)
 
-    q, k, v, do = W.make_inputs(W.Workload(**{**w.__dict__, "seed": w.seed + rank}), device=dev)
+    q, k, v, do = W.make_inputs(rank_workload(w, rank), device=dev)
     O, L = fa.forward(q, k, v, causal=True)
     dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
     ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d), dtype=torch.uint8,
@@ -246,10 +277,7 @@ def main():
     fwd_ms = [ev["s0"][i].elapsed_time(ev["f1"][i]) for i in range(K)]
     bwd_main_ms = [ev["b0"][i].elapsed_time(ev["b1"][i]) for i in range(K)]
     bwd_ms = [ev["f1"][i].elapsed_time(ev["s1"][i]) for i in range(K)]
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if pg:
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-    total_ms = float(t.item())
+    total_ms = reduce_max(total_ms, pg, dev)
     ms_per_step = total_ms / K
     flops_step = w.fwd_flops + w.bwd_flops
     value = flops_step * K * world / (total_ms * 1e-3) / 1e12
@@ -288,10 +316,8 @@ def main():
             e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
-        et = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if pg:
-            pg.all_reduce(et, op=pg.ReduceOp.MAX)
-        e2e = {"value": flops_step * ksteps * world / (float(et.item()) * 1e-3) / 1e12,
+        et = reduce_max(a.elapsed_time(b), pg, dev)
+        e2e = {"value": flops_step * ksteps * world / (et * 1e-3) / 1e12,
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ksteps}
 
@@ -351,7 +377,11 @@ def main():
         "pct_of_peak": value / world / peak_burst,
         "roofline": {"bound": "tensor", "kernel": "bwd_main_kernel", "achieved": achieved_bwd,
                      "peak": peak_burst, "unit": "TFLOP/s", "frac": achieved_bwd / peak_burst,
-                     "peak_kind": f"{peak_kind} burst bf16", "traffic": None},
+                     "peak_kind": f"{peak_kind} burst bf16",
+                     "traffic": kernel_traffic("bwd_main_kernel", (
+                         "exact_attention_115_b200/csrc/bwd.cu",
+                         "exact_attention_115_b200/csrc/common.cuh")),
+                     "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": e2e,
         "gpu_launches": 4 * K,
         "clocks": clocks,
