@@ -27,11 +27,15 @@
 // round trip).  dSᵀ also goes to shared memory for the dQ product:
 //   d = 128: BM = 64 query rows per step, dQᵀ = Kᵀ dSᵀ (M = d = 128);
 //   d = 64:  BM = 128, dQ = dS K (M = BM = 128).
-// Roles (384 threads):
-//   warpgroup 0: thread = key row: P, dS, and the final dK/dV store;
-//   warpgroup 1: reads dQ from TMEM, stages it in shared memory, issues the
+// Roles (512 threads):
+//   warpgroups 0 and 1: thread = key row; warpgroup c computes P and dS for
+//                half of each step's query columns, and writes half of the
+//                final dK/dV columns;
+//   warpgroup 2: reads dQ from TMEM, stages it in shared memory, issues the
 //                bulk reduction (or partial store);
-//   warp 8: tcgen05.mma issuer, TMEM owner; warp 9: TMA producer.
+//   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: TMA producer.
+// The dSᵀ shared-memory tile is double buffered, so step i's dS is written
+// while step i-1's dQ product still reads the other buffer.
 // TMEM (512 columns), d = 128: Sᵀ[2] | dPᵀ[2] | dV | dK (64,64,64,64,128,128);
 //                    d = 64:  Sᵀ[2] | dPᵀ | dV | dK (128,128,128,64,64).
 // Sᵀ is double buffered so the next step's Sᵀ MMA runs while the current
@@ -94,6 +98,7 @@ struct BwdTraits {
   static constexpr int ES = 2;
   static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
   static constexpr int BM = D == 128 ? 64 : 128;     // query rows per step
+  static constexpr int CWC = BM / 2;                 // query columns per compute warpgroup
   static constexpr bool DQ_T = D == 128;             // dQᵀ = Kᵀ dSᵀ (else dQ = dS K)
   static constexpr int NSTG = 2;                     // Q/dO pipeline stages
   static constexpr int KV_TILE = BN * D * ES;        // bytes of the K (or V) tile
@@ -107,8 +112,8 @@ struct BwdTraits {
   static constexpr int OFF_V = OFF_K + KV_TILE;
   static constexpr int OFF_Q = OFF_V + KV_TILE;
   static constexpr int OFF_DO = OFF_Q + NSTG * Q_TILE;
-  static constexpr int OFF_DS = OFF_DO + NSTG * Q_TILE;
-  static constexpr int OFF_DQ = OFF_DS + DS_TILE;
+  static constexpr int OFF_DS = OFF_DO + NSTG * Q_TILE;   // two dSᵀ buffers
+  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;
   static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;        // L·log2e and D per stage
   static constexpr int OFF_BAR = OFF_LD + NSTG * 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
@@ -120,15 +125,29 @@ struct BwdTraits {
   static constexpr int COL_DV = D == 128 ? 4 * BM : 3 * BM;
   static constexpr int COL_DK = COL_DV + D;
   static_assert(COL_DK + D <= 512, "TMEM budget");
-  static constexpr int THREADS = 384;
-  static constexpr int REGS_COMPUTE = 232;
-  static constexpr int REGS_DQ = 120;
-  static constexpr int REGS_OTHER = 56;
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared-memory budget");
+  static constexpr int THREADS = 512;
+  // No setmaxnreg: every warp keeps the 128 registers per thread it is
+  // launched with (the compute code works in 32-column chunks to fit).
   static constexpr uint32_t F = ElemTraits<T>::fmt;
   static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
   static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV, dK (A in TMEM)
   static constexpr uint32_t IDESC_DQ = make_idesc(F, 128, DQ_T ? BM : D, 1, 1);
 };
+
+#ifdef FA_TRACE
+// One fixed slot per event code (plain stores; no atomics on the critical path).
+__device__ long long g_btrace[16384];
+__device__ __forceinline__ void btrace(bool on, int code) {
+  if (!on || code >= 16384) return;
+  long long t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  g_btrace[code] = t;
+}
+#define BTRACE(code) btrace(trace_on, (code))
+#else
+#define BTRACE(code) ((void)0)
+#endif
 
 struct BwdBarriers {
   uint64_t kv_full;
@@ -136,15 +155,15 @@ struct BwdBarriers {
   uint64_t qdo_empty[2];
   uint64_t s_full[2];
   uint64_t dp_full[2];
-  // One barrier per Sᵀ buffer for the signals whose producer can otherwise
-  // run two phases ahead of a parity wait (the next step's Sᵀ is already
-  // there, or the last step skips the back-pressure wait).
+  // One barrier per buffer for every signal whose producer could otherwise
+  // run two phases ahead of a parity wait.
   uint64_t p_ready[2];
   uint64_t ds_ready;
   uint64_t dq_full[2];
-  uint64_t dq_empty;
-  uint64_t ds_free;
+  uint64_t dq_empty[2];
+  uint64_t ds_free[2];
   uint64_t dkv_done;
+  uint64_t watch;  // trace builds only
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -160,13 +179,35 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
   n = max(0, nt - i0);
 }
 
+// Load / store N (16, 32 or 64) consecutive TMEM columns of this warp's lanes.
+template <int N>
+__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 16) {
+    tmem_ld16(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 32) tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
+  }
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 16) {
+    tmem_st16(taddr, r);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N; c += 32)
+      tmem_st32(taddr + c, *reinterpret_cast<const uint32_t(*)[32]>(r + c));
+  }
+}
+
 template <typename T, int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     BwdParams p) {
   using Tr = BwdTraits<T, D>;
   constexpr int BM = Tr::BM;
+  constexpr int CWC = Tr::CWC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -180,6 +221,9 @@ __global__ void __launch_bounds__(384, 1)
   const int off = p.Nk - p.Nq;
   int i0, n_q;
   q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
+#ifdef FA_TRACE
+  const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+#endif
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
@@ -188,23 +232,23 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->qdo_empty[s], 1);
       mbar_init(&bars->s_full[s], 1);
       mbar_init(&bars->dp_full[s], 1);
+      mbar_init(&bars->p_ready[s], 256);
+      mbar_init(&bars->dq_full[s], 1);
+      mbar_init(&bars->ds_free[s], 1);
     }
-    mbar_init(&bars->p_ready[0], 128);
-    mbar_init(&bars->p_ready[1], 128);
-    mbar_init(&bars->ds_ready, 128);
-    mbar_init(&bars->dq_full[0], 1);
-    mbar_init(&bars->dq_full[1], 1);
-    mbar_init(&bars->dq_empty, 128);
-    mbar_init(&bars->ds_free, 1);
+    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->dq_empty[0], 128);
+    mbar_init(&bars->dq_empty[1], 128);
     mbar_init(&bars->dkv_done, 1);
+    mbar_init(&bars->watch, 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == 13 && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -223,11 +267,17 @@ __global__ void __launch_bounds__(384, 1)
   float* sdQ = reinterpret_cast<float*>(smem + Tr::OFF_DQ);
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
 
-  if (warp >= 10) {
-    regs_dec<Tr::REGS_OTHER>();
-  } else if (warp == 9) {
+  if (warp >= 14) {
+#ifdef FA_TRACE
+    if (warp == 14 && lane == 0 && trace_on) {
+      for (int g = 0; g < n_q; ++g) {
+        if (!MBAR_WAIT(&bars->watch, g & 1, abort_flag)) break;
+        btrace(true, 10000 + g);  // all MMAs of step g complete
+      }
+    }
+#endif
+  } else if (warp == 13) {
     // ------------------------------------------------------------ producer
-    regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars->kv_full, 2 * Tr::KV_TILE);
 #pragma unroll
@@ -257,9 +307,8 @@ __global__ void __launch_bounds__(384, 1)
         MBAR_WAIT(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
       MBAR_WAIT(&bars->kv_full, 0, abort_flag);
     }
-  } else if (warp == 8) {
+  } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
-    regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
@@ -267,37 +316,49 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t colDP[2] = {tmem + Tr::COL_DP0, tmem + Tr::COL_DP1};
       const uint32_t colDV = tmem + Tr::COL_DV, colDK = tmem + Tr::COL_DK;
 
+      // Operand descriptors are built once; inside the unrolled loops each
+      // MMA only adds a compile-time offset (16-byte units), so the issuing
+      // thread keeps ahead of the tensor core.
+      const uint64_t dK_k = sw128_desc(aK, 16, 1024), dV_k = sw128_desc(aV, 16, 1024);
+      const uint64_t dK_mn = sw128_desc(aK, Tr::KV_CHUNK, 1024);
+      // Stage / buffer s of a tile lives s * (tile bytes) further on: add
+      // that (in 16-byte units) to the stage-0 descriptor.
+      const uint64_t dQ_k0 = sw128_desc(aQ, 16, 1024), dO_k0 = sw128_desc(adO, 16, 1024);
+      const uint64_t dQ_mn0 = sw128_desc(aQ, Tr::Q_CHUNK, 1024);
+      const uint64_t dO_mn0 = sw128_desc(adO, Tr::Q_CHUNK, 1024);
+      const uint64_t dS_mn0 = sw128_desc(adS, Tr::BN * 128, 1024);
+      auto stg = [](uint64_t d0, int s, int bytes) { return d0 + uint64_t(s) * uint64_t(bytes >> 4); };
+
       // Sᵀ (or dPᵀ) = X[128 keys × D] · Y[BM × D]ᵀ, both K-major.
-      auto mma_st = [&](uint32_t dcol, uint32_t aX, uint32_t aY) {
+      auto mma_st = [&](uint32_t dcol, uint64_t dx, uint64_t dy) {
 #pragma unroll
         for (int ks = 0; ks < D / 16; ++ks) {
-          const uint32_t oa = (ks >> 2) * Tr::KV_CHUNK + (ks & 3) * 32;
-          const uint32_t ob = (ks >> 2) * Tr::Q_CHUNK + (ks & 3) * 32;
-          mma_ss<false>(dcol, sw128_desc(aX + oa, 16, 1024), sw128_desc(aY + ob, 16, 1024),
-                        Tr::IDESC_ST, ks > 0);
+          const uint64_t oa = uint64_t((ks >> 2) * (Tr::KV_CHUNK / 16) + (ks & 3) * 2);
+          const uint64_t ob = uint64_t((ks >> 2) * (Tr::Q_CHUNK / 16) + (ks & 3) * 2);
+          mma_ss<false>(dcol, dx + oa, dy + ob, Tr::IDESC_ST, ks > 0);
         }
       };
       // dV or dK [128 × D] += A[128 × BM] (TMEM) · Y[BM × D] (MN-major).
-      auto mma_grad = [&](uint32_t dcol, uint32_t acol, uint32_t aY, bool acc) {
+      // A (Pᵀ or dSᵀ, bf16 pairs) was written by the two compute
+      // warpgroups, each into the first half of the columns it had read, so
+      // k-step ks sits at column (ks / kPerWg)·CWC + (ks % kPerWg)·8.
+      auto mma_grad = [&](uint32_t dcol, uint32_t acol, uint64_t dy, bool acc) {
+        constexpr int kPerWg = CWC / 16;
 #pragma unroll
         for (int ks = 0; ks < BM / 16; ++ks)
-          mma_ts<false>(dcol, acol + ks * 8, sw128_desc(aY + ks * 2048, Tr::Q_CHUNK, 1024),
-                        Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
+          mma_ts<false>(dcol, acol + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
+                        dy + uint64_t(ks * 128), Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
       };
       // dQᵀ [D × BM] = Kᵀ · dSᵀ  (d = 128), or dQ [BM × D] = dS · K (d = 64);
       // both operands MN-major, K dimension = the 128 keys.
-      auto mma_dq = [&](uint32_t dcol) {
+      auto mma_dq = [&](uint32_t dcol, uint64_t dds) {
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / 16; ++ks) {
-          uint64_t da, db;
-          if constexpr (Tr::DQ_T) {
-            da = sw128_desc(aK + ks * 2048, Tr::KV_CHUNK, 1024);
-            db = sw128_desc(adS + ks * 2048, Tr::BN * 128, 1024);
-          } else {
-            da = sw128_desc(adS + ks * 2048, Tr::BN * 128, 1024);
-            db = sw128_desc(aK + ks * 2048, Tr::KV_CHUNK, 1024);
-          }
-          mma_ss<false>(dcol, da, db, Tr::IDESC_DQ, ks > 0);
+          const uint64_t o = uint64_t(ks * 128);
+          if constexpr (Tr::DQ_T)
+            mma_ss<false>(dcol, dK_mn + o, dds + o, Tr::IDESC_DQ, ks > 0);
+          else
+            mma_ss<false>(dcol, dds + o, dK_mn + o, Tr::IDESC_DQ, ks > 0);
         }
       };
       auto qwait = [&](int i) {
@@ -307,106 +368,150 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = MBAR_WAIT(&bars->kv_full, 0, abort_flag) && (n_q == 0 || qwait(0));
       tc_fence_after();
       if (ok && n_q > 0) {
-        mma_st(colS[0], aK, aQ);
+        mma_st(colS[0], dK_k, dQ_k0);
         tc_commit(&bars->s_full[0]);
-        mma_st(colDP[0], aV, adO);
+        mma_st(colDP[0], dV_k, dO_k0);
         tc_commit(&bars->dp_full[0]);
       }
       for (int i = 0; i < n_q && ok; ++i) {
         const int s = i % Tr::NSTG, b2 = i & 1;
-        const uint32_t aQs = aQ + s * Tr::Q_TILE, adOs = adO + s * Tr::Q_TILE;
         const bool more = i + 1 < n_q;
-        // Next step's Sᵀ into the other buffer (its previous dQ must have
-        // been read by the dQ warpgroup).
-        if (more) {
-          ok = qwait(i + 1) && (i < 1 || MBAR_WAIT(&bars->dq_empty, (i - 1) & 1, abort_flag));
+        const int s1 = (i + 1) % Tr::NSTG;
+        if constexpr (D == 128) {
+          // d = 128: dQᵀ of step i goes to dPᵀ[i % 2] once the dK product
+          // has read dSᵀ from there.  Order per step: the next Sᵀ (its
+          // buffer is free: Pᵀ of step i-1 was consumed last step), dV, dK,
+          // dQ of this step, and last the next dPᵀ, whose buffer held dQ of
+          // step i-1 and must first be drained by the dQ warpgroup; a whole
+          // step has passed since that dQ was produced, so this rarely waits.
+          if (more) {
+            ok = qwait(i + 1);
+            tc_fence_after();
+            if (!ok) break;
+            mma_st(colS[b2 ^ 1], dK_k, stg(dQ_k0, s1, Tr::Q_TILE));
+            tc_commit(&bars->s_full[b2 ^ 1]);
+          }
+          BTRACE(1000 + i);
+          ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          const int s1 = (i + 1) % Tr::NSTG;
-          mma_st(colS[b2 ^ 1], aK, aQ + s1 * Tr::Q_TILE);
-          tc_commit(&bars->s_full[b2 ^ 1]);
-          if constexpr (D == 128) {
-            mma_st(colDP[b2 ^ 1], aV, adO + s1 * Tr::Q_TILE);
+          BTRACE(2000 + i);
+          mma_grad(colDV, colS[b2], stg(dO_mn0, s, Tr::Q_TILE), i > 0);
+          BTRACE(3000 + i);
+          ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          BTRACE(4000 + i);
+          mma_grad(colDK, colDP[b2], stg(dQ_mn0, s, Tr::Q_TILE), i > 0);
+          tc_commit(&bars->qdo_empty[s]);
+          if (!more) tc_commit(&bars->dkv_done);
+          mma_dq(colDP[b2], stg(dS_mn0, b2, Tr::DS_TILE));
+          tc_commit(&bars->dq_full[b2]);
+          tc_commit(&bars->ds_free[b2]);
+          BTRACE(5000 + i);
+#ifdef FA_TRACE
+          if (trace_on) tc_commit(&bars->watch);
+#endif
+          if (more) {
+            ok = i < 1 || MBAR_WAIT(&bars->dq_empty[b2 ^ 1], ((i - 1) >> 1) & 1, abort_flag);
+            tc_fence_after();
+            if (!ok) break;
+            mma_st(colDP[b2 ^ 1], dV_k, stg(dO_k0, s1, Tr::Q_TILE));
             tc_commit(&bars->dp_full[b2 ^ 1]);
           }
-        }
-        ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
-        tc_fence_after();
-        if (!ok) break;
-        mma_grad(colDV, colS[b2], adOs, i > 0);
-        ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
-        tc_fence_after();
-        if (!ok) break;
-        mma_grad(colDK, colDP[D == 128 ? b2 : 0], aQs, i > 0);
-        tc_commit(&bars->qdo_empty[s]);
-        if (!more) tc_commit(&bars->dkv_done);
-        mma_dq(colS[b2]);
-        tc_commit(&bars->dq_full[b2]);
-        tc_commit(&bars->ds_free);
-        if constexpr (D == 64) {
+        } else {
+          // d = 64: dQ of step i goes to Sᵀ[i % 2]; the next Sᵀ needs the dQ
+          // of step i-1 drained from its buffer.
           if (more) {
-            mma_st(colDP[0], aV, adO + ((i + 1) % Tr::NSTG) * Tr::Q_TILE);
+            ok = qwait(i + 1) &&
+                 (i < 1 || MBAR_WAIT(&bars->dq_empty[b2 ^ 1], ((i - 1) >> 1) & 1, abort_flag));
+            tc_fence_after();
+            if (!ok) break;
+            mma_st(colS[b2 ^ 1], dK_k, stg(dQ_k0, s1, Tr::Q_TILE));
+            tc_commit(&bars->s_full[b2 ^ 1]);
+          }
+          ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          mma_grad(colDV, colS[b2], stg(dO_mn0, s, Tr::Q_TILE), i > 0);
+          ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          mma_grad(colDK, colDP[0], stg(dQ_mn0, s, Tr::Q_TILE), i > 0);
+          tc_commit(&bars->qdo_empty[s]);
+          if (!more) tc_commit(&bars->dkv_done);
+          mma_dq(colS[b2], stg(dS_mn0, b2, Tr::DS_TILE));
+          tc_commit(&bars->dq_full[b2]);
+          tc_commit(&bars->ds_free[b2]);
+          if (more) {
+            mma_st(colDP[0], dV_k, stg(dO_k0, s1, Tr::Q_TILE));
             tc_commit(&bars->dp_full[0]);
           }
         }
       }
       if (n_q == 0) tc_commit(&bars->dkv_done);
     }
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P / dS (thread = key)
-    regs_inc<Tr::REGS_COMPUTE>();
-    const int quad = warp;
+    // Two warpgroups; warpgroup cw handles query columns [cw·CWC, (cw+1)·CWC)
+    // of each step for all 128 key rows.
+    const int cw = warp >> 2;
+    const int quad = warp & 3;
     const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
     const int key = key0 + kr;
     const bool key_live = key < p.Nk;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const float sl2 = p.scale_log2;
     const float scale = p.scale;
+    const int qmin = key - off;  // first query row that sees this key
     bool ok = true;
     for (int i = 0; i < n_q; ++i) {
       const int s = i % Tr::NSTG, b2 = i & 1;
-      const int q0 = (i0 + i) * BM;
-      const float* sL = sLD + (s * 2 + 0) * BM;
-      const float* sDv = sLD + (s * 2 + 1) * BM;
+      const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
+      const float* sL = sLD + (s * 2 + 0) * BM + cw * CWC;
+      const float* sDv = sLD + (s * 2 + 1) * BM + cw * CWC;
       // ---- P = exp2(S·c − L·log2e), causal / ragged masking
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[b2], (i >> 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
+#ifdef FA_TRACE
+      btrace(trace_on && quad == 0 && lane == 0, 6000 + 100 * cw + i);  // compute got S
+#endif
       const uint32_t tS = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
-      // A key sees query q iff key <= q + off; keys past Nk contribute nothing.
       const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
-      const int qmin = key - off;  // first query row that sees this key
-      float P[BM];
+      float P[CWC];
       const uint64_t c2 = pk2(sl2, sl2);
-      // Processed 64 columns at a time: Pᵀ is packed to bf16 pairs and stored
-      // straight back to TMEM; the fp32 P stays in registers for dS.
+      // 32 columns at a time: load, exponentiate, pack to bf16 pairs, store
+      // Pᵀ back to TMEM into the columns this warpgroup has already read (the
+      // other warpgroup may still be reading its own half); the fp32 P stays
+      // in registers for dS.
 #pragma unroll
-      for (int c = 0; c < BM; c += 64) {
-        uint32_t w[32];
+      for (int c = 0; c < CWC; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tS + cw * CWC + c, u);
+        tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-        for (int h = 0; h < 64; h += 32) {
-          uint32_t u[32];
-          tmem_ld32(tS + c + h, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int q = c + h + e;
-            const float2 x = upk2(ffma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
-                                        pk2(-sL[q], -sL[q + 1])));
-            float p0 = ex2(x.x), p1 = ex2(x.y);
-            if (need_mask) {
-              if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
-              if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
-            }
-            P[q] = p0;
-            P[q + 1] = p1;
-            w[(h + e) / 2] = ElemTraits<T>::pack2(p0, p1);
+        for (int e = 0; e < 32; e += 2) {
+          const int q = c + e;
+          const float2 x = upk2(ffma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
+                                      pk2(-sL[q], -sL[q + 1])));
+          float p0 = ex2(x.x), p1 = ex2(x.y);
+          if (need_mask) {
+            if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
+            if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
           }
+          P[q] = p0;
+          P[q + 1] = p1;
+          w[e / 2] = ElemTraits<T>::pack2(p0, p1);
         }
-        tmem_st32(tS + c / 2, w);
+        tmem_st16(tS + cw * CWC + c / 2, w);
       }
       tmem_st_wait();
       tc_fence_before();
+#ifdef FA_TRACE
+      btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // P done
+#endif
       mbar_arrive(&bars->p_ready[b2]);
 
       // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
@@ -415,80 +520,80 @@ __global__ void __launch_bounds__(384, 1)
       ok = __all_sync(0xffffffffu,
                       MBAR_WAIT(&bars->dp_full[D == 128 ? b2 : 0], (D == 128 ? (i >> 1) : i) & 1,
                                 abort_flag));
-      if (ok && i > 0)
-        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (i - 1) & 1, abort_flag));
+      if (ok && i >= 2)
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free[b2], ((i - 2) >> 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
       const uint32_t tDP = tmem + lane_off + (D == 128 && b2 ? Tr::COL_DP1 : Tr::COL_DP0);
+      uint8_t* buf = sdS + b2 * Tr::DS_TILE;
+      const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
-      for (int c = 0; c < BM; c += 64) {
-        uint32_t w[32];
+      for (int c = 0; c < CWC; c += 32) {
+        uint32_t u[32];
+        tmem_ld32(tDP + cw * CWC + c, u);
+        tmem_ld_wait();
+        uint32_t w[16];
 #pragma unroll
-        for (int h = 0; h < 64; h += 32) {
-          uint32_t u[32];
-          tmem_ld32(tDP + c + h, u);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int q = c + h + e;
-            const uint64_t t = fadd2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])),
-                                     pk2(-sDv[q], -sDv[q + 1]));
-            const float2 ds = upk2(fmul2(t, pk2(P[q] * scale, P[q + 1] * scale)));
-            w[(h + e) / 2] = ElemTraits<T>::pack2(ds.x, ds.y);
-          }
+        for (int e = 0; e < 32; e += 2) {
+          const int q = c + e;
+          const uint64_t t = fadd2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])),
+                                   pk2(-sDv[q], -sDv[q + 1]));
+          const float2 ds = upk2(fmul2(t, fmul2(pk2(P[q], P[q + 1]), sc2)));
+          w[e / 2] = ElemTraits<T>::pack2(ds.x, ds.y);
         }
-        tmem_st32(tDP + c / 2, w);
-        uint8_t* rowp = sdS + (c / 64) * (Tr::BN * 128) + kr * 128;
+        tmem_st16(tDP + cw * CWC + c / 2, w);
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch)
-          *reinterpret_cast<uint4*>(rowp + ((ch ^ (kr & 7)) << 4)) =
-              make_uint4(w[ch * 4], w[ch * 4 + 1], w[ch * 4 + 2], w[ch * 4 + 3]);
+        for (int c16 = 0; c16 < 4; ++c16) {
+          const int col = cw * CWC + c + c16 * 8;  // first query column of this 16-byte chunk
+          const int blk = col >> 6, ch = (col >> 3) & 7;
+          *reinterpret_cast<uint4*>(buf + blk * (Tr::BN * 128) + kr * 128 + ((ch ^ (kr & 7)) << 4)) =
+              make_uint4(w[c16 * 4], w[c16 * 4 + 1], w[c16 * 4 + 2], w[c16 * 4 + 3]);
+        }
       }
       fence_async_smem();
       tmem_st_wait();
       tc_fence_before();
+#ifdef FA_TRACE
+      btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
+#endif
       mbar_arrive(&bars->ds_ready);
     }
-    // ---- dK, dV out (once per CTA)
+    // ---- dK, dV out (once per CTA); warpgroup cw writes columns [cw·D/2, (cw+1)·D/2)
     if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dkv_done, 0, abort_flag));
     tc_fence_after();
     if (ok) {
-      T* dKrow = reinterpret_cast<T*>(p.dK) + (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
-      T* dVrow = reinterpret_cast<T*>(p.dV) + (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
+      const size_t rowoff = (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
 #pragma unroll 1
       for (int which = 0; which < 2; ++which) {
-        const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV);
-        T* out = which ? dKrow : dVrow;
+        const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV) + cw * (D / 2);
+        T* out = reinterpret_cast<T*>(which ? p.dK : p.dV) + rowoff + cw * (D / 2);
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D / 2; c += 32) {
           uint32_t u[32];
           tmem_ld32(tcol + c, u);
           tmem_ld_wait();
-          if (key_live && n_q > 0) {
+          if (key_live) {
 #pragma unroll
             for (int e = 0; e < 32; e += 8) {
-              uint4 v;
-              v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]), __uint_as_float(u[e + 1]));
-              v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
-              v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]), __uint_as_float(u[e + 5]));
-              v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]), __uint_as_float(u[e + 7]));
+              uint4 v = make_uint4(0, 0, 0, 0);
+              if (n_q > 0) {
+                v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]), __uint_as_float(u[e + 1]));
+                v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
+                v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]), __uint_as_float(u[e + 5]));
+                v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]), __uint_as_float(u[e + 7]));
+              }
               *reinterpret_cast<uint4*>(out + c + e) = v;
             }
-          } else if (key_live) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8)
-              *reinterpret_cast<uint4*>(out + c + e) = make_uint4(0, 0, 0, 0);
           }
         }
       }
     }
   } else {
-    // ------------------------------------------------------------ dQ (warpgroup 1)
-    regs_dec<Tr::REGS_DQ>();
+    // ------------------------------------------------------------ dQ (warpgroup 2)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane: d index (dQᵀ) or query row (dQ)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const bool leader = (warp == 4 && lane == 0);
+    const bool leader = (warp == 8 && lane == 0);
     bool ok = true;
     for (int i = 0; i < n_q; ++i) {
       const int b2 = i & 1;
@@ -496,26 +601,25 @@ __global__ void __launch_bounds__(384, 1)
       ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full[b2], (i >> 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
-      const uint32_t tQ = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
+#ifdef FA_TRACE
+      btrace(trace_on && leader, 9000 + i);  // dQ ready seen
+#endif
+      // dQ of step i: dPᵀ[i % 2] for d = 128, Sᵀ[i % 2] for d = 64
+      const uint32_t tQ = tmem + lane_off +
+                          (D == 128 ? (b2 ? Tr::COL_DP1 : Tr::COL_DP0) : (b2 ? Tr::COL_S1 : Tr::COL_S0));
       constexpr int NV = Tr::DQ_T ? BM : D;  // values per thread
-      float v[NV];
-#pragma unroll
-      for (int c = 0; c < NV; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tQ + c, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[c + e] = __uint_as_float(u[e]);
-      }
+      uint32_t v[NV];
+      tmem_ld_n<NV>(tQ, v);
+      tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars->dq_empty);
+      mbar_arrive(&bars->dq_empty[b2]);
       // The previous bulk operation must have finished reading the staging buffer.
       if (leader) bulk_wait_read0();
       named_bar(1, 128);
       if constexpr (Tr::DQ_T) {
         // thread = d index r; staging is [BM][D] row-major fp32
 #pragma unroll
-        for (int q = 0; q < BM; ++q) sdQ[q * D + r] = v[q];
+        for (int q = 0; q < BM; ++q) sdQ[q * D + r] = __uint_as_float(v[q]);
       } else {
         // thread = query row r; write its D values, rotating the 16-byte
         // chunk order by lane to spread shared-memory banks
@@ -523,10 +627,10 @@ __global__ void __launch_bounds__(384, 1)
         for (int cc = 0; cc < D / 4; ++cc) {
           const int c4 = (cc + lane) % (D / 4);
           float4 x;
-          x.x = v[c4 * 4 + 0];
-          x.y = v[c4 * 4 + 1];
-          x.z = v[c4 * 4 + 2];
-          x.w = v[c4 * 4 + 3];
+          x.x = __uint_as_float(v[c4 * 4 + 0]);
+          x.y = __uint_as_float(v[c4 * 4 + 1]);
+          x.z = __uint_as_float(v[c4 * 4 + 2]);
+          x.w = __uint_as_float(v[c4 * 4 + 3]);
           *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
         }
       }
@@ -548,7 +652,7 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -752,15 +856,6 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   auto kern = bwd_main_kernel<T, D, CAUSAL>;
   e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  static int regs_ok = -1;
-  if (regs_ok < 0) {
-    cudaFuncAttributes attr;
-    e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
-    if (e != cudaSuccess) return e;
-    regs_ok = attr.numRegs * Tr::THREADS >=
-              128 * (Tr::REGS_COMPUTE + Tr::REGS_DQ + Tr::REGS_OTHER);
-  }
-  if (!regs_ok) return cudaErrorInvalidConfiguration;
   if (a.ev_start) {
     e = cudaEventRecord(a.ev_start, a.stream);
     if (e != cudaSuccess) return e;
@@ -797,5 +892,17 @@ cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
 }
 
 FA_ERROR_ACCESSOR(take_error_bwd)
+
+#ifdef FA_TRACE
+}  // namespace fa
+extern "C" int fa_btrace_read(long long* out, int max) {
+  const int n = max < 16384 ? max : 16384;
+  cudaMemcpyFromSymbol(out, fa::g_btrace, sizeof(long long) * n);
+  static long long zeros[16384];
+  cudaMemcpyToSymbol(fa::g_btrace, zeros, sizeof(zeros));
+  return n;
+}
+namespace fa {
+#endif
 
 }  // namespace fa

@@ -60,6 +60,21 @@ struct FwdTraits {
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
 
+#ifdef FA_TRACE
+// One fixed slot per event code (no atomics: a plain store does not stall).
+__device__ long long g_trace[16384][2];
+__device__ int g_trace_n;
+__device__ __forceinline__ void trace_ev(bool on, int code) {
+  if (!on) return;
+  long long t;
+  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
+  if (code < 16384) { g_trace[code][0] = code; g_trace[code][1] = t; }
+}
+#define TRACE(code) trace_ev(trace_on, (code))
+#else
+#define TRACE(code) ((void)0)
+#endif
+
 struct FwdBarriers {
   uint64_t q_full[2];
   uint64_t s_full[2];
@@ -75,6 +90,40 @@ __device__ __forceinline__ float round_tf32(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
+}
+
+#ifndef FA_EXP2_EMU_PERIOD
+#define FA_EXP2_EMU_PERIOD 4
+#endif
+// One pair in every kEmuPeriod evaluates 2^x on the FMA pipe (exp2_pair<true>)
+// instead of the special-function unit, to balance the two pipes.
+constexpr int kEmuPeriod = FA_EXP2_EMU_PERIOD;
+
+// 2^x for a pair of floats on the FMA/ALU pipes: x = n + f with n = round(x)
+// (via the 1.5·2^23 rounding constant), f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial with minimal maximum relative error (1.0e-4; coefficients from
+// gen_exp2_poly.py); 2^n added to the exponent field.  x is clamped at -125
+// so masked (-inf) scores give ~2^-125 instead of a wrapped exponent.
+template <bool EMU>
+__device__ __forceinline__ float2 exp2_pair(uint64_t x2) {
+  if constexpr (!EMU) {
+    const float2 x = upk2(x2);
+    return make_float2(ex2(x.x), ex2(x.y));
+  } else {
+    float2 x = upk2(x2);
+    x.x = fmaxf(x.x, -125.f);
+    x.y = fmaxf(x.y, -125.f);
+    const uint64_t magic = pk2(12582912.f, 12582912.f);
+    const uint64_t t = fadd2(pk2(x.x, x.y), magic);
+    const uint64_t n = fadd2(t, pk2(-12582912.f, -12582912.f));
+    const uint64_t f = ffma2(n, pk2(-1.f, -1.f), pk2(x.x, x.y));
+    uint64_t pp = ffma2(pk2(0.05500893f, 0.05500893f), f, pk2(0.24221095f, 0.24221095f));
+    pp = ffma2(pp, f, pk2(0.6932829f, 0.6932829f));
+    pp = ffma2(pp, f, pk2(1.f, 1.f));
+    const float2 pv = upk2(pp), tv = upk2(t);
+    return make_float2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
+                       __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
+  }
 }
 
 // fp32 inputs (TF32 tensor-core products).  The tensor core reads only the
@@ -141,6 +190,9 @@ __global__ void __launch_bounds__(384, 1)
   const int h = blockIdx.y, b = blockIdx.z;
   const int bh = b * p.H + h;
   const int q_row0 = qb * 256;
+#ifdef FA_TRACE
+  const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+#endif
   const int off = p.Nk - p.Nq;  // bottom-right causal alignment
 
   int kv_end = p.Nk;
@@ -157,7 +209,7 @@ __global__ void __launch_bounds__(384, 1)
       mbar_init(&bars->p_full[i], 128);
       mbar_init(&bars->o_full[i], 1);
     }
-    for (int i = 0; i < Tr::NS; ++i) {
+    for (int i = 0; i < 8; ++i) {
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
@@ -184,6 +236,14 @@ __global__ void __launch_bounds__(384, 1)
   if (warp >= 10) {
     // idle warps of the producer/MMA warpgroup
     regs_dec<Tr::REGS_OTHER>();
+#ifdef FA_TRACE
+    if (warp == 10 && lane == 0 && trace_on && Tr::NS < 8) {
+      for (int g = 0; g < 4 * n_kv; ++g) {
+        if (!MBAR_WAIT(&bars->kv_full[7], g & 1, abort_flag)) break;
+        trace_ev(true, 7000 + g);
+      }
+    }
+#endif
   } else if (warp == 9) {
     // ------------------------------------------------------------ producer
     regs_dec<Tr::REGS_OTHER>();
@@ -239,25 +299,30 @@ __global__ void __launch_bounds__(384, 1)
       const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
       const uint32_t aKV = smem_u32(sKV);
 
+      // Operand descriptors are built once per tile; inside the unrolled
+      // loops each MMA only adds a compile-time offset (in 16-byte units), so
+      // the issuing thread keeps ahead of the tensor core.
+      const uint64_t descQ[2] = {sw128_desc(aQ[0], 16, 1024), sw128_desc(aQ[1], 16, 1024)};
       auto issue_qk = [&](int t, int slot) {
-        const uint32_t kb = aKV + slot * Tr::TILE;
+        const uint64_t da = descQ[t];
+        const uint64_t db = sw128_desc(aKV + slot * Tr::TILE, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < D / Tr::KSTEP; ++ks) {
-          const uint32_t o = (ks >> 2) * Tr::CHUNK + (ks & 3) * 32;
-          mma_ss<TF32>(tS[t], sw128_desc(aQ[t] + o, 16, 1024), sw128_desc(kb + o, 16, 1024),
-                       Tr::IDESC_QK, ks > 0);
+          constexpr int kChunk16 = Tr::CHUNK / 16;
+          const uint64_t o = uint64_t((ks >> 2) * kChunk16 + (ks & 3) * 2);
+          mma_ss<TF32>(tS[t], da + o, db + o, Tr::IDESC_QK, ks > 0);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
         const uint32_t vb = aKV + slot * Tr::TILE;
+        // 16-bit: V tile [key][d] is an MN-major B operand; step = KSTEP key rows.
+        // TF32: V tile was stored transposed ([d][key], K-major); step = 32 bytes.
+        const uint64_t db = TF32 ? sw128_desc(vb, 16, 1024) : sw128_desc(vb, Tr::CHUNK, 1024);
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / Tr::KSTEP; ++ks) {
-          // 16-bit: V tile [key][d] is an MN-major B operand; step = KSTEP key rows.
-          // TF32: V tile was stored transposed ([d][key], K-major); step = 32 bytes.
-          const uint64_t bdesc =
-              TF32 ? sw128_desc(vb + (ks >> 2) * (D * 128) + (ks & 3) * 32, 16, 1024)
-                   : sw128_desc(vb + ks * Tr::KSTEP * 128, Tr::CHUNK, 1024);
-          mma_ts<TF32>(tO[t], tS[t] + ks * 8, bdesc, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
+          const uint64_t o = TF32 ? uint64_t((ks >> 2) * (D * 8) + (ks & 3) * 2)
+                                  : uint64_t(ks * Tr::KSTEP * 8);
+          mma_ts<TF32>(tO[t], tS[t] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
         }
       };
       auto kv_wait = [&](int i) {
@@ -268,18 +333,31 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       if (ok) issue_qk(0, 0);
       tc_commit(&bars->s_full[0]);
+#ifdef FA_TRACE
+      if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
       ok = ok && MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
       tc_fence_after();
       if (ok) issue_qk(1, 0);
       tc_commit(&bars->s_full[1]);
+#ifdef FA_TRACE
+      if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
       tc_commit(&bars->kv_empty[0]);
       for (int j = 0; j < n_kv && ok; ++j) {
         const int iv = 2 * j + 1, ik = 2 * j + 2;
         const int sv = iv % Tr::NS, sk = ik % Tr::NS;
-        ok = kv_wait(iv) && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
+        ok = kv_wait(iv);
+        TRACE(6000 + j);
+        ok = ok && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
+        TRACE(3000 + j);
         issue_pv(0, sv, j > 0);
+        TRACE(4000 + j);
+#ifdef FA_TRACE
+        if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
         tc_commit(&bars->o_full[0]);
         const bool more = j + 1 < n_kv;
         if (more) {
@@ -288,17 +366,30 @@ __global__ void __launch_bounds__(384, 1)
           if (!ok) break;
           issue_qk(0, sk);
           tc_commit(&bars->s_full[0]);
+          TRACE(5000 + j);
+#ifdef FA_TRACE
+          if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
         }
         ok = MBAR_WAIT(&bars->p_full[1], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
+        TRACE(3100 + j);
         issue_pv(1, sv, j > 0);
+        TRACE(4100 + j);
+#ifdef FA_TRACE
+        if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
         tc_commit(&bars->o_full[1]);
         tc_commit(&bars->kv_empty[sv]);
         if (more) {
           issue_qk(1, sk);
           tc_commit(&bars->s_full[1]);
           tc_commit(&bars->kv_empty[sk]);
+          TRACE(5100 + j);
+#ifdef FA_TRACE
+          if (trace_on) tc_commit(&bars->kv_full[7]);
+#endif
         }
       }
     }
@@ -316,23 +407,24 @@ __global__ void __launch_bounds__(384, 1)
     const int tile_first_row = q_row0 + t * 128;
 
     float m_ref = -INFINITY;  // reference maximum, scaled log2 units
-    float row_sum = 0.f;      // Σ exp2 of the scores: gives the logsumexp L
-    float row_sum_p = 0.f;    // Σ of P as rounded for the P·V product: normalises O
+    float row_sum = 0.f;    // Σ exp2 of the scores: gives the logsumexp L
+    float row_sum_p = 0.f;  // Σ of P as rounded for the P·V product: normalises O
     bool ok = true;
 
     for (int j = 0; j < n_kv; ++j) {
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
-      float s[Tr::BN];
+#ifdef FA_TRACE
+      const bool tr = trace_on && quad == 0 && lane == 0;
+      trace_ev(tr, 1000 + 100 * t + j);
+#endif
+      // All four 32-column loads in flight, one wait.
+      uint32_t su[4][32];
 #pragma unroll
-      for (int c = 0; c < Tr::BN; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tS + c, u);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) s[c + e] = __uint_as_float(u[e]);
-      }
+      for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, su[q]);
+      tmem_ld_wait();
+      float* s = reinterpret_cast<float*>(&su[0][0]);
       const int k0 = j * Tr::BN;
       const bool tail = k0 + Tr::BN > p.Nk;
       const bool diag = CAUSAL && (k0 + Tr::BN - 1 > tile_first_row + off);
@@ -343,10 +435,17 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < Tr::BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      float mx = fmax3(s[0], s[1], s[2]);
+      // Row maximum: four independent chains of 3-input max.
+      float mq[4];
 #pragma unroll
-      for (int c = 3; c + 1 < Tr::BN; c += 2) mx = fmax3(mx, s[c], s[c + 1]);
-      if constexpr ((Tr::BN - 3) % 2 == 1) mx = fmaxf(mx, s[Tr::BN - 1]);
+      for (int q = 0; q < 4; ++q) {
+        const float* v = s + 32 * q;
+        float a = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+        for (int i = 3; i < 31; i += 2) a = fmax3(a, v[i], v[i + 1]);
+        mq[q] = fmaxf(a, v[31]);
+      }
+      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float m_tile = mx * sl2;
       const bool upd = m_tile > m_ref + kRescaleThreshold;
       float alpha = 1.f;
@@ -373,18 +472,24 @@ __global__ void __launch_bounds__(384, 1)
       }
       const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
       const uint64_t c2 = pk2(sl2, sl2), negm2 = pk2(-m_use, -m_use);
-      uint64_t sum2 = pk2(0.f, 0.f), sum2_p = pk2(0.f, 0.f);
+      // Four independent partial sums (one per 32-column quarter) of the
+      // unrounded P (for L) and of P as rounded for the P·V product (to
+      // normalise O, so that a row's weights add up to one exactly: with a
+      // peaky softmax the rounding of the largest P would otherwise show in O).
+      uint64_t sum2[4], sum2_p[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) sum2[q] = sum2_p[q] = pk2(0.f, 0.f);
       if constexpr (TF32) {
 #pragma unroll
         for (int c = 0; c < Tr::BN; c += 32) {
           uint32_t u[32];
 #pragma unroll
           for (int e = 0; e < 32; e += 2) {
-            const float2 x = upk2(ffma2(pk2(s[c + e], s[c + e + 1]), c2, negm2));
-            const float p0 = ex2(x.x), p1 = ex2(x.y);
-            const float r0 = round_tf32(p0), r1 = round_tf32(p1);
-            sum2 = fadd2(sum2, pk2(p0, p1));
-            sum2_p = fadd2(sum2_p, pk2(r0, r1));
+            const uint64_t x = ffma2(pk2(s[c + e], s[c + e + 1]), c2, negm2);
+            const float2 pe = exp2_pair<false>(x);
+            const float r0 = round_tf32(pe.x), r1 = round_tf32(pe.y);
+            sum2[c / 32] = fadd2(sum2[c / 32], pk2(pe.x, pe.y));
+            sum2_p[c / 32] = fadd2(sum2_p[c / 32], pk2(r0, r1));
             u[e] = __float_as_uint(r0);
             u[e + 1] = __float_as_uint(r1);
           }
@@ -396,26 +501,30 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t u[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float2 x = upk2(ffma2(pk2(s[c + 2 * e], s[c + 2 * e + 1]), c2, negm2));
-            const float p0 = ex2(x.x), p1 = ex2(x.y);
-            u[e] = ElemTraits<T>::pack2(p0, p1);
-            // O is normalised by the sum of the same rounded P the P·V
-            // product uses, so a row's weights add up to one exactly; L keeps
-            // the unrounded sum (the exact logsumexp).
+            const int q = (c + 2 * e) / 32;
+            const uint64_t x = ffma2(pk2(s[c + 2 * e], s[c + 2 * e + 1]), c2, negm2);
+            // every kEmuPeriod-th pair of exponentials on the FMA pipe
+            const float2 pe = (e % kEmuPeriod == kEmuPeriod - 1) ? exp2_pair<true>(x)
+                                                                  : exp2_pair<false>(x);
+            u[e] = ElemTraits<T>::pack2(pe.x, pe.y);
             const float2 pr = ElemTraits<T>::unpack2(u[e]);
-            sum2 = fadd2(sum2, pk2(p0, p1));
-            sum2_p = fadd2(sum2_p, pk2(pr.x, pr.y));
+            sum2[q] = fadd2(sum2[q], pk2(pe.x, pe.y));
+            sum2_p[q] = fadd2(sum2_p[q], pk2(pr.x, pr.y));
           }
           tmem_st32(tS + c / 2, u);
         }
       }
       {
-        const float2 a = upk2(sum2), b = upk2(sum2_p);
+        const float2 a = upk2(fadd2(fadd2(sum2[0], sum2[1]), fadd2(sum2[2], sum2[3])));
+        const float2 b = upk2(fadd2(fadd2(sum2_p[0], sum2_p[1]), fadd2(sum2_p[2], sum2_p[3])));
         row_sum += a.x + a.y;
         row_sum_p += b.x + b.y;
       }
       tmem_st_wait();
       tc_fence_before();
+#ifdef FA_TRACE
+      trace_ev(tr, 2000 + 100 * t + j);
+#endif
       mbar_arrive(&bars->p_full[t]);
     }
 
@@ -512,5 +621,18 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
 }
 
 FA_ERROR_ACCESSOR(take_error_fwd)
+
+#ifdef FA_TRACE
+}  // namespace fa
+extern "C" int fa_trace_read(long long* out, int max) {
+  const int n = max < 16384 ? max : 16384;
+  cudaMemcpyFromSymbol(out, fa::g_trace, sizeof(long long) * 2 * n);
+  cudaMemset(out, 0, 0);
+  static long long zeros[16384][2];
+  cudaMemcpyToSymbol(fa::g_trace, zeros, sizeof(zeros));
+  return n;
+}
+namespace fa {
+#endif
 
 }  // namespace fa
