@@ -21,6 +21,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libfa_b200.so")
 
 FA_FP32, FA_BF16, FA_FP16 = 0, 1, 2
+FA_DECODE_NOALLOC_SCRATCH_BYTES = 8 << 20  # include/fa.h
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5)
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED",
@@ -39,6 +40,7 @@ SIGNATURES = {
     "fa_status": (_I, [_VP]),
     "fa_bwd_set_timing_events": (_I, [_VP, _VP]),
     "fa_last_timeout_site": (_I, []),
+    "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_version": (ctypes.c_char_p, []),
 }
 
@@ -189,6 +191,33 @@ def decode(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, l
                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                          _stream(q.device))
     _raise("fa_decode", rc)
+    return out, lse
+
+
+def decode_noalloc(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, lse=None):
+    """Split-KV decode like decode(), for callers that cannot allocate device
+    memory: no workspace is created or passed; the partial results go to the
+    library's own 8 MiB device scratch array (see fa_decode_noalloc in
+    include/fa.h: calls share it, so overlapping calls on the GPU race)."""
+    _check("q", q)
+    B, H, one, d = q.shape
+    if one != 1:
+        raise ValueError("decode takes exactly one query row per (batch, head)")
+    Nk = k.shape[2]
+    _check("k", k, (B, H, Nk, d), q.dtype)
+    _check("v", v, (B, H, Nk, d), q.dtype)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
+    _check("out", out, q.shape, q.dtype)
+    _check("lse", lse, (B, H, 1), torch.float32)
+    rc = lib().fa_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
+                                 int(num_splits), _stream(q.device))
+    _raise("fa_decode_noalloc", rc)
     return out, lse
 
 

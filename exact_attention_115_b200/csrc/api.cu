@@ -271,6 +271,46 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
              : FA_ERR_CUDA;
 }
 
+int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
+                      int Nk, int d, float scale, int dtype, int num_splits, void* stream) {
+  int st = check_common(B, H, 1, Nk, d, scale, dtype);
+  if (st != FA_OK) return st;
+  if (dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (num_splits < 0) return FA_ERR_INVALID;
+  const void* ptrs[] = {Q, K, V, O, L};
+  for (const void* p : ptrs)
+    if (!p || !aligned16(p)) return FA_ERR_INVALID;
+  const int BH = B * H;
+  // Scratch bytes for s parts: partial outputs [BH, s, d] then logsumexps [BH, s].
+  auto need_for = [&](int s) {
+    return round_up(size_t(BH) * s * d * sizeof(float), 256) + round_up(size_t(BH) * s * 4, 256);
+  };
+  const size_t cap = decode_scratch_bytes();
+  int s = num_splits > 0 ? num_splits : decode_auto_splits(BH, Nk);
+  s = std::min(s, Nk);
+  if (num_splits == 0)
+    while (s > 1 && need_for(s) > cap) --s;  // automatic: fewer parts until they fit
+  if (s > 65535) return FA_ERR_UNSUPPORTED;
+  const int kps = decode_keys_per_split(Nk, s);
+  s = (Nk + kps - 1) / kps;
+  if (need_for(s) > cap) return FA_ERR_WORKSPACE;  // beyond the built-in scratch
+  void* scratch = nullptr;
+  if (decode_scratch_ptr(&scratch) != cudaSuccess) return FA_ERR_CUDA;
+  DecodeParams p;
+  p.Q = Q; p.K = K; p.V = V; p.O = O; p.L = L;
+  p.Opart = static_cast<float*>(scratch);
+  p.Lpart = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
+                                     round_up(size_t(BH) * s * d * sizeof(float), 256));
+  p.BH = BH;
+  p.Nk = Nk;
+  p.splits = s;
+  p.keys_per_split = kps;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
 int fa_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return FA_ERR_CUDA;

@@ -16,6 +16,8 @@
 #include "common.cuh"
 #include "launch.h"
 
+#include <mutex>
+
 namespace fa {
 
 namespace {
@@ -202,6 +204,42 @@ cudaError_t launch_decode(int dtype, int d, const DecodeParams& p, cudaStream_t 
     if (d == 128) return launch_decode_t<__half, 128>(p, s);
   }
   return cudaErrorInvalidValue;
+}
+
+// ------------------------------------------------------------------
+// Scratch of fa_decode_noalloc: the partial outputs and logsumexps of the
+// split-KV decode, kept in a device array that belongs to this library
+// instead of a workspace the caller allocates.  Every GPU that loads the
+// library holds these 8 MiB until the process exits.  All calls on a device
+// share the array and it keeps whatever the last call left there; nothing
+// in it has to start at zero, because a call writes every partial result
+// its combine step reads.  Two calls whose kernels overlap on the GPU (on
+// different streams or from different host threads) race on it.
+constexpr size_t kDecodeScratchBytes = FA_DECODE_NOALLOC_SCRATCH_BYTES;  // 8 MiB
+static __device__ __align__(256) unsigned char g_decode_scratch[kDecodeScratchBytes];
+
+size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
+
+// In host code g_decode_scratch names a host-side stand-in, not device
+// memory, so its device address on the current device is looked up with
+// cudaGetSymbolAddress, once per device (by the first no-alloc call made
+// with that device current), and cached.
+cudaError_t decode_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* cached[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cached[dev] == nullptr) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    cached[dev] = ptr;
+  }
+  *out = cached[dev];
+  return cudaSuccess;
 }
 
 FA_ERROR_ACCESSOR(take_error_decode)

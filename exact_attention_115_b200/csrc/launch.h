@@ -72,6 +72,10 @@ struct DecodeParams {
 };
 
 cudaError_t launch_decode(int dtype, int d, const DecodeParams& p, cudaStream_t s);
+// Library-owned scratch of fa_decode_noalloc (decode.cu): its size, and its
+// device address on the current device.
+size_t decode_scratch_bytes();
+cudaError_t decode_scratch_ptr(void** out);
 
 // Read-and-clear accessors of each kernel file's device error word.
 cudaError_t take_error_fwd(int* word, int* site);

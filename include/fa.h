@@ -48,6 +48,9 @@ extern "C" {
 
 typedef enum { FA_FP32 = 0, FA_BF16 = 1, FA_FP16 = 2 } fa_dtype;
 
+/* Size of the device scratch array that fa_decode_noalloc uses (below). */
+#define FA_DECODE_NOALLOC_SCRATCH_BYTES ((size_t)8 << 20)
+
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = -1,     /* null pointer, size <= 0, non-finite scale, misaligned pointer */
@@ -100,7 +103,37 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
               int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
               void* stream);
 
-/* Synchronises `stream`, then returns and clears the device error word:
+/* fa_decode_noalloc: the split-KV decode of fa_decode for callers that
+ * cannot allocate device memory.  The pages have no counterpart for it.
+ *
+ * Some callers own every byte of device memory themselves and hand a
+ * library only its input and output buffers: a plugin or runtime whose
+ * interface has no way to pass a workspace, or a service whose device
+ * memory is fixed once it has started.  They cannot provide fa_decode's
+ * workspace and must not call cudaMalloc.  This entry point needs no
+ * workspace: the per-part partial outputs and logsumexps go to a scratch
+ * array that the library itself holds in device memory (a file-scope
+ * __device__ array of FA_DECODE_NOALLOC_SCRATCH_BYTES = 8 MiB, present on
+ * every GPU that loads the library until the process exits).  It calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Arguments and results are those of fa_decode without the workspace.  The
+ * scratch needed is about B*H*num_splits*(d+1)*4 bytes: with num_splits = 0
+ * the number of parts is reduced until it fits; FA_ERR_WORKSPACE is returned,
+ * before anything is enqueued, when an explicit num_splits does not fit or
+ * when even one part per (batch, head) does not (B*H*(d+1)*4 bytes above the
+ * 8 MiB, i.e. B*H above about 16000 at d = 128).
+ *
+ * The first call on each device looks up the array's device address (with
+ * that device current) and caches it; make that first call before any
+ * stream capture.  All calls share the one array and it keeps the last
+ * call's contents (nothing in it needs to start at zero); calls whose
+ * kernels overlap on the GPU, on different streams or host threads, race on
+ * it and must be serialised by the caller. */
+int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
+                      int Nk, int d, float scale, int dtype, int num_splits, void* stream);
+
+/* Synchronises `stream`, then returns and clears the device error word:/* Synchronises `stream`, then returns and clears the device error word:
  * FA_OK, FA_ERR_TIMEOUT if a kernel's bounded wait expired, FA_ERR_CUDA if
  * the stream reports a CUDA error. */
 int fa_status(void* stream);
