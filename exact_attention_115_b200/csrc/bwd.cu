@@ -97,38 +97,38 @@ template <typename T, int D>
 struct BwdTraits {
   static constexpr int ES = 2;
   static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
-  static constexpr int BM = D == 128 ? 64 : 128;     // query rows per step
+  static constexpr int BM = 128;                     // query rows per step
   static constexpr int CWC = BM / 2;                 // query columns per compute warpgroup
   static constexpr bool DQ_T = D == 128;             // dQᵀ = Kᵀ dSᵀ (else dQ = dS K)
-  static constexpr int NSTG = 2;                     // Q/dO pipeline stages
   static constexpr int KV_TILE = BN * D * ES;        // bytes of the K (or V) tile
   static constexpr int KV_CHUNK = BN * 128;          // one 128-byte column block of it
   static constexpr int Q_TILE = BM * D * ES;         // bytes of a Q (or dO) tile
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int DS_TILE = BN * BM * ES;       // dSᵀ, rows = keys, q contiguous
-  static constexpr int DQ_STAGE = BM * D * 4;        // fp32 dQ tile staging
-  // shared-memory offsets (all 1024-aligned)
+  // dQ staging: d = 128 drains dQᵀ in four 32-row quarters (16 KB each);
+  // d = 64 stages the whole [BM × 64] fp32 tile (32 KB) at once.
+  static constexpr int DQ_PARTS = D == 128 ? 4 : 1;
+  static constexpr int DQ_STAGE = BM * D * 4 / DQ_PARTS;
+  // shared-memory offsets (all 1024-aligned).  Q is double buffered (the
+  // next step's Sᵀ needs it while this step's dK still reads the current
+  // one); dO is single buffered (the next dPᵀ comes after this step's dV).
   static constexpr int OFF_K = 0;
   static constexpr int OFF_V = OFF_K + KV_TILE;
-  static constexpr int OFF_Q = OFF_V + KV_TILE;
-  static constexpr int OFF_DO = OFF_Q + NSTG * Q_TILE;
-  static constexpr int OFF_DS = OFF_DO + NSTG * Q_TILE;   // two dSᵀ buffers
-  static constexpr int OFF_DQ = OFF_DS + 2 * DS_TILE;
-  static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;        // L·log2e and D per stage
-  static constexpr int OFF_BAR = OFF_LD + NSTG * 2 * BM * 4;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;      // 2 stages
+  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_DS = OFF_DO + Q_TILE;
+  static constexpr int OFF_DQ = OFF_DS + DS_TILE;
+  static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;   // L·log2e and D per Q stage
+  static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BM * 4;
   static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
-  // TMEM columns
-  static constexpr int COL_S0 = 0;
-  static constexpr int COL_S1 = BM;
-  static constexpr int COL_DP0 = 2 * BM;
-  static constexpr int COL_DP1 = D == 128 ? 3 * BM : 2 * BM;  // single dPᵀ buffer for d = 64
-  static constexpr int COL_DV = D == 128 ? 4 * BM : 3 * BM;
+  // TMEM columns: Sᵀ | dPᵀ (dQ of the step lands here after dK read dSᵀ) | dV | dK
+  static constexpr int COL_S = 0;
+  static constexpr int COL_DP = BM;
+  static constexpr int COL_DV = 2 * BM;
   static constexpr int COL_DK = COL_DV + D;
   static_assert(COL_DK + D <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared-memory budget");
   static constexpr int THREADS = 512;
-  // No setmaxnreg: every warp keeps the 128 registers per thread it is
-  // launched with (the compute code works in 32-column chunks to fit).
   static constexpr uint32_t F = ElemTraits<T>::fmt;
   static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
   static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV, dK (A in TMEM)
@@ -149,19 +149,23 @@ __device__ __forceinline__ void btrace(bool on, int code) {
 #define BTRACE(code) ((void)0)
 #endif
 
+// Every barrier below completes once per step except q_full / q_empty (one
+// per Q stage, every other step).  A producer of any of them cannot run two
+// phases ahead of its waiter (each step's signal needs the waiter's
+// previous step to have finished), so parity waits are unambiguous.
 struct BwdBarriers {
   uint64_t kv_full;
-  uint64_t qdo_full[2];
-  uint64_t qdo_empty[2];
-  uint64_t s_full[2];
-  uint64_t dp_full[2];
-  // One barrier per buffer for every signal whose producer could otherwise
-  // run two phases ahead of a parity wait.
-  uint64_t p_ready[2];
+  uint64_t q_full[2];
+  uint64_t q_empty[2];
+  uint64_t do_full;
+  uint64_t do_empty;
+  uint64_t s_full;
+  uint64_t dp_full;
+  uint64_t p_ready;
   uint64_t ds_ready;
-  uint64_t dq_full[2];
-  uint64_t dq_empty[2];
-  uint64_t ds_free[2];
+  uint64_t dq_full;
+  uint64_t dq_empty;
+  uint64_t ds_free;
   uint64_t dkv_done;
   uint64_t watch;  // trace builds only
   uint32_t tmem_base;
@@ -177,27 +181,6 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
   i0 = first / BM;
   const int nt = (Nq + BM - 1) / BM;
   n = max(0, nt - i0);
-}
-
-// Load / store N (16, 32 or 64) consecutive TMEM columns of this warp's lanes.
-template <int N>
-__device__ __forceinline__ void tmem_ld_n(uint32_t taddr, uint32_t* r) {
-  if constexpr (N == 16) {
-    tmem_ld16(taddr, r);
-  } else {
-#pragma unroll
-    for (int c = 0; c < N; c += 32) tmem_ld32(taddr + c, *reinterpret_cast<uint32_t(*)[32]>(r + c));
-  }
-}
-template <int N>
-__device__ __forceinline__ void tmem_st_n(uint32_t taddr, const uint32_t* r) {
-  if constexpr (N == 16) {
-    tmem_st16(taddr, r);
-  } else {
-#pragma unroll
-    for (int c = 0; c < N; c += 32)
-      tmem_st32(taddr + c, *reinterpret_cast<const uint32_t(*)[32]>(r + c));
-  }
 }
 
 template <typename T, int D, bool CAUSAL>
@@ -228,17 +211,18 @@ __global__ void __launch_bounds__(512, 1)
   if (threadIdx.x == 0) {
     mbar_init(&bars->kv_full, 1);
     for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->qdo_full[s], 1);
-      mbar_init(&bars->qdo_empty[s], 1);
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->dp_full[s], 1);
-      mbar_init(&bars->p_ready[s], 256);
-      mbar_init(&bars->dq_full[s], 1);
-      mbar_init(&bars->ds_free[s], 1);
+      mbar_init(&bars->q_full[s], 1);
+      mbar_init(&bars->q_empty[s], 1);
     }
+    mbar_init(&bars->do_full, 1);
+    mbar_init(&bars->do_empty, 1);
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->dp_full, 1);
+    mbar_init(&bars->p_ready, 256);
     mbar_init(&bars->ds_ready, 256);
-    mbar_init(&bars->dq_empty[0], 128);
-    mbar_init(&bars->dq_empty[1], 128);
+    mbar_init(&bars->dq_full, 1);
+    mbar_init(&bars->dq_empty, 128);
+    mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dkv_done, 1);
     mbar_init(&bars->watch, 1);
     bars->abort_flag = 0;
@@ -286,25 +270,29 @@ __global__ void __launch_bounds__(512, 1)
         tma_load_3d(sV + c * Tr::KV_CHUNK, &tmV, &bars->kv_full, c * 64, key0, bh);
       }
       for (int i = 0; i < n_q; ++i) {
-        const int s = i % Tr::NSTG;
-        if (i >= Tr::NSTG &&
-            !MBAR_WAIT(&bars->qdo_empty[s], ((i / Tr::NSTG) - 1) & 1, abort_flag))
-          break;
+        const int s = i & 1;
         const int q0 = (i0 + i) * BM;
-        uint64_t* bar = &bars->qdo_full[s];
-        mbar_arrive_expect_tx(bar, 2 * Tr::Q_TILE + 2 * BM * 4);
+        // Q (with L and D) into stage s, once step i-2 has released it
+        if (i >= 2 && !MBAR_WAIT(&bars->q_empty[s], ((i >> 1) - 1) & 1, abort_flag)) break;
+        uint64_t* bar = &bars->q_full[s];
+        mbar_arrive_expect_tx(bar, Tr::Q_TILE + 2 * BM * 4);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
-          tma_load_3d(sdO + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmdO, bar, c * 64, q0, bh);
-        }
         const size_t row = size_t(bh) * p.Nq_pad + q0;
         bulk_load(sLD + (s * 2 + 0) * BM, p.Lsc + row, BM * 4, bar);
         bulk_load(sLD + (s * 2 + 1) * BM, p.Dsum + row, BM * 4, bar);
+        // dO into its single buffer, once step i-1's dV product has read it
+        if (i >= 1 && !MBAR_WAIT(&bars->do_empty, (i - 1) & 1, abort_flag)) break;
+        mbar_arrive_expect_tx(&bars->do_full, Tr::Q_TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sdO + c * Tr::Q_CHUNK, &tmdO, &bars->do_full, c * 64, q0, bh);
       }
       // Drain every issued load before the CTA may exit.
-      for (int i = max(0, n_q - Tr::NSTG); i < n_q; ++i)
-        MBAR_WAIT(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
+      for (int i = max(0, n_q - 2); i < n_q; ++i)
+        MBAR_WAIT(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag);
+      if (n_q > 0) MBAR_WAIT(&bars->do_full, (n_q - 1) & 1, abort_flag);
       MBAR_WAIT(&bars->kv_full, 0, abort_flag);
     }
   } else if (warp == 12) {
@@ -312,22 +300,17 @@ __global__ void __launch_bounds__(512, 1)
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
-      const uint32_t colS[2] = {tmem + Tr::COL_S0, tmem + Tr::COL_S1};
-      const uint32_t colDP[2] = {tmem + Tr::COL_DP0, tmem + Tr::COL_DP1};
+      const uint32_t colS = tmem + Tr::COL_S, colDP = tmem + Tr::COL_DP;
       const uint32_t colDV = tmem + Tr::COL_DV, colDK = tmem + Tr::COL_DK;
-
       // Operand descriptors are built once; inside the unrolled loops each
-      // MMA only adds a compile-time offset (16-byte units), so the issuing
-      // thread keeps ahead of the tensor core.
+      // MMA only adds a compile-time offset (16-byte units).
       const uint64_t dK_k = sw128_desc(aK, 16, 1024), dV_k = sw128_desc(aV, 16, 1024);
       const uint64_t dK_mn = sw128_desc(aK, Tr::KV_CHUNK, 1024);
-      // Stage / buffer s of a tile lives s * (tile bytes) further on: add
-      // that (in 16-byte units) to the stage-0 descriptor.
-      const uint64_t dQ_k0 = sw128_desc(aQ, 16, 1024), dO_k0 = sw128_desc(adO, 16, 1024);
+      const uint64_t dQ_k0 = sw128_desc(aQ, 16, 1024), dO_k = sw128_desc(adO, 16, 1024);
       const uint64_t dQ_mn0 = sw128_desc(aQ, Tr::Q_CHUNK, 1024);
-      const uint64_t dO_mn0 = sw128_desc(adO, Tr::Q_CHUNK, 1024);
-      const uint64_t dS_mn0 = sw128_desc(adS, Tr::BN * 128, 1024);
-      auto stg = [](uint64_t d0, int s, int bytes) { return d0 + uint64_t(s) * uint64_t(bytes >> 4); };
+      const uint64_t dO_mn = sw128_desc(adO, Tr::Q_CHUNK, 1024);
+      const uint64_t dS_mn = sw128_desc(adS, Tr::BN * 128, 1024);
+      auto stg = [](uint64_t d0, int s) { return d0 + uint64_t(s) * uint64_t(Tr::Q_TILE >> 4); };
 
       // Sᵀ (or dPᵀ) = X[128 keys × D] · Y[BM × D]ᵀ, both K-major.
       auto mma_st = [&](uint32_t dcol, uint64_t dx, uint64_t dy) {
@@ -351,102 +334,71 @@ __global__ void __launch_bounds__(512, 1)
       };
       // dQᵀ [D × BM] = Kᵀ · dSᵀ  (d = 128), or dQ [BM × D] = dS · K (d = 64);
       // both operands MN-major, K dimension = the 128 keys.
-      auto mma_dq = [&](uint32_t dcol, uint64_t dds) {
+      auto mma_dq = [&](uint32_t dcol) {
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / 16; ++ks) {
           const uint64_t o = uint64_t(ks * 128);
           if constexpr (Tr::DQ_T)
-            mma_ss<false>(dcol, dK_mn + o, dds + o, Tr::IDESC_DQ, ks > 0);
+            mma_ss<false>(dcol, dK_mn + o, dS_mn + o, Tr::IDESC_DQ, ks > 0);
           else
-            mma_ss<false>(dcol, dds + o, dK_mn + o, Tr::IDESC_DQ, ks > 0);
+            mma_ss<false>(dcol, dS_mn + o, dK_mn + o, Tr::IDESC_DQ, ks > 0);
         }
       };
-      auto qwait = [&](int i) {
-        return MBAR_WAIT(&bars->qdo_full[i % Tr::NSTG], (i / Tr::NSTG) & 1, abort_flag);
-      };
 
-      bool ok = MBAR_WAIT(&bars->kv_full, 0, abort_flag) && (n_q == 0 || qwait(0));
+      bool ok = MBAR_WAIT(&bars->kv_full, 0, abort_flag);
+      if (ok && n_q > 0)
+        ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && MBAR_WAIT(&bars->do_full, 0, abort_flag);
       tc_fence_after();
       if (ok && n_q > 0) {
-        mma_st(colS[0], dK_k, dQ_k0);
-        tc_commit(&bars->s_full[0]);
-        mma_st(colDP[0], dV_k, dO_k0);
-        tc_commit(&bars->dp_full[0]);
+        mma_st(colS, dK_k, dQ_k0);
+        tc_commit(&bars->s_full);
+        mma_st(colDP, dV_k, dO_k);
+        tc_commit(&bars->dp_full);
       }
+      // Per step i: dV (needs Pᵀ_i), then the next Sᵀ into the same columns
+      // (in issue order after dV read them), dK (needs dSᵀ_i), dQ into the
+      // dPᵀ columns (after dK read dSᵀ_i), and last the next dPᵀ, once the
+      // dQ warpgroup has drained dQ_i from those columns.
       for (int i = 0; i < n_q && ok; ++i) {
-        const int s = i % Tr::NSTG, b2 = i & 1;
+        const int s = i & 1;
         const bool more = i + 1 < n_q;
-        const int s1 = (i + 1) % Tr::NSTG;
-        if constexpr (D == 128) {
-          // d = 128: dQᵀ of step i goes to dPᵀ[i % 2] once the dK product
-          // has read dSᵀ from there.  Order per step: the next Sᵀ (its
-          // buffer is free: Pᵀ of step i-1 was consumed last step), dV, dK,
-          // dQ of this step, and last the next dPᵀ, whose buffer held dQ of
-          // step i-1 and must first be drained by the dQ warpgroup; a whole
-          // step has passed since that dQ was produced, so this rarely waits.
-          if (more) {
-            ok = qwait(i + 1);
-            tc_fence_after();
-            if (!ok) break;
-            mma_st(colS[b2 ^ 1], dK_k, stg(dQ_k0, s1, Tr::Q_TILE));
-            tc_commit(&bars->s_full[b2 ^ 1]);
-          }
-          BTRACE(1000 + i);
-          ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
+        ok = MBAR_WAIT(&bars->p_ready, i & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        BTRACE(2000 + i);
+        mma_grad(colDV, colS, dO_mn, i > 0);
+        tc_commit(&bars->do_empty);
+        BTRACE(3000 + i);
+        if (more) {
+          ok = MBAR_WAIT(&bars->q_full[s ^ 1], ((i + 1) >> 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          BTRACE(2000 + i);
-          mma_grad(colDV, colS[b2], stg(dO_mn0, s, Tr::Q_TILE), i > 0);
-          BTRACE(3000 + i);
-          ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
-          tc_fence_after();
-          if (!ok) break;
-          BTRACE(4000 + i);
-          mma_grad(colDK, colDP[b2], stg(dQ_mn0, s, Tr::Q_TILE), i > 0);
-          tc_commit(&bars->qdo_empty[s]);
-          if (!more) tc_commit(&bars->dkv_done);
-          mma_dq(colDP[b2], stg(dS_mn0, b2, Tr::DS_TILE));
-          tc_commit(&bars->dq_full[b2]);
-          tc_commit(&bars->ds_free[b2]);
-          BTRACE(5000 + i);
+          mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
+          tc_commit(&bars->s_full);
+        }
+        BTRACE(1000 + i);
+        ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        BTRACE(4000 + i);
+        mma_grad(colDK, colDP, stg(dQ_mn0, s), i > 0);
+        tc_commit(&bars->q_empty[s]);
+        if (!more) tc_commit(&bars->dkv_done);
+        mma_dq(colDP);
+        tc_commit(&bars->dq_full);
+        tc_commit(&bars->ds_free);
+        BTRACE(5000 + i);
 #ifdef FA_TRACE
-          if (trace_on) tc_commit(&bars->watch);
+        if (trace_on) tc_commit(&bars->watch);
 #endif
-          if (more) {
-            ok = i < 1 || MBAR_WAIT(&bars->dq_empty[b2 ^ 1], ((i - 1) >> 1) & 1, abort_flag);
-            tc_fence_after();
-            if (!ok) break;
-            mma_st(colDP[b2 ^ 1], dV_k, stg(dO_k0, s1, Tr::Q_TILE));
-            tc_commit(&bars->dp_full[b2 ^ 1]);
-          }
-        } else {
-          // d = 64: dQ of step i goes to Sᵀ[i % 2]; the next Sᵀ needs the dQ
-          // of step i-1 drained from its buffer.
-          if (more) {
-            ok = qwait(i + 1) &&
-                 (i < 1 || MBAR_WAIT(&bars->dq_empty[b2 ^ 1], ((i - 1) >> 1) & 1, abort_flag));
-            tc_fence_after();
-            if (!ok) break;
-            mma_st(colS[b2 ^ 1], dK_k, stg(dQ_k0, s1, Tr::Q_TILE));
-            tc_commit(&bars->s_full[b2 ^ 1]);
-          }
-          ok = MBAR_WAIT(&bars->p_ready[b2], (i >> 1) & 1, abort_flag);
+        if (more) {
+          ok = MBAR_WAIT(&bars->dq_empty, i & 1, abort_flag) &&
+               MBAR_WAIT(&bars->do_full, (i + 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          mma_grad(colDV, colS[b2], stg(dO_mn0, s, Tr::Q_TILE), i > 0);
-          ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
-          tc_fence_after();
-          if (!ok) break;
-          mma_grad(colDK, colDP[0], stg(dQ_mn0, s, Tr::Q_TILE), i > 0);
-          tc_commit(&bars->qdo_empty[s]);
-          if (!more) tc_commit(&bars->dkv_done);
-          mma_dq(colS[b2], stg(dS_mn0, b2, Tr::DS_TILE));
-          tc_commit(&bars->dq_full[b2]);
-          tc_commit(&bars->ds_free[b2]);
-          if (more) {
-            mma_st(colDP[0], dV_k, stg(dO_k0, s1, Tr::Q_TILE));
-            tc_commit(&bars->dp_full[0]);
-          }
+          mma_st(colDP, dV_k, dO_k);
+          tc_commit(&bars->dp_full);
+          BTRACE(6000 + i);
         }
       }
       if (n_q == 0) tc_commit(&bars->dkv_done);
@@ -464,20 +416,21 @@ __global__ void __launch_bounds__(512, 1)
     const float sl2 = p.scale_log2;
     const float scale = p.scale;
     const int qmin = key - off;  // first query row that sees this key
+    const uint32_t tS = tmem + lane_off + Tr::COL_S;
+    const uint32_t tDP = tmem + lane_off + Tr::COL_DP;
     bool ok = true;
     for (int i = 0; i < n_q; ++i) {
-      const int s = i % Tr::NSTG, b2 = i & 1;
+      const int s = i & 1;
       const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
       const float* sL = sLD + (s * 2 + 0) * BM + cw * CWC;
       const float* sDv = sLD + (s * 2 + 1) * BM + cw * CWC;
       // ---- P = exp2(S·c − L·log2e), causal / ragged masking
-      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[b2], (i >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, i & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
 #ifdef FA_TRACE
-      btrace(trace_on && quad == 0 && lane == 0, 6000 + 100 * cw + i);  // compute got S
+      btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // got S
 #endif
-      const uint32_t tS = tmem + lane_off + (b2 ? Tr::COL_S1 : Tr::COL_S0);
       const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
       float P[CWC];
       const uint64_t c2 = pk2(sl2, sl2);
@@ -509,23 +462,16 @@ __global__ void __launch_bounds__(512, 1)
       }
       tmem_st_wait();
       tc_fence_before();
-#ifdef FA_TRACE
-      btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // P done
-#endif
-      mbar_arrive(&bars->p_ready[b2]);
+      mbar_arrive(&bars->p_ready);
 
       // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
       // and to shared memory for the dQ product (row = key, BM query values
       // contiguous, 128-byte swizzled, 64 values per column block).
-      ok = __all_sync(0xffffffffu,
-                      MBAR_WAIT(&bars->dp_full[D == 128 ? b2 : 0], (D == 128 ? (i >> 1) : i) & 1,
-                                abort_flag));
-      if (ok && i >= 2)
-        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free[b2], ((i - 2) >> 1) & 1, abort_flag));
+      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dp_full, i & 1, abort_flag));
+      if (ok && i >= 1)
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (i - 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
-      const uint32_t tDP = tmem + lane_off + (D == 128 && b2 ? Tr::COL_DP1 : Tr::COL_DP0);
-      uint8_t* buf = sdS + b2 * Tr::DS_TILE;
       const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
       for (int c = 0; c < CWC; c += 32) {
@@ -546,7 +492,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int c16 = 0; c16 < 4; ++c16) {
           const int col = cw * CWC + c + c16 * 8;  // first query column of this 16-byte chunk
           const int blk = col >> 6, ch = (col >> 3) & 7;
-          *reinterpret_cast<uint4*>(buf + blk * (Tr::BN * 128) + kr * 128 + ((ch ^ (kr & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(sdS + blk * (Tr::BN * 128) + kr * 128 + ((ch ^ (kr & 7)) << 4)) =
               make_uint4(w[c16 * 4], w[c16 * 4 + 1], w[c16 * 4 + 2], w[c16 * 4 + 3]);
         }
       }
@@ -593,58 +539,61 @@ __global__ void __launch_bounds__(512, 1)
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane: d index (dQᵀ) or query row (dQ)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
+    const uint32_t tQ = tmem + lane_off + Tr::COL_DP;  // dQ of the step sits in the dPᵀ columns
     const bool leader = (warp == 8 && lane == 0);
     bool ok = true;
     for (int i = 0; i < n_q; ++i) {
-      const int b2 = i & 1;
       const int q0 = (i0 + i) * BM;
-      ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full[b2], (i >> 1) & 1, abort_flag));
+      ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full, i & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
 #ifdef FA_TRACE
       btrace(trace_on && leader, 9000 + i);  // dQ ready seen
 #endif
-      // dQ of step i: dPᵀ[i % 2] for d = 128, Sᵀ[i % 2] for d = 64
-      const uint32_t tQ = tmem + lane_off +
-                          (D == 128 ? (b2 ? Tr::COL_DP1 : Tr::COL_DP0) : (b2 ? Tr::COL_S1 : Tr::COL_S0));
       constexpr int NV = Tr::DQ_T ? BM : D;  // values per thread
       uint32_t v[NV];
-      tmem_ld_n<NV>(tQ, v);
+#pragma unroll
+      for (int c = 0; c < NV; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
       tmem_ld_wait();
       tc_fence_before();
-      mbar_arrive(&bars->dq_empty[b2]);
-      // The previous bulk operation must have finished reading the staging buffer.
-      if (leader) bulk_wait_read0();
-      named_bar(1, 128);
-      if constexpr (Tr::DQ_T) {
-        // thread = d index r; staging is [BM][D] row-major fp32
+      mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
 #pragma unroll
-        for (int q = 0; q < BM; ++q) sdQ[q * D + r] = __uint_as_float(v[q]);
-      } else {
-        // thread = query row r; write its D values, rotating the 16-byte
-        // chunk order by lane to spread shared-memory banks
+      for (int part = 0; part < Tr::DQ_PARTS; ++part) {
+        // The previous bulk operation must have finished reading the staging buffer.
+        if (leader) bulk_wait_read0();
+        named_bar(1, 128);
+        constexpr int ROWS = BM / Tr::DQ_PARTS;  // query rows staged per part
+        if constexpr (Tr::DQ_T) {
+          // thread = d index r; staging is [ROWS][D] row-major fp32
 #pragma unroll
-        for (int cc = 0; cc < D / 4; ++cc) {
-          const int c4 = (cc + lane) % (D / 4);
-          float4 x;
-          x.x = __uint_as_float(v[c4 * 4 + 0]);
-          x.y = __uint_as_float(v[c4 * 4 + 1]);
-          x.z = __uint_as_float(v[c4 * 4 + 2]);
-          x.w = __uint_as_float(v[c4 * 4 + 3]);
-          *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
-        }
-      }
-      fence_async_smem();
-      named_bar(1, 128);
-      if (leader) {
-        if (p.dq_mode == 2) {
-          float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
-          bulk_store(dst, sdQ, Tr::DQ_STAGE);
+          for (int q = 0; q < ROWS; ++q) sdQ[q * D + r] = __uint_as_float(v[part * ROWS + q]);
         } else {
-          float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
-          bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+          // thread = query row r; write its D values, rotating the 16-byte
+          // chunk order by lane to spread shared-memory banks
+#pragma unroll
+          for (int cc = 0; cc < D / 4; ++cc) {
+            const int c4 = (cc + lane) % (D / 4);
+            float4 x;
+            x.x = __uint_as_float(v[c4 * 4 + 0]);
+            x.y = __uint_as_float(v[c4 * 4 + 1]);
+            x.z = __uint_as_float(v[c4 * 4 + 2]);
+            x.w = __uint_as_float(v[c4 * 4 + 3]);
+            *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
+          }
         }
-        bulk_commit();
+        fence_async_smem();
+        named_bar(1, 128);
+        if (leader) {
+          const int qr = q0 + part * ROWS;
+          if (p.dq_mode == 2) {
+            float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + qr) * D;
+            bulk_store(dst, sdQ, Tr::DQ_STAGE);
+          } else {
+            float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + qr) * D;
+            bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+          }
+          bulk_commit();
+        }
       }
     }
     if (leader) bulk_wait0();
@@ -872,7 +821,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   return cudaGetLastError();
 }
 
-int bwd_block_rows(int d) { return d == 128 ? 64 : 128; }
+int bwd_block_rows(int d) { (void)d; return 128; }
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
 #define FA_BWD_CASE(TY, DD) \
