@@ -153,6 +153,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
     return FA_ERR_INVALID;
   if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
+  if (int64_t((Nq + 255) / 256) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
@@ -170,6 +171,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
   a.params.Nk = Nk;
   a.params.scale_log2 = scale * 1.4426950408889634f;
   a.params.n_qblocks = (Nq + 255) / 256;
+  a.params.head_group = head_group_for(size_t(Nk) * d * 2 * elem_size(dtype), BH);
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_fwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -196,6 +198,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
     if (!p || !aligned16(p)) return FA_ERR_INVALID;
   if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
+  // grids: (rows, B·H) for the per-row kernels, one CTA per (K/V block, head)
+  if (int64_t(B) * H > 65535 || int64_t((Nk + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
   const int mode = effective_dq_mode(B, H, Nq, Nk, d);
   const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
@@ -212,8 +216,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   BwdParams& p = a.params;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;
   p.dQ = dQ; p.dK = dK; p.dV = dV;
-  p.Dsum = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
-  p.Lsc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.l_off);
+  p.neg_D = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
+  p.neg_Lsc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.l_off);
   p.dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dq_off);
   p.B = B; p.H = H; p.Nq = Nq; p.Nk = Nk;
   p.Nq_pad = bwd_pad_rows(Nq);
@@ -221,6 +225,7 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_kblocks = (Nk + 127) / 128;
   p.dq_mode = mode;
+  p.head_group = head_group_for(size_t(p.Nq_pad) * (size_t(d) * (2 * elem_size(dtype) + 4) + 8), BH);
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;

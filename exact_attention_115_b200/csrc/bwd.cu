@@ -13,34 +13,33 @@
 //   section "Sequence Parallel": dQ receives a contribution from every K/V
 //     block, so it is reduced across CTAs, either by atomic adds into one
 //     buffer or by one buffer per K/V block and a separate reduction kernel.
-//     Both are implemented (dq_mode 1 and 2).  Mode 1 uses bulk reductions
-//     (cp.reduce.async.bulk .add.f32): a whole [BM × d] fp32 tile per
-//     instruction, performed in L2, instead of one atomic per element.
+//     Both are implemented (dq_mode 1 and 2); mode 1 is the default.
 //
-// Kernels: bwd_preprocess (D = rowsum(dO ∘ O), L·log2e into a padded buffer,
-// dQ accumulator cleared), bwd_main (below), bwd_dq_finalise (sum/convert).
+// Kernels: bwd_preprocess (−D = −rowsum(dO ∘ O) and −L·log2e into padded
+// buffers, dQ accumulator cleared), bwd_main (below), bwd_dq_finalise
+// (sum / convert).
 //
-// bwd_main, B200 design.  The two score-like products are computed
-// transposed (keys on TMEM lanes): Sᵀ = K Qᵀ and dPᵀ = V dOᵀ, so that the
-// thread owning key row k holds Pᵀ[k, :] and dSᵀ[k, :] and writes them back
-// to TMEM as the A operand of dV += Pᵀ dO and dK += dSᵀ Q (no shared-memory
-// round trip).  dSᵀ also goes to shared memory for the dQ product:
-//   d = 128: BM = 64 query rows per step, dQᵀ = Kᵀ dSᵀ (M = d = 128);
-//   d = 64:  BM = 128, dQ = dS K (M = BM = 128).
-// Roles (512 threads):
+// bwd_main, B200 design.  One CTA per (K/V block of 128 keys, head), issued
+// heaviest first within groups of heads.  A step handles BM = 128 query rows.
+// The two score-like products are computed transposed (keys on TMEM lanes):
+// Sᵀ = K Qᵀ and dPᵀ = V dOᵀ, so that the thread owning key row k holds
+// Pᵀ[k, :] and dSᵀ[k, :] and writes them back to TMEM as the A operand of
+// dV += Pᵀ dO and dK += dSᵀ Q (no shared-memory round trip).  dSᵀ also goes
+// to shared memory (one buffer) for the dQ product:
+//   d = 128: dQᵀ = Kᵀ dSᵀ (M = d = 128), reduced from registers with one
+//            coalesced red.global.add.f32 per warp and query row;
+//   d = 64:  dQ = dS K (M = BM = 128), staged in shared memory and reduced
+//            with one bulk reduce-add (cp.reduce.async.bulk .add.f32).
+// Roles (512 threads, setmaxnreg split 136 / 136 / 104 registers):
 //   warpgroups 0 and 1: thread = key row; warpgroup c computes P and dS for
-//                half of each step's query columns, and writes half of the
-//                final dK/dV columns;
-//   warpgroup 2: reads dQ from TMEM, stages it in shared memory, issues the
-//                bulk reduction (or partial store);
+//                query columns [64c, 64c + 64) of each step, and writes half
+//                of the final dK/dV columns;
+//   warpgroup 2: moves dQ of the step from TMEM to the fp32 accumulator;
 //   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: TMA producer.
-// The dSᵀ shared-memory tile is double buffered, so step i's dS is written
-// while step i-1's dQ product still reads the other buffer.
-// TMEM (512 columns), d = 128: Sᵀ[2] | dPᵀ[2] | dV | dK (64,64,64,64,128,128);
-//                    d = 64:  Sᵀ[2] | dPᵀ | dV | dK (128,128,128,64,64).
-// Sᵀ is double buffered so the next step's Sᵀ MMA runs while the current
-// step is still in the softmax warps; dQ of step i reuses Sᵀ[i % 2] once
-// Pᵀ has been consumed by the dV product.
+// TMEM (512 columns): Sᵀ | dPᵀ | dV | dK (128, 128, d, d).  dQ of a step is
+// written into the dPᵀ columns once dK has read dSᵀ from them; the next dPᵀ
+// waits until warpgroup 2 has the dQ values in registers.  Q (with −L·log2e
+// and −D) is double buffered, dO single buffered.
 #define FA_SITE_BASE 20000
 #include "common.cuh"
 #include "launch.h"
@@ -66,6 +65,9 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
                "r"(smem_u32(src)), "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void red_add_f32(float* dst, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(v) : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() {
@@ -105,10 +107,10 @@ struct BwdTraits {
   static constexpr int Q_TILE = BM * D * ES;         // bytes of a Q (or dO) tile
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int DS_TILE = BN * BM * ES;       // dSᵀ, rows = keys, q contiguous
-  // dQ staging: d = 128 drains dQᵀ in four 32-row quarters (16 KB each);
-  // d = 64 stages the whole [BM × 64] fp32 tile (32 KB) at once.
-  static constexpr int DQ_PARTS = D == 128 ? 4 : 1;
-  static constexpr int DQ_STAGE = BM * D * 4 / DQ_PARTS;
+  // dQ staging (d = 64 only): the whole [BM × 64] fp32 tile (32 KB) goes to
+  // shared memory and out with one bulk reduce-add; d = 128 reduces dQᵀ from
+  // registers and needs no staging.
+  static constexpr int DQ_STAGE = DQ_T ? 0 : BM * D * 4;
   // shared-memory offsets (all 1024-aligned).  Q is double buffered (the
   // next step's Sᵀ needs it while this step's dK still reads the current
   // one); dO is single buffered (the next dPᵀ comes after this step's dV).
@@ -129,6 +131,12 @@ struct BwdTraits {
   static_assert(COL_DK + D <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared-memory budget");
   static constexpr int THREADS = 512;
+  // setmaxnreg split; 256·REGS_COMPUTE + 128·(REGS_DQ + REGS_OTHER) must not
+  // exceed the 512 × 128 registers the CTA is launched with.
+  static constexpr int REGS_COMPUTE = 136;
+  static constexpr int REGS_DQ = 136;
+  static constexpr int REGS_OTHER = 104;
+  static_assert(256 * REGS_COMPUTE + 128 * (REGS_DQ + REGS_OTHER) <= THREADS * 128, "register split");
   static constexpr uint32_t F = ElemTraits<T>::fmt;
   static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
   static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV, dK (A in TMEM)
@@ -137,9 +145,9 @@ struct BwdTraits {
 
 #ifdef FA_TRACE
 // One fixed slot per event code (plain stores; no atomics on the critical path).
-__device__ long long g_btrace[16384];
+__device__ long long g_btrace[32768];
 __device__ __forceinline__ void btrace(bool on, int code) {
-  if (!on || code >= 16384) return;
+  if (!on || code >= 32768) return;
   long long t;
   asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
   g_btrace[code] = t;
@@ -198,14 +206,14 @@ __global__ void __launch_bounds__(512, 1)
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int kb = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
+  int bh, kb;  // causal: the first key blocks are seen by the most query tiles
+  grouped_order(blockIdx.x, p.B * p.H, p.n_kblocks, p.head_group, bh, kb);
   const int key0 = kb * Tr::BN;
   const int off = p.Nk - p.Nq;
   int i0, n_q;
   q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
 #ifdef FA_TRACE
-  const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  const bool trace_on = blockIdx.x == 0;
 #endif
 
   if (threadIdx.x == 0) {
@@ -242,6 +250,9 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
+#ifdef FA_TRACE
+  btrace(trace_on && threadIdx.x == 0, 15000);  // set-up done
+#endif
 
   uint8_t* sK = smem + Tr::OFF_K;
   uint8_t* sV = smem + Tr::OFF_V;
@@ -251,7 +262,11 @@ __global__ void __launch_bounds__(512, 1)
   float* sdQ = reinterpret_cast<float*>(smem + Tr::OFF_DQ);
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
 
+  // Register split (the CTA launches with 128 per thread): the compute and
+  // dQ warpgroups hold a step's TMEM columns in registers, the MMA / TMA
+  // warpgroup (warps 12-15) needs few.  Each role sets its own count.
   if (warp >= 14) {
+    regs_dec<Tr::REGS_OTHER>();
 #ifdef FA_TRACE
     if (warp == 14 && lane == 0 && trace_on) {
       for (int g = 0; g < n_q; ++g) {
@@ -262,6 +277,7 @@ __global__ void __launch_bounds__(512, 1)
 #endif
   } else if (warp == 13) {
     // ------------------------------------------------------------ producer
+    regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
       mbar_arrive_expect_tx(&bars->kv_full, 2 * Tr::KV_TILE);
 #pragma unroll
@@ -280,8 +296,8 @@ __global__ void __launch_bounds__(512, 1)
         for (int c = 0; c < D / 64; ++c)
           tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
         const size_t row = size_t(bh) * p.Nq_pad + q0;
-        bulk_load(sLD + (s * 2 + 0) * BM, p.Lsc + row, BM * 4, bar);
-        bulk_load(sLD + (s * 2 + 1) * BM, p.Dsum + row, BM * 4, bar);
+        bulk_load(sLD + (s * 2 + 0) * BM, p.neg_Lsc + row, BM * 4, bar);
+        bulk_load(sLD + (s * 2 + 1) * BM, p.neg_D + row, BM * 4, bar);
         // dO into its single buffer, once step i-1's dV product has read it
         if (i >= 1 && !MBAR_WAIT(&bars->do_empty, (i - 1) & 1, abort_flag)) break;
         mbar_arrive_expect_tx(&bars->do_full, Tr::Q_TILE);
@@ -297,6 +313,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
+    regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
       const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
@@ -349,6 +366,7 @@ __global__ void __launch_bounds__(512, 1)
       if (ok && n_q > 0)
         ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && MBAR_WAIT(&bars->do_full, 0, abort_flag);
       tc_fence_after();
+      BTRACE(15001);  // K, V, Q0, dO0 landed
       if (ok && n_q > 0) {
         mma_st(colS, dK_k, dQ_k0);
         tc_commit(&bars->s_full);
@@ -407,6 +425,7 @@ __global__ void __launch_bounds__(512, 1)
     // ------------------------------------------------------------ P / dS (thread = key)
     // Two warpgroups; warpgroup cw handles query columns [cw·CWC, (cw+1)·CWC)
     // of each step for all 128 key rows.
+    regs_inc<Tr::REGS_COMPUTE>();
     const int cw = warp >> 2;
     const int quad = warp & 3;
     const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
@@ -422,8 +441,9 @@ __global__ void __launch_bounds__(512, 1)
     for (int i = 0; i < n_q; ++i) {
       const int s = i & 1;
       const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
-      const float* sL = sLD + (s * 2 + 0) * BM + cw * CWC;
-      const float* sDv = sLD + (s * 2 + 1) * BM + cw * CWC;
+      // −L·log2e and −D of this warpgroup's query columns (16-byte aligned)
+      const float4* sL4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 0) * BM + cw * CWC);
+      const float4* sD4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 1) * BM + cw * CWC);
       // ---- P = exp2(S·c − L·log2e), causal / ragged masking
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, i & 1, abort_flag));
       tc_fence_after();
@@ -432,36 +452,46 @@ __global__ void __launch_bounds__(512, 1)
       btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // got S
 #endif
       const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
-      float P[CWC];
+      uint32_t Pk[CWC / 2];  // P as packed pairs of the input type
       const uint64_t c2 = pk2(sl2, sl2);
-      // 32 columns at a time: load, exponentiate, pack to bf16 pairs, store
-      // Pᵀ back to TMEM into the columns this warpgroup has already read (the
-      // other warpgroup may still be reading its own half); the fp32 P stays
-      // in registers for dS.
+      // Load the warpgroup's CWC columns at once (one TMEM round trip), then
+      // 32 at a time: exponentiate, pack to pairs of the input type, store Pᵀ
+      // back to TMEM into the columns this warpgroup has read (the other
+      // warpgroup may still be reading its own half).  The packed P stays in
+      // registers for dS, so dS uses the same rounded P as the dV product.
+      uint32_t u[CWC];
+#pragma unroll
+      for (int c = 0; c < CWC; c += 32)
+        tmem_ld32(tS + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
+      tmem_ld_wait();
+#ifdef FA_TRACE
+      btrace(trace_on && lane == 0, 17000 + (cw * 4 + quad) * 20 + i);  // S in registers
+#endif
 #pragma unroll
       for (int c = 0; c < CWC; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tS + cw * CWC + c, u);
-        tmem_ld_wait();
-        uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q = c + e;
-          const float2 x = upk2(ffma2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])), c2,
-                                      pk2(-sL[q], -sL[q + 1])));
-          float p0 = ex2(x.x), p1 = ex2(x.y);
-          if (need_mask) {
-            if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
-            if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
+        for (int e = 0; e < 32; e += 4) {
+          const float4 nl = sL4[(c + e) >> 2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int q = c + e + 2 * h2;
+            const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2,
+                                        h2 ? pk2(nl.z, nl.w) : pk2(nl.x, nl.y)));
+            float p0 = ex2(x.x), p1 = ex2(x.y);
+            if (need_mask) {
+              if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
+              if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
+            }
+            Pk[q >> 1] = ElemTraits<T>::pack2(p0, p1);
           }
-          P[q] = p0;
-          P[q + 1] = p1;
-          w[e / 2] = ElemTraits<T>::pack2(p0, p1);
         }
-        tmem_st16(tS + cw * CWC + c / 2, w);
+        tmem_st16(tS + cw * CWC + c / 2, Pk + (c >> 1));
       }
       tmem_st_wait();
       tc_fence_before();
+#ifdef FA_TRACE
+      btrace(trace_on && lane == 0, 12000 + (cw * 4 + quad) * 20 + i);  // P done
+#endif
       mbar_arrive(&bars->p_ready);
 
       // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
@@ -472,20 +502,29 @@ __global__ void __launch_bounds__(512, 1)
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (i - 1) & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
+#ifdef FA_TRACE
+      btrace(trace_on && lane == 0, 11000 + (cw * 4 + quad) * 20 + i);  // dP seen, dS buffer free
+#endif
       const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
       for (int c = 0; c < CWC; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tDP + cw * CWC + c, u);
+        // one 32-column TMEM load per chunk (measured faster here than
+        // loading all CWC columns before the arithmetic)
+        tmem_ld32(tDP + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
         tmem_ld_wait();
         uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int q = c + e;
-          const uint64_t t = fadd2(pk2(__uint_as_float(u[e]), __uint_as_float(u[e + 1])),
-                                   pk2(-sDv[q], -sDv[q + 1]));
-          const float2 ds = upk2(fmul2(t, fmul2(pk2(P[q], P[q + 1]), sc2)));
-          w[e / 2] = ElemTraits<T>::pack2(ds.x, ds.y);
+        for (int e = 0; e < 32; e += 4) {
+          const float4 nd = sD4[(c + e) >> 2];
+#pragma unroll
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int q = c + e + 2 * h2;
+            const uint64_t t = fadd2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])),
+                                     h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
+            const float2 pq = ElemTraits<T>::unpack2(Pk[q >> 1]);
+            const float2 ds = upk2(fmul2(t, fmul2(pk2(pq.x, pq.y), sc2)));
+            w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
+          }
         }
         tmem_st16(tDP + cw * CWC + c / 2, w);
 #pragma unroll
@@ -496,17 +535,24 @@ __global__ void __launch_bounds__(512, 1)
               make_uint4(w[c16 * 4], w[c16 * 4 + 1], w[c16 * 4 + 2], w[c16 * 4 + 3]);
         }
       }
+#ifdef FA_TRACE
+      btrace(trace_on && lane == 0, 18000 + (cw * 4 + quad) * 20 + i);  // dS computed and issued
+#endif
       fence_async_smem();
       tmem_st_wait();
       tc_fence_before();
 #ifdef FA_TRACE
       btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
+      btrace(trace_on && lane == 0, 13000 + (cw * 4 + quad) * 20 + i);
 #endif
       mbar_arrive(&bars->ds_ready);
     }
     // ---- dK, dV out (once per CTA); warpgroup cw writes columns [cw·D/2, (cw+1)·D/2)
     if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dkv_done, 0, abort_flag));
     tc_fence_after();
+#ifdef FA_TRACE
+    btrace(trace_on && lane == 0, 14000 + (cw * 4 + quad));  // dK, dV complete in TMEM
+#endif
     if (ok) {
       const size_t rowoff = (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
 #pragma unroll 1
@@ -536,6 +582,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else {
     // ------------------------------------------------------------ dQ (warpgroup 2)
+    regs_inc<Tr::REGS_DQ>();
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane: d index (dQᵀ) or query row (dQ)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
@@ -550,46 +597,58 @@ __global__ void __launch_bounds__(512, 1)
 #ifdef FA_TRACE
       btrace(trace_on && leader, 9000 + i);  // dQ ready seen
 #endif
-      constexpr int NV = Tr::DQ_T ? BM : D;  // values per thread
-      uint32_t v[NV];
+      if constexpr (Tr::DQ_T) {
+        // thread = d index r, TMEM column q = query row q0 + q.  All BM
+        // columns come to registers first, so the dPᵀ columns are released
+        // after one TMEM round trip; then for each q a warp adds 32
+        // consecutive floats (one 128-byte line) of the fp32 accumulator
+        // (mode 1), or stores them into this K/V block's partial (mode 2).
+        uint32_t v[BM];
 #pragma unroll
-      for (int c = 0; c < NV; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
+        for (int c = 0; c < BM; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
+        float* dst = p.dq_mode == 2
+                         ? p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D + r
+                         : p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D + r;
+        if (p.dq_mode == 2) {
 #pragma unroll
-      for (int part = 0; part < Tr::DQ_PARTS; ++part) {
+          for (int q = 0; q < BM; ++q) dst[q * D] = __uint_as_float(v[q]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < BM; ++q) red_add_f32(dst + q * D, __uint_as_float(v[q]));
+        }
+      } else {
+        uint32_t v[D];  // thread = query row r: its D values
+#pragma unroll
+        for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->dq_empty);  // the dP columns may take the next dPᵀ
         // The previous bulk operation must have finished reading the staging buffer.
         if (leader) bulk_wait_read0();
         named_bar(1, 128);
-        constexpr int ROWS = BM / Tr::DQ_PARTS;  // query rows staged per part
-        if constexpr (Tr::DQ_T) {
-          // thread = d index r; staging is [ROWS][D] row-major fp32
+        // write the row's D values, rotating the 16-byte chunk order by lane
+        // to spread shared-memory banks
 #pragma unroll
-          for (int q = 0; q < ROWS; ++q) sdQ[q * D + r] = __uint_as_float(v[part * ROWS + q]);
-        } else {
-          // thread = query row r; write its D values, rotating the 16-byte
-          // chunk order by lane to spread shared-memory banks
-#pragma unroll
-          for (int cc = 0; cc < D / 4; ++cc) {
-            const int c4 = (cc + lane) % (D / 4);
-            float4 x;
-            x.x = __uint_as_float(v[c4 * 4 + 0]);
-            x.y = __uint_as_float(v[c4 * 4 + 1]);
-            x.z = __uint_as_float(v[c4 * 4 + 2]);
-            x.w = __uint_as_float(v[c4 * 4 + 3]);
-            *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
-          }
+        for (int cc = 0; cc < D / 4; ++cc) {
+          const int c4 = (cc + lane) % (D / 4);
+          float4 x;
+          x.x = __uint_as_float(v[c4 * 4 + 0]);
+          x.y = __uint_as_float(v[c4 * 4 + 1]);
+          x.z = __uint_as_float(v[c4 * 4 + 2]);
+          x.w = __uint_as_float(v[c4 * 4 + 3]);
+          *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
         }
         fence_async_smem();
         named_bar(1, 128);
         if (leader) {
-          const int qr = q0 + part * ROWS;
           if (p.dq_mode == 2) {
-            float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + qr) * D;
+            float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
             bulk_store(dst, sdQ, Tr::DQ_STAGE);
           } else {
-            float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + qr) * D;
+            float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
             bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
           }
           bulk_commit();
@@ -599,6 +658,9 @@ __global__ void __launch_bounds__(512, 1)
     if (leader) bulk_wait0();
   }
 
+#ifdef FA_TRACE
+  btrace(trace_on && lane == 0, 14100 + warp);  // warp finished
+#endif
   tc_fence_before();
   __syncthreads();
   if (warp == 12) {
@@ -607,8 +669,9 @@ __global__ void __launch_bounds__(512, 1)
   }
 }
 
-// D = rowsum(dO ∘ O); L·log2e copied into a padded buffer (+inf on padding
-// rows, so their P is 0); in mode 1 the fp32 dQ accumulator is cleared.
+// −D = −rowsum(dO ∘ O) and −L·log2e into padded buffers (−inf on padding
+// rows, so their P is 0), stored negated so the main kernel adds them; in
+// mode 1 the fp32 dQ accumulator is cleared.
 // A group of D/8 lanes handles one row (8 elements per lane).
 template <typename T, int D>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
@@ -637,8 +700,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   for (int o = LPR / 2; o > 0; o >>= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, o);
   const size_t row = size_t(bh) * p.Nq_pad + q;
   if (sl == 0) {
-    p.Dsum[row] = q < p.Nq ? dsum : 0.f;
-    p.Lsc[row] = lsc;
+    p.neg_D[row] = q < p.Nq ? -dsum : 0.f;
+    p.neg_Lsc[row] = -lsc;
   }
   if (p.dq_mode == 1) {
     float4* z = reinterpret_cast<float4*>(p.dQacc + row * D + sl * 8);
@@ -805,12 +868,22 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   auto kern = bwd_main_kernel<T, D, CAUSAL>;
   e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
+  // setmaxnreg.inc draws on the registers the CTA was launched with: refuse
+  // to launch if the compiled count cannot cover the split.
+  static int regs_ok = -1;
+  if (regs_ok < 0) {
+    cudaFuncAttributes attr;
+    e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
+    if (e != cudaSuccess) return e;
+    regs_ok = attr.numRegs * Tr::THREADS >= 256 * Tr::REGS_COMPUTE + 128 * (Tr::REGS_DQ + Tr::REGS_OTHER);
+  }
+  if (!regs_ok) return cudaErrorInvalidConfiguration;
   if (a.ev_start) {
     e = cudaEventRecord(a.ev_start, a.stream);
     if (e != cudaSuccess) return e;
   }
-  kern<<<dim3(p.n_kblocks, p.H, p.B), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV,
-                                                                               a.tmdO, p);
+  kern<<<dim3(p.n_kblocks * BH), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV,
+                                                                          a.tmdO, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.ev_stop) {
@@ -845,9 +918,9 @@ FA_ERROR_ACCESSOR(take_error_bwd)
 #ifdef FA_TRACE
 }  // namespace fa
 extern "C" int fa_btrace_read(long long* out, int max) {
-  const int n = max < 16384 ? max : 16384;
+  const int n = max < 32768 ? max : 32768;
   cudaMemcpyFromSymbol(out, fa::g_btrace, sizeof(long long) * n);
-  static long long zeros[16384];
+  static long long zeros[32768];
   cudaMemcpyToSymbol(fa::g_btrace, zeros, sizeof(zeros));
   return n;
 }

@@ -54,6 +54,23 @@ __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// Launch order of a 1-D grid over (head, block) pairs.  Heads (b·H + h) go in
+// groups of `group`; inside a group the CTAs run block index by block index,
+// every head of the group at each index.  The caller numbers its blocks so
+// that index 0 is the most work (the longest causal row or column range):
+// the hardware then starts the heavy CTAs first and the short ones fill the
+// end of the launch, while the CTAs alive at one time touch the inputs of
+// only one or two groups of heads, sized on the host to stay in L2.
+__device__ __forceinline__ void grouped_order(int lin, int BH, int nblk, int group, int& bh,
+                                              int& blk) {
+  const int per_group = group * nblk;
+  const int g = lin / per_group;
+  const int rem = lin - g * per_group;
+  const int gh = min(group, BH - g * group);  // heads in this group (the last one may be short)
+  blk = rem / gh;
+  bh = g * group + (rem - blk * gh);
+}
+
 __device__ __forceinline__ unsigned long long globaltimer_ns() {
   unsigned long long t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -186,12 +186,12 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
 
   const int n_qb = p.n_qblocks;
-  const int qb = CAUSAL ? (n_qb - 1 - int(blockIdx.x)) : int(blockIdx.x);  // heavy blocks first
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
+  int bh, blk;
+  grouped_order(blockIdx.x, p.B * p.H, n_qb, p.head_group, bh, blk);
+  const int qb = CAUSAL ? n_qb - 1 - blk : blk;  // causal: the last query blocks see the most keys
   const int q_row0 = qb * 256;
 #ifdef FA_TRACE
-  const bool trace_on = blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0;
+  const bool trace_on = blockIdx.x == 0;
 #endif
   const int off = p.Nk - p.Nq;  // bottom-right causal alignment
 
@@ -597,7 +597,7 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
     regs_ok = attr.numRegs * Tr::THREADS >= 256 * Tr::REGS_SOFTMAX + 128 * Tr::REGS_OTHER;
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
-  dim3 grid(a.params.n_qblocks, a.params.H, a.params.B);
+  dim3 grid(a.params.n_qblocks * a.params.H * a.params.B);
   kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.params);
   return cudaGetLastError();
 }

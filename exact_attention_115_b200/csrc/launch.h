@@ -16,6 +16,7 @@ struct FwdParams {
   int B, H, Nq, Nk;
   float scale_log2;  // scale * log2(e)
   int n_qblocks;     // ceil(Nq / 256): one CTA per 256 query rows
+  int head_group;    // heads per launch-order group (see head_group_for)
 };
 
 struct FwdLaunch {
@@ -38,14 +39,15 @@ struct BwdParams {
   void* dQ;
   void* dK;
   void* dV;
-  float* Dsum;    // [B*H, Nq_pad] rowsum(dO * O), padded rows zero
-  float* Lsc;     // [B*H, Nq_pad] L * log2(e), padded rows +inf
+  float* neg_D;    // [B*H, Nq_pad] -rowsum(dO * O), padded rows zero
+  float* neg_Lsc;  // [B*H, Nq_pad] -L * log2(e), padded rows -inf
   float* dQacc;   // [B*H, Nq_pad, d] fp32 (mode 1) or [nkv, B*H, Nq_pad, d] (mode 2)
   int B, H, Nq, Nk, Nq_pad;
   float scale;        // softmax scale
   float scale_log2;   // scale * log2(e)
   int n_kblocks;      // ceil(Nk / 128)
   int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials
+  int head_group;     // heads per launch-order group (see head_group_for)
 };
 
 struct BwdLaunch {
@@ -56,6 +58,19 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a);
+
+// Heads per launch-order group: as many as keep the bytes one head's CTAs
+// share (K and V in the forward; Q, dO, the fp32 dQ accumulator, L and D in
+// the backward) within a slice of L2, at least 1 and at most B·H.
+#ifndef FA_L2_GROUP_BYTES
+#define FA_L2_GROUP_BYTES (48ull << 20)
+#endif
+inline int head_group_for(size_t bytes_per_head, int BH) {
+  size_t g = bytes_per_head ? FA_L2_GROUP_BYTES / bytes_per_head : size_t(BH);
+  if (g < 1) g = 1;
+  if (g > size_t(BH)) g = size_t(BH);
+  return int(g);
+}
 // Query rows per backward step (the TMA box height of Q and dO).
 int bwd_block_rows(int d);
 
