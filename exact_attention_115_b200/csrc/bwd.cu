@@ -23,9 +23,10 @@
 // heaviest first within groups of heads.  A step handles BM = 128 query rows.
 // The two score-like products are computed transposed (keys on TMEM lanes):
 // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ, so that the thread owning key row k holds
-// Pᵀ[k, :] and dSᵀ[k, :] and writes them back to TMEM as the A operand of
-// dV += Pᵀ dO and dK += dSᵀ Q (no shared-memory round trip).  dSᵀ also goes
-// to shared memory (one buffer) for the dQ product:
+// Pᵀ[k, :] and dSᵀ[k, :].  Pᵀ goes back to TMEM as the A operand of
+// dV += Pᵀ dO; dSᵀ goes to shared memory (one buffer, key rows, 128-byte
+// swizzled), where it is the K-major A operand of dK += dSᵀ Q and the
+// MN-major operand of the dQ product:
 //   d = 128: dQᵀ = Kᵀ dSᵀ (M = d = 128), reduced from registers with one
 //            coalesced red.global.add.f32 per warp and query row;
 //   d = 64:  dQ = dS K (M = BM = 128), staged in shared memory and reduced
@@ -36,8 +37,9 @@
 //                of the final dK/dV columns;
 //   warpgroup 2: moves dQ of the step from TMEM to the fp32 accumulator;
 //   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: TMA producer.
-// TMEM (512 columns): Sᵀ | dPᵀ | dV | dK (128, 128, d, d).  dQ of a step is
-// written into the dPᵀ columns once dK has read dSᵀ from them; the next dPᵀ
+// TMEM (512 columns): Sᵀ | dPᵀ | dV | dK (128, 128, d, d).  Per step the
+// MMA order is dV, next Sᵀ, dQ, dK, next dPᵀ: dQ lands in the dPᵀ columns
+// (read by then), warpgroup 2 drains it while dK runs, and the next dPᵀ
 // waits until warpgroup 2 has the dQ values in registers.  Q (with −L·log2e
 // and −D) is double buffered, dO single buffered.
 #define FA_SITE_BASE 20000
@@ -139,7 +141,7 @@ struct BwdTraits {
   static_assert(256 * REGS_COMPUTE + 128 * (REGS_DQ + REGS_OTHER) <= THREADS * 128, "register split");
   static constexpr uint32_t F = ElemTraits<T>::fmt;
   static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
-  static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV, dK (A in TMEM)
+  static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV (A in TMEM), dK (A = dSᵀ K-major)
   static constexpr uint32_t IDESC_DQ = make_idesc(F, 128, DQ_T ? BM : D, 1, 1);
 };
 
@@ -327,6 +329,7 @@ __global__ void __launch_bounds__(512, 1)
       const uint64_t dQ_mn0 = sw128_desc(aQ, Tr::Q_CHUNK, 1024);
       const uint64_t dO_mn = sw128_desc(adO, Tr::Q_CHUNK, 1024);
       const uint64_t dS_mn = sw128_desc(adS, Tr::BN * 128, 1024);
+      const uint64_t dS_k = sw128_desc(adS, 16, 1024);
       auto stg = [](uint64_t d0, int s) { return d0 + uint64_t(s) * uint64_t(Tr::Q_TILE >> 4); };
 
       // Sᵀ (or dPᵀ) = X[128 keys × D] · Y[BM × D]ᵀ, both K-major.
@@ -348,6 +351,16 @@ __global__ void __launch_bounds__(512, 1)
         for (int ks = 0; ks < BM / 16; ++ks)
           mma_ts<false>(dcol, acol + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
                         dy + uint64_t(ks * 128), Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
+      };
+      // dK [128 × D] += dSᵀ [128 keys × BM] (shared memory, K-major: key rows of
+      // BM query values in 64-column blocks) · Q [BM × D] (MN-major).
+      auto mma_dk = [&](uint64_t dy, bool acc) {
+#pragma unroll
+        for (int ks = 0; ks < BM / 16; ++ks) {
+          const uint64_t oa = uint64_t((ks >> 2) * (Tr::BN * 128 / 16) + (ks & 3) * 2);
+          mma_ss<false>(colDK, dS_k + oa, dy + uint64_t(ks * 128), Tr::IDESC_GRAD,
+                        (acc || ks > 0) ? 1u : 0u);
+        }
       };
       // dQᵀ [D × BM] = Kᵀ · dSᵀ  (d = 128), or dQ [BM × D] = dS · K (d = 64);
       // both operands MN-major, K dimension = the 128 keys.
@@ -399,12 +412,14 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_after();
         if (!ok) break;
         BTRACE(4000 + i);
-        mma_grad(colDK, colDP, stg(dQ_mn0, s), i > 0);
-        tc_commit(&bars->q_empty[s]);
-        if (!more) tc_commit(&bars->dkv_done);
+        // dQ first (into the dPᵀ columns, which the compute warpgroups have
+        // read), so warpgroup 2 drains it while the tensor core runs dK.
         mma_dq(colDP);
         tc_commit(&bars->dq_full);
+        mma_dk(stg(dQ_mn0, s), i > 0);
+        tc_commit(&bars->q_empty[s]);
         tc_commit(&bars->ds_free);
+        if (!more) tc_commit(&bars->dkv_done);
         BTRACE(5000 + i);
 #ifdef FA_TRACE
         if (trace_on) tc_commit(&bars->watch);
@@ -526,7 +541,6 @@ __global__ void __launch_bounds__(512, 1)
             w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
           }
         }
-        tmem_st16(tDP + cw * CWC + c / 2, w);
 #pragma unroll
         for (int c16 = 0; c16 < 4; ++c16) {
           const int col = cw * CWC + c + c16 * 8;  // first query column of this 16-byte chunk
@@ -539,7 +553,6 @@ __global__ void __launch_bounds__(512, 1)
       btrace(trace_on && lane == 0, 18000 + (cw * 4 + quad) * 20 + i);  // dS computed and issued
 #endif
       fence_async_smem();
-      tmem_st_wait();
       tc_fence_before();
 #ifdef FA_TRACE
       btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
