@@ -211,7 +211,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   // (the fp32 path stages its operands without TMA)
   if (dtype != FA_FP32 &&
       (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, bm) || !make_map(&a.tmdO, dO, dtype, d, Nq, BH, bm) ||
-       !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128)))
+       !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128) ||
+       !make_map(&a.tmdK, dK, dtype, d, Nk, BH, 128) || !make_map(&a.tmdV, dV, dtype, d, Nk, BH, 128)))
     return FA_ERR_CUDA;
   BwdParams& p = a.params;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;

@@ -197,6 +197,7 @@ template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                    const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
                     BwdParams p) {
   using Tr = BwdTraits<T, D>;
   constexpr int BM = Tr::BM;
@@ -215,7 +216,10 @@ __global__ void __launch_bounds__(512, 1)
   int i0, n_q;
   q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
 #ifdef FA_TRACE
-  const bool trace_on = blockIdx.x == 0;
+#ifndef FA_TRACE_CTA
+#define FA_TRACE_CTA 0
+#endif
+  const bool trace_on = blockIdx.x == FA_TRACE_CTA;
 #endif
 
   if (threadIdx.x == 0) {
@@ -560,37 +564,67 @@ __global__ void __launch_bounds__(512, 1)
 #endif
       mbar_arrive(&bars->ds_ready);
     }
-    // ---- dK, dV out (once per CTA); warpgroup cw writes columns [cw·D/2, (cw+1)·D/2)
+    // ---- dK, dV of the tile: TMEM → registers (packed to the dtype) → shared
+    // memory → TMA tensor stores.  The Q stages are free by now: dV goes to
+    // stage 0 and dK to stage 1, each as D/64 blocks of BN rows × 128 bytes,
+    // 128-byte swizzled like the loads; warpgroup cw stages columns
+    // [cw·D/2, (cw+1)·D/2).  The tensor maps clip rows past Nk.
     if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dkv_done, 0, abort_flag));
     tc_fence_after();
 #ifdef FA_TRACE
     btrace(trace_on && lane == 0, 14000 + (cw * 4 + quad));  // dK, dV complete in TMEM
 #endif
-    if (ok) {
-      const size_t rowoff = (size_t(bh) * p.Nk + (key_live ? key : 0)) * D;
-#pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV) + cw * (D / 2);
-        T* out = reinterpret_cast<T*>(which ? p.dK : p.dV) + rowoff + cw * (D / 2);
-#pragma unroll 1
-        for (int c = 0; c < D / 2; c += 32) {
-          uint32_t u[32];
-          tmem_ld32(tcol + c, u);
-          tmem_ld_wait();
-          if (key_live) {
+    // Stage one matrix's columns of this warpgroup (zeros if the tile saw no query).
+    auto stage_out = [&](int which) {
+      const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV) + cw * (D / 2);
+      uint8_t* stage = sQ + which * Tr::Q_TILE;
 #pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 v = make_uint4(0, 0, 0, 0);
-              if (n_q > 0) {
-                v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]), __uint_as_float(u[e + 1]));
-                v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]), __uint_as_float(u[e + 3]));
-                v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]), __uint_as_float(u[e + 5]));
-                v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]), __uint_as_float(u[e + 7]));
-              }
-              *reinterpret_cast<uint4*>(out + c + e) = v;
-            }
+      for (int c = 0; c < D / 2; c += 32) {
+        uint32_t v[32];
+        tmem_ld32(tcol + c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int c8 = 0; c8 < 32; c8 += 8) {
+          const int col = cw * (D / 2) + c + c8;  // first column of this 16-byte chunk
+          const int blk = col >> 6, ch = (col >> 3) & 7;
+          uint4 x = make_uint4(0u, 0u, 0u, 0u);
+          if (n_q > 0) {
+            x.x = ElemTraits<T>::pack2(__uint_as_float(v[c8]), __uint_as_float(v[c8 + 1]));
+            x.y = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 2]), __uint_as_float(v[c8 + 3]));
+            x.z = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 4]), __uint_as_float(v[c8 + 5]));
+            x.w = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 6]), __uint_as_float(v[c8 + 7]));
           }
+          *reinterpret_cast<uint4*>(stage + blk * Tr::KV_CHUNK + kr * 128 + ((ch ^ (kr & 7)) << 4)) = x;
         }
+      }
+      fence_async_smem();
+    };
+    if constexpr (D == 128) {
+      // Warpgroup cw owns column block cw of both matrices: it stores dV's
+      // block while it stages dK's.
+      const bool elected = kr == 0;
+#pragma unroll
+      for (int which = 0; which < 2; ++which) {
+        if (ok) stage_out(which);
+        ok = named_bar_and(2 + cw, 128, ok);
+        if (ok && elected) {
+          tma_store_3d(which ? &tmdK : &tmdV, sQ + which * Tr::Q_TILE + cw * Tr::KV_CHUNK, cw * 64,
+                       key0, bh);
+          bulk_commit();
+        }
+      }
+      if (elected) bulk_wait_read0();  // the staging must outlive TMA's reads
+    } else {
+      if (ok) {
+        stage_out(0);
+        stage_out(1);
+      }
+      // Both warpgroups share the one column block: one thread stores it.
+      if (named_bar_and(2, 256, ok) && threadIdx.x == 0) {
+        tma_store_3d(&tmdV, sQ, 0, key0, bh);
+        tma_store_3d(&tmdK, sQ + Tr::Q_TILE, 0, key0, bh);
+        bulk_commit();
+        bulk_wait_read0();
       }
     }
   } else {
@@ -895,8 +929,8 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
     e = cudaEventRecord(a.ev_start, a.stream);
     if (e != cudaSuccess) return e;
   }
-  kern<<<dim3(p.n_kblocks * BH), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV,
-                                                                          a.tmdO, p);
+  kern<<<dim3(p.n_kblocks * BH), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(
+      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK, a.tmdV, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.ev_stop) {

@@ -52,6 +52,7 @@ struct BwdParams {
 
 struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmdO;
+  CUtensorMap tmdK, tmdV;  // outputs, written by TMA stores
   BwdParams params;
   cudaStream_t stream;
   cudaEvent_t ev_start, ev_stop;  // optional timing events around the main kernel
