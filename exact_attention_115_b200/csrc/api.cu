@@ -158,7 +158,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, 128) || !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) ||
-      !make_map(&a.tmV, V, dtype, d, Nk, BH, 128))
+      !make_map(&a.tmV, V, dtype, d, Nk, BH, 128) || !make_map(&a.tmO, O, dtype, d, Nq, BH, 128))
     return FA_ERR_CUDA;
   a.params.Q = Q;
   a.params.K = K;

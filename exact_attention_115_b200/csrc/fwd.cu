@@ -173,7 +173,8 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 template <typename T, int D, bool CAUSAL>
 __global__ void __launch_bounds__(384, 1)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-               const __grid_constant__ CUtensorMap tmV, FwdParams p) {
+               const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+               FwdParams p) {
   using Tr = FwdTraits<T, D>;
   constexpr bool TF32 = ElemTraits<T>::tf32;
   extern __shared__ uint8_t smem_raw[];
@@ -534,14 +535,14 @@ __global__ void __launch_bounds__(384, 1)
     if (ok) {
       const float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;
       const bool live = qi < p.Nq;
-      T* orow = reinterpret_cast<T*>(p.O) + (size_t(bh) * p.Nq + (live ? qi : 0)) * D;
+      if constexpr (TF32) {
+        float* orow = reinterpret_cast<float*>(p.O) + (size_t(bh) * p.Nq + (live ? qi : 0)) * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t u[32];
-        tmem_ld32(tO + c, u);
-        tmem_ld_wait();
-        if (live) {
-          if constexpr (TF32) {
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tO + c, u);
+          tmem_ld_wait();
+          if (live) {
 #pragma unroll
             for (int e = 0; e < 32; e += 4) {
               float4 v = make_float4(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv,
@@ -549,25 +550,46 @@ __global__ void __launch_bounds__(384, 1)
                                      __uint_as_float(u[e + 3]) * inv);
               *reinterpret_cast<float4*>(orow + c + e) = v;
             }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; e += 8) {
-              uint4 v;
-              v.x = ElemTraits<T>::pack2(__uint_as_float(u[e]) * inv, __uint_as_float(u[e + 1]) * inv);
-              v.y = ElemTraits<T>::pack2(__uint_as_float(u[e + 2]) * inv,
-                                         __uint_as_float(u[e + 3]) * inv);
-              v.z = ElemTraits<T>::pack2(__uint_as_float(u[e + 4]) * inv,
-                                         __uint_as_float(u[e + 5]) * inv);
-              v.w = ElemTraits<T>::pack2(__uint_as_float(u[e + 6]) * inv,
-                                         __uint_as_float(u[e + 7]) * inv);
-              *reinterpret_cast<uint4*>(orow + c + e) = v;
-            }
           }
         }
+      } else {
+        // O/ℓ to the tile's Q buffer (every MMA of the tile is complete), in
+        // the 128-byte swizzled layout of the loads; TMA writes it below.
+        uint8_t* stage = smem + t * Tr::TILE;  // = sQ[t], without indexing the array
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t u[32];
+          tmem_ld32(tO + c, u);
+          tmem_ld_wait();
+#pragma unroll
+          for (int c8 = 0; c8 < 32; c8 += 8) {
+            const int col = c + c8;  // first column of this 16-byte chunk
+            const int blk = col / Tr::AW, ch = (col % Tr::AW) / 8;
+            uint4 v;
+            v.x = ElemTraits<T>::pack2(__uint_as_float(u[c8]) * inv, __uint_as_float(u[c8 + 1]) * inv);
+            v.y = ElemTraits<T>::pack2(__uint_as_float(u[c8 + 2]) * inv, __uint_as_float(u[c8 + 3]) * inv);
+            v.z = ElemTraits<T>::pack2(__uint_as_float(u[c8 + 4]) * inv, __uint_as_float(u[c8 + 5]) * inv);
+            v.w = ElemTraits<T>::pack2(__uint_as_float(u[c8 + 6]) * inv, __uint_as_float(u[c8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(stage + blk * Tr::CHUNK + r * 128 + ((ch ^ (r & 7)) << 4)) = v;
+          }
+        }
+        fence_async_smem();
       }
       if (live)
         p.L[size_t(bh) * p.Nq + qi] =
             row_sum > 0.f ? (m_ref + lg2(row_sum)) * kLn2 : -INFINITY;
+    }
+    if constexpr (!TF32) {
+      // The tile's 128 rows are staged: one thread stores its D/64 column
+      // blocks (rows past Nq are clipped by the tensor map) and waits until
+      // TMA has read them before the CTA may exit.
+      if (named_bar_and(1 + t, 128, ok) && r == 0) {
+#pragma unroll
+        for (int blk = 0; blk < Tr::DC; ++blk)
+          tma_store_3d(&tmO, smem + t * Tr::TILE + blk * Tr::CHUNK, blk * Tr::AW, tile_first_row, bh);
+        bulk_commit();
+        bulk_wait_read0();
+      }
     }
   }
 
@@ -598,7 +620,7 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
   dim3 grid(a.params.n_qblocks * a.params.H * a.params.B);
-  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.params);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.params);
   return cudaGetLastError();
 }
 

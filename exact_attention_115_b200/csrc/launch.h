@@ -21,6 +21,7 @@ struct FwdParams {
 
 struct FwdLaunch {
   CUtensorMap tmQ, tmK, tmV;
+  CUtensorMap tmO;  // output, written by TMA stores (16-bit types)
   FwdParams params;
   cudaStream_t stream;
 };
