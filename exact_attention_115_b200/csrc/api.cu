@@ -153,7 +153,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
     return FA_ERR_INVALID;
   if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
-  if (int64_t((Nq + 255) / 256) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid
+  if (int64_t((Nq + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
@@ -170,7 +170,8 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
   a.params.Nq = Nq;
   a.params.Nk = Nk;
   a.params.scale_log2 = scale * 1.4426950408889634f;
-  a.params.n_qblocks = (Nq + 255) / 256;
+  const int rows = fwd_rows_per_cta(dtype, d);
+  a.params.n_qblocks = (Nq + rows - 1) / rows;
   a.params.head_group = head_group_for(size_t(Nk) * d * 2 * elem_size(dtype), BH);
   a.stream = static_cast<cudaStream_t>(stream);
   return launch_fwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;

@@ -11,19 +11,22 @@
 // K) are masked.  The notes' instruction-level section: the softmax uses
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
-// B200 design (not the pages'): one CTA owns two 128-row Q tiles and
+// B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
+// (fwd_tiles: one for 16-bit d = 128, two otherwise).  With two tiles it
 // ping-pongs them so the tensor core works on one tile while the softmax
-// warps work on the other.  Roles per CTA (384 threads, 3 warpgroups):
-//   warpgroup 0 (warps 0-3)  softmax + correction + epilogue, Q tile 0
-//                            (thread = row), 200 registers
-//   warpgroup 1 (warps 4-7)  the same for Q tile 1, 200 registers
-//   warpgroup 2: warp 8 tcgen05.mma issuer (one thread) and TMEM owner,
-//                warp 9 TMA producer, warps 10-11 idle; 80 registers
-// TMEM (512 columns): S0 | S1 | O0 | O1.  P overwrites S in place (bf16 pairs
-// or tf32) and is read by the P·V MMA straight from TMEM.  The running max is
-// only moved when it grows by more than kRescaleThreshold (log2 units), so
-// the O accumulator is rescaled rarely; the result is exact either way
-// because O and ℓ always share the same reference maximum.
+// warps work on the other; with one tile two CTAs share an SM and interleave
+// the same way.  Roles per CTA (128 threads per tile + 128):
+//   warpgroup t (warps 4t..4t+3)  softmax + correction + epilogue of Q tile t
+//                                 (thread = row), 200 registers
+//   last warpgroup: warp 4·TILES issues the tcgen05 MMAs (one thread) and
+//                   owns TMEM, the next warp is the TMA producer, the rest idle
+// TMEM: S[tiles] | O[tiles] (256 or 512 columns).  P overwrites S in place
+// (bf16 pairs or tf32) and is read by the P·V MMA straight from TMEM.  The
+// running max is only moved when it grows by more than kRescaleThreshold
+// (log2 units), so the O accumulator is rescaled rarely; the result is exact
+// either way because O and ℓ always share the same reference maximum.
+// O is written through the tile's Q buffer (free once the tile's products
+// are done) with TMA tensor stores.
 #define FA_SITE_BASE 10000
 #include "common.cuh"
 #include "launch.h"
@@ -37,6 +40,8 @@ namespace {
 #endif
 constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entries stay <= 2^8
 
+constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 1 : 2; }
+
 template <typename T, int D>
 struct FwdTraits {
   static constexpr int ES = sizeof(T);
@@ -46,13 +51,27 @@ struct FwdTraits {
   static constexpr int CHUNK = 128 * 128;        // bytes of one column block (128 rows)
   static constexpr int TILE = 128 * D * ES;      // bytes of one 128-row tile
   static constexpr int KSTEP = 32 / ES;          // K extent of one MMA instruction
-  static constexpr int NS_RAW = (200 * 1024 - 2 * TILE) / TILE;
+  // 128-row Q tiles per CTA.  With one tile a CTA needs 256 TMEM columns and
+  // under half of shared memory, so two CTAs share an SM: one's softmax runs
+  // while the other's products run, and one's set-up and epilogue overlap the
+  // other's main loop, at the price of loading each K/V tile twice per SM.
+  // With two tiles the CTA ping-pongs its own tiles over one K/V stream.
+  // Measured: one tile is faster for 16-bit d = 128 at causal N = 2048 (+4 %)
+  // and two tiles for d = 64 (+5 %); fp32 keeps two.
+  static constexpr int TILES = fwd_tiles(ElemTraits<T>::tf32, D);
+  static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
+  static constexpr int SMEM_BUDGET = TILES == 1 ? 110 * 1024 : 200 * 1024;  // tiles, per CTA
+  static constexpr int NS_RAW = (SMEM_BUDGET - TILES * TILE) / TILE;
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
-  static constexpr int SMEM_BAR = 2 * TILE + NS * TILE;
+  static constexpr int SMEM_BAR = TILES * TILE + NS * TILE;
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers + alignment slack
-  static constexpr int THREADS = 384;
-  static constexpr int REGS_SOFTMAX = 200;  // per thread, warpgroups 0-1
-  static constexpr int REGS_OTHER = 80;     // per thread, warpgroup 2
+  static constexpr int THREADS = 128 * TILES + 128;
+  static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES]
+  static constexpr int MMA_WARP = 4 * TILES;                // then the TMA producer
+  static constexpr int PRODUCER_WARP = MMA_WARP + 1;
+  // setmaxnreg split of the registers a CTA launches with (65536 / CTAS_PER_SM)
+  static constexpr int REGS_SOFTMAX = TILES == 1 ? 200 : 200;  // per thread, softmax warpgroups
+  static constexpr int REGS_OTHER = TILES == 1 ? 56 : 80;      // per thread, the last warpgroup
   static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
@@ -171,7 +190,7 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 }
 
 template <typename T, int D, bool CAUSAL>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                FwdParams p) {
@@ -190,7 +209,7 @@ __global__ void __launch_bounds__(384, 1)
   int bh, blk;
   grouped_order(blockIdx.x, p.B * p.H, n_qb, p.head_group, bh, blk);
   const int qb = CAUSAL ? n_qb - 1 - blk : blk;  // causal: the last query blocks see the most keys
-  const int q_row0 = qb * 256;
+  const int q_row0 = qb * 128 * Tr::TILES;
 #ifdef FA_TRACE
   const bool trace_on = blockIdx.x == 0;
 #endif
@@ -198,7 +217,7 @@ __global__ void __launch_bounds__(384, 1)
 
   int kv_end = p.Nk;
   if (CAUSAL) {
-    const int q_last = min(q_row0 + 255, p.Nq - 1);
+    const int q_last = min(q_row0 + 128 * Tr::TILES - 1, p.Nq - 1);
     kv_end = min(p.Nk, q_last + off + 1);
   }
   const int n_kv = (kv_end + Tr::BN - 1) / Tr::BN;
@@ -217,11 +236,11 @@ __global__ void __launch_bounds__(384, 1)
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 8) {
-    tmem_alloc(&bars->tmem_base, 512);
+  if (warp == Tr::MMA_WARP) {
+    tmem_alloc(&bars->tmem_base, Tr::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == Tr::PRODUCER_WARP && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -231,21 +250,21 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 
-  uint8_t* sQ[2] = {smem, smem + Tr::TILE};
-  uint8_t* sKV = smem + 2 * Tr::TILE;
+  uint8_t* sQ[2] = {smem, smem + Tr::TILE};  // (the second only with two tiles)
+  uint8_t* sKV = smem + Tr::TILES * Tr::TILE;
 
-  if (warp >= 10) {
+  if (warp > Tr::PRODUCER_WARP) {
     // idle warps of the producer/MMA warpgroup
     regs_dec<Tr::REGS_OTHER>();
 #ifdef FA_TRACE
-    if (warp == 10 && lane == 0 && trace_on && Tr::NS < 8) {
+    if (warp == Tr::PRODUCER_WARP + 1 && lane == 0 && trace_on && Tr::NS < 8) {
       for (int g = 0; g < 4 * n_kv; ++g) {
         if (!MBAR_WAIT(&bars->kv_full[7], g & 1, abort_flag)) break;
         trace_ev(true, 7000 + g);
       }
     }
 #endif
-  } else if (warp == 9) {
+  } else if (warp == Tr::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     regs_dec<Tr::REGS_OTHER>();
     // Lane 0 issues the TMA loads (16-bit types).  fp32 tiles are staged by
@@ -281,7 +300,7 @@ __global__ void __launch_bounds__(384, 1)
     };
     load_tile(0, sQ[0], &bars->q_full[0], q_row0);
     load_kv(0);
-    load_tile(0, sQ[1], &bars->q_full[1], q_row0 + 128);
+    if constexpr (Tr::TILES == 2) load_tile(0, sQ[1], &bars->q_full[1], q_row0 + 128);
     for (int i = 1; i < 2 * n_kv; ++i)
       if (!load_kv(i)) break;
     if (lane == 0) {
@@ -289,14 +308,14 @@ __global__ void __launch_bounds__(384, 1)
       for (int i = max(0, 2 * n_kv - Tr::NS); i < 2 * n_kv; ++i)
         MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       MBAR_WAIT(&bars->q_full[0], 0, abort_flag);
-      MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
+      if constexpr (Tr::TILES == 2) MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
     }
-  } else if (warp == 8) {
+  } else if (warp == Tr::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
       const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO[2] = {tmem + 256, tmem + 256 + D};
+      const uint32_t tO[2] = {tmem + 128 * Tr::TILES, tmem + 128 * Tr::TILES + D};
       const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
       const uint32_t aKV = smem_u32(sKV);
 
@@ -330,6 +349,36 @@ __global__ void __launch_bounds__(384, 1)
         return MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       };
 
+      if constexpr (Tr::TILES == 1) {
+        // One tile: S(j), then (once the softmax has written P(j)) P(j)·V(j)
+        // and S(j+1) into the same columns, in issue order after P·V read P.
+        bool ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+        tc_fence_after();
+        if (ok) issue_qk(0, 0);
+        tc_commit(&bars->s_full[0]);
+        tc_commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int iv = 2 * j + 1, ik = 2 * j + 2;
+          const int sv = iv % Tr::NS, sk = ik % Tr::NS;
+          ok = kv_wait(iv) && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          TRACE(3000 + j);
+          issue_pv(0, sv, j > 0);
+          tc_commit(&bars->o_full[0]);
+          tc_commit(&bars->kv_empty[sv]);
+          TRACE(4000 + j);
+          if (j + 1 < n_kv) {
+            ok = kv_wait(ik);
+            tc_fence_after();
+            if (!ok) break;
+            issue_qk(0, sk);
+            tc_commit(&bars->s_full[0]);
+            tc_commit(&bars->kv_empty[sk]);
+            TRACE(5000 + j);
+          }
+        }
+      } else {
       bool ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
       tc_fence_after();
       if (ok) issue_qk(0, 0);
@@ -393,6 +442,7 @@ __global__ void __launch_bounds__(384, 1)
 #endif
         }
       }
+      }
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -403,7 +453,7 @@ __global__ void __launch_bounds__(384, 1)
     const int qi = q_row0 + t * 128 + r;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 256 + t * D;
+    const uint32_t tO = tmem + lane_off + 128 * Tr::TILES + t * D;
     const float sl2 = p.scale_log2;
     const int tile_first_row = q_row0 + t * 128;
 
@@ -595,9 +645,9 @@ __global__ void __launch_bounds__(384, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == Tr::MMA_WARP) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, Tr::TMEM_COLS);
   }
 }
 
@@ -616,7 +666,7 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
     cudaFuncAttributes attr;
     e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
     if (e != cudaSuccess) return e;
-    regs_ok = attr.numRegs * Tr::THREADS >= 256 * Tr::REGS_SOFTMAX + 128 * Tr::REGS_OTHER;
+    regs_ok = attr.numRegs * Tr::THREADS >= 128 * Tr::TILES * Tr::REGS_SOFTMAX + 128 * Tr::REGS_OTHER;
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
   dim3 grid(a.params.n_qblocks * a.params.H * a.params.B);
@@ -625,6 +675,8 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
 }
 
 int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
+
+int fwd_rows_per_cta(int dtype, int d) { return 128 * fwd_tiles(dtype == FA_FP32, d); }
 
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
 #define FA_FWD_CASE(TY, DD)                                                      \

@@ -15,7 +15,7 @@ struct FwdParams {
   float* L;
   int B, H, Nq, Nk;
   float scale_log2;  // scale * log2(e)
-  int n_qblocks;     // ceil(Nq / 256): one CTA per 256 query rows
+  int n_qblocks;     // ceil(Nq / fwd_rows_per_cta): one CTA per block of query rows
   int head_group;    // heads per launch-order group (see head_group_for)
 };
 
@@ -28,6 +28,8 @@ struct FwdLaunch {
 
 // Elements in one 128-byte swizzled row for the dtype (the TMA box width).
 int fwd_tile_elems(int dtype);
+// Query rows per forward CTA.
+int fwd_rows_per_cta(int dtype, int d);
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a);
 
 struct BwdParams {
