@@ -88,7 +88,7 @@ int effective_dq_mode(int B, int H, int Nq, int Nk, int d) {
 }
 
 struct BwdWorkspace {
-  size_t d_off, l_off, dq_off, total;
+  size_t d_off, l_off, dq_off, ctr_off, total;
 };
 
 BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
@@ -100,7 +100,8 @@ BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
   w.l_off = round_up(BH * rows * sizeof(float), 256);
   w.dq_off = w.l_off + round_up(BH * rows * sizeof(float), 256);
   const size_t dq = BH * rows * size_t(d) * sizeof(float) * (mode == 2 ? nkv : 1);
-  w.total = w.dq_off + round_up(dq, 256);
+  w.ctr_off = w.dq_off + round_up(dq, 256);  // work-item counter of the main kernel
+  w.total = w.ctr_off + 256;
   return w;
 }
 
@@ -136,6 +137,20 @@ cudaError_t set_smem_once(const void* kernel, int bytes) {
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
   if (e == cudaSuccess && track && done_n[dev] < 64) done_k[dev][done_n[dev]++] = kernel;
   return e;
+}
+
+int sm_count() {
+  static std::mutex mu;
+  static int n_sm[kMaxDevices] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  std::lock_guard<std::mutex> lk(mu);
+  if (n_sm[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    n_sm[dev] = n;
+  }
+  return n_sm[dev];
 }
 
 }  // namespace fa
@@ -221,6 +236,7 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   p.neg_D = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.d_off);
   p.neg_Lsc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.l_off);
   p.dQacc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + w.dq_off);
+  p.item_ctr = reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + w.ctr_off);
   p.B = B; p.H = H; p.Nq = Nq; p.Nk = Nk;
   p.Nq_pad = bwd_pad_rows(Nq);
   p.scale = scale;
@@ -326,6 +342,7 @@ int fa_status(void* stream) {
   if (take_error_bwd(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
   if (take_error_decode(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
   if (site != 0) g_last_site = site;
+  if (word & 2) return FA_ERR_CUDA;  // a kernel found its shared memory misaligned (kErrLayout)
   if (word != 0) return FA_ERR_TIMEOUT;
   return FA_OK;
 }

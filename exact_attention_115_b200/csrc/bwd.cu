@@ -35,7 +35,8 @@
 //   warpgroups 0 and 1: thread = key row; warpgroup c computes P and dS for
 //                query columns [64c, 64c + 64) of each step, and writes half
 //                of the final dK/dV columns;
-//   warpgroup 2: moves dQ of the step from TMEM to the fp32 accumulator;
+//   warpgroup 2: moves dQ of the step from TMEM to the fp32 accumulator,
+//                and writes each work item's dK and dV;
 //   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: TMA producer.
 // TMEM (512 columns): Sᵀ | dPᵀ | dV | dK (128, 128, d, d).  Per step the
 // MMA order is dV, next Sᵀ, dQ, dK, next dPᵀ: dQ lands in the dPᵀ columns
@@ -43,6 +44,8 @@
 // waits until warpgroup 2 has the dQ values in registers.  Q (with −L·log2e
 // and −D) is double buffered, dO single buffered.
 #define FA_SITE_BASE 20000
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -89,18 +92,19 @@ struct BwdTraits {
   // shared memory and out with one bulk reduce-add; d = 128 reduces dQᵀ from
   // registers and needs no staging.
   static constexpr int DQ_STAGE = DQ_T ? 0 : BM * D * 4;
-  // shared-memory offsets (all 1024-aligned).  Q is double buffered (the
-  // next step's Sᵀ needs it while this step's dK still reads the current
-  // one); dO is single buffered (the next dPᵀ comes after this step's dV).
-  static constexpr int OFF_K = 0;
-  static constexpr int OFF_V = OFF_K + KV_TILE;
+  // shared-memory offsets (all 1024-aligned).  K is double buffered (the
+  // next work item's K loads while this item runs); Q is double buffered
+  // (the next step's Sᵀ needs it while this step's dK still reads the
+  // current one); V and dO are single buffered.
+  static constexpr int OFF_K = 0;                    // 2 buffers
+  static constexpr int OFF_V = OFF_K + 2 * KV_TILE;
   static constexpr int OFF_Q = OFF_V + KV_TILE;      // 2 stages
   static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;
   static constexpr int OFF_DS = OFF_DO + Q_TILE;
   static constexpr int OFF_DQ = OFF_DS + DS_TILE;
   static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;   // L·log2e and D per Q stage
   static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BM * 4;
-  static constexpr int SMEM_BYTES = OFF_BAR + 512 + 1024;
+  static constexpr int SMEM_BYTES = OFF_BAR + 512;  // the base is checked to be 1024-aligned
   // TMEM columns: Sᵀ | dPᵀ (dQ of the step lands here after dK read dSᵀ) | dV | dK
   static constexpr int COL_S = 0;
   static constexpr int COL_DP = BM;
@@ -131,16 +135,26 @@ __device__ __forceinline__ void btrace(bool on, int code) {
   g_btrace[code] = t;
 }
 #define BTRACE(code) btrace(trace_on, (code))
+// per CTA: globaltimer and clock64 at set-up and at exit
+__device__ long long g_cta_times[4][1024];
 #else
 #define BTRACE(code) ((void)0)
 #endif
 
-// Every barrier below completes once per step except q_full / q_empty (one
-// per Q stage, every other step).  A producer of any of them cannot run two
-// phases ahead of its waiter (each step's signal needs the waiter's
-// previous step to have finished), so parity waits are unambiguous.
+// The kernel is persistent: a CTA takes work items (K/V block, head) in turn
+// and numbers its steps across items (g).  The per-step barriers complete
+// once per step except q_full / q_empty (one per Q stage, every other
+// step); v_full, v_free, dkv_done and dkv_free complete once per work item,
+// k_full[b] / k_free[b] once per item that uses K buffer b (every other
+// item), item_full[s] once per item published in ring slot s.  A producer
+// of any of them cannot run two phases ahead of its waiter (each signal
+// needs the waiter's previous phase to have been seen), so parity waits are
+// unambiguous.
 struct BwdBarriers {
-  uint64_t kv_full;
+  uint64_t k_full[2];
+  uint64_t k_free[2];
+  uint64_t v_full;
+  uint64_t v_free;
   uint64_t q_full[2];
   uint64_t q_empty[2];
   uint64_t do_full;
@@ -152,8 +166,10 @@ struct BwdBarriers {
   uint64_t dq_full;
   uint64_t dq_empty;
   uint64_t ds_free;
-  uint64_t dkv_done;
-  uint64_t watch;  // trace builds only
+  uint64_t dkv_done;      // the item's last dK / dV products are complete
+  uint64_t dkv_free;      // the epilogue has read the item's dK / dV from TMEM
+  uint64_t item_full[4];  // the scheduler published work item `it` in slot it % 4
+  int item_idx[4];        // its index in the grouped order, or -1 after the last
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -178,32 +194,48 @@ __global__ void __launch_bounds__(512, 1)
   using Tr = BwdTraits<T, D>;
   constexpr int BM = Tr::BM;
   constexpr int CWC = Tr::CWC;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  // The layout uses all but a few hundred bytes of shared memory, with no
+  // slack to align the base: it must already start on a 1024-byte boundary
+  // (the 128-byte swizzle atoms and the MMA descriptors assume it).
+  if ((smem_u32(smem_raw) & 1023u) != 0) {
+    if (threadIdx.x == 0) atomicOr(&g_fa_error, kErrLayout);
+    return;
+  }
+  uint8_t* smem = smem_raw;
   BwdBarriers* bars = reinterpret_cast<BwdBarriers*>(smem + Tr::OFF_BAR);
   volatile int* abort_flag = &bars->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  int bh, kb;  // causal: the first key blocks are seen by the most query tiles
-  grouped_order(blockIdx.x, p.B * p.H, p.n_kblocks, p.head_group, bh, kb);
-  const int key0 = kb * Tr::BN;
   const int off = p.Nk - p.Nq;
-  int i0, n_q;
-  q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
+  const int n_items = p.n_kblocks * p.B * p.H;
+
+  // Work item j: (K/V block kb, head bh) in the grouped order (causal: the
+  // first key blocks are seen by the most query tiles) and its query-tile
+  // range [i0, i0 + n_q).
+  auto item = [&](int j, int& bh, int& kb, int& i0, int& n_q) {
+    grouped_order(j, p.B * p.H, p.n_kblocks, p.head_group, bh, kb);
+    q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
+  };
+  // The it-th work item of this CTA, as the scheduler published it in the
+  // item ring; false after the last one (or on abort).
+  auto take_item = [&](int it, int& j) -> bool {
+    if (!MBAR_WAIT(&bars->item_full[it & 3], (it >> 2) & 1, abort_flag)) return false;
+    j = *reinterpret_cast<volatile int*>(&bars->item_idx[it & 3]);
+    return j >= 0;
+  };
 #ifdef FA_TRACE
-#ifndef FA_TRACE_CTA
-#define FA_TRACE_CTA 0
-#endif
-  const bool trace_on = blockIdx.x == FA_TRACE_CTA;
+  const bool trace_cta = blockIdx.x == 0;
 #endif
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars->kv_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->q_full[s], 1);
-      mbar_init(&bars->q_empty[s], 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars->k_full[b], 1);
+      mbar_init(&bars->k_free[b], 1);
+      mbar_init(&bars->q_full[b], 1);
+      mbar_init(&bars->q_empty[b], 1);
     }
+    mbar_init(&bars->v_full, 1);
+    mbar_init(&bars->v_free, 1);
     mbar_init(&bars->do_full, 1);
     mbar_init(&bars->do_empty, 1);
     mbar_init(&bars->s_full, 1);
@@ -214,7 +246,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dkv_done, 1);
-    mbar_init(&bars->watch, 1);
+    mbar_init(&bars->dkv_free, 128);
+    for (int k = 0; k < 4; ++k) mbar_init(&bars->item_full[k], 1);
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -227,16 +260,22 @@ __global__ void __launch_bounds__(512, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
+    tma_prefetch_desc(&tmdK);
+    tma_prefetch_desc(&tmdV);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
 #ifdef FA_TRACE
-  btrace(trace_on && threadIdx.x == 0, 15000);  // set-up done
+  btrace(trace_cta && threadIdx.x == 0, 15000);  // set-up done
+  if (threadIdx.x == 0 && blockIdx.x < 1024) {
+    g_cta_times[0][blockIdx.x] = (long long)globaltimer_ns();
+    g_cta_times[1][blockIdx.x] = clock64();
+  }
 #endif
 
-  uint8_t* sK = smem + Tr::OFF_K;
+  uint8_t* sK0 = smem + Tr::OFF_K;  // two K buffers, KV_TILE apart
   uint8_t* sV = smem + Tr::OFF_V;
   uint8_t* sQ = smem + Tr::OFF_Q;
   uint8_t* sdO = smem + Tr::OFF_DO;
@@ -245,72 +284,118 @@ __global__ void __launch_bounds__(512, 1)
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
 
   // Register split (the CTA launches with 128 per thread): the compute and
-  // dQ warpgroups hold a step's TMEM columns in registers, the MMA / TMA
-  // warpgroup (warps 12-15) needs few.  Each role sets its own count.
+  // dQ warpgroups hold a step's TMEM columns in registers, warps 12-15
+  // (MMA issue, loads, scheduling) need few.  Each role sets its own count.
   if (warp >= 14) {
     regs_dec<Tr::REGS_OTHER>();
+    if (warp == 14 && lane == 0) {
+      // ---------------------------------------------------- scheduler + K/V loads
+      // Work items are handed out dynamically in the grouped order: the first
+      // wave by CTA index, the rest from a global counter, each taken when
+      // the previous item has issued its last dPᵀ (about one step before it
+      // ends), so no CTA holds a claim on work it cannot start soon.  The
+      // item's K goes to buffer it % 2 (the previous item still reads the
+      // other), its V to the one V buffer, which that last dPᵀ released.
+      bool ok = true;
+      int it = 0;
+      for (;; ++it) {
+        int j = blockIdx.x;
+        if (it >= 1) {
+          ok = ok && MBAR_WAIT(&bars->v_free, (it - 1) & 1, abort_flag);
+          j = int(gridDim.x) + atomicAdd(p.item_ctr, 1);
+        }
+        const bool last = !ok || j >= n_items;
+        bars->item_idx[it & 3] = last ? -1 : j;
+        mbar_arrive(&bars->item_full[it & 3]);  // release: the index is visible to the waiters
+        if (last) break;
+        int bh, kb, i0, n_q;
+        item(j, bh, kb, i0, n_q);
+        const int key0 = kb * Tr::BN, b = it & 1;
+        if (it >= 2 && !MBAR_WAIT(&bars->k_free[b], ((it >> 1) - 1) & 1, abort_flag)) {
+          ok = false;
+          continue;
+        }
 #ifdef FA_TRACE
-    if (warp == 14 && lane == 0 && trace_on) {
-      for (int g = 0; g < n_q; ++g) {
-        if (!MBAR_WAIT(&bars->watch, g & 1, abort_flag)) break;
-        btrace(true, 10000 + g);  // all MMAs of step g complete
-      }
-    }
+        btrace(trace_cta && it < 200, 19600 + it);  // item: K load issued
 #endif
+        mbar_arrive_expect_tx(&bars->k_full[b], Tr::KV_TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sK0 + b * Tr::KV_TILE + c * Tr::KV_CHUNK, &tmK, &bars->k_full[b], c * 64, key0, bh);
+#ifdef FA_TRACE
+        btrace(trace_cta && it < 200, 19400 + it);  // item: V load issued
+#endif
+        mbar_arrive_expect_tx(&bars->v_full, Tr::KV_TILE);
+#pragma unroll
+        for (int c = 0; c < D / 64; ++c)
+          tma_load_3d(sV + c * Tr::KV_CHUNK, &tmV, &bars->v_full, c * 64, key0, bh);
+      }
+      // Drain every issued load before the CTA may exit (it items loaded).
+      for (int k = max(0, it - 2); k < it; ++k)
+        MBAR_WAIT(&bars->k_full[k & 1], (k >> 1) & 1, abort_flag);
+      if (it > 0) MBAR_WAIT(&bars->v_full, (it - 1) & 1, abort_flag);
+    }
   } else if (warp == 13) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ Q / dO producer
     regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
-      mbar_arrive_expect_tx(&bars->kv_full, 2 * Tr::KV_TILE);
+      bool ok = true;
+      int g = 0, it = 0;
+      for (int j; ok && take_item(it, j); ++it) {
+        int bh, kb, i0, n_q;
+        item(j, bh, kb, i0, n_q);
+        for (int i = 0; i < n_q && ok; ++i) {
+          const int gs = g + i, s = gs & 1;
+          const int q0 = (i0 + i) * BM;
+          // Q (with −L·log2e and −D) into stage s, once step gs-2 has released it
+          if (gs >= 2 && !MBAR_WAIT(&bars->q_empty[s], ((gs >> 1) - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          uint64_t* bar = &bars->q_full[s];
+          mbar_arrive_expect_tx(bar, Tr::Q_TILE + 2 * BM * 4);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        tma_load_3d(sK + c * Tr::KV_CHUNK, &tmK, &bars->kv_full, c * 64, key0, bh);
-        tma_load_3d(sV + c * Tr::KV_CHUNK, &tmV, &bars->kv_full, c * 64, key0, bh);
-      }
-      for (int i = 0; i < n_q; ++i) {
-        const int s = i & 1;
-        const int q0 = (i0 + i) * BM;
-        // Q (with L and D) into stage s, once step i-2 has released it
-        if (i >= 2 && !MBAR_WAIT(&bars->q_empty[s], ((i >> 1) - 1) & 1, abort_flag)) break;
-        uint64_t* bar = &bars->q_full[s];
-        mbar_arrive_expect_tx(bar, Tr::Q_TILE + 2 * BM * 4);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
+          const size_t row = size_t(bh) * p.Nq_pad + q0;
+          bulk_load(sLD + (s * 2 + 0) * BM, p.neg_Lsc + row, BM * 4, bar);
+          bulk_load(sLD + (s * 2 + 1) * BM, p.neg_D + row, BM * 4, bar);
+          // dO into its single buffer, once step gs-1's dV product has read it
+          if (gs >= 1 && !MBAR_WAIT(&bars->do_empty, (gs - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&bars->do_full, Tr::Q_TILE);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
-        const size_t row = size_t(bh) * p.Nq_pad + q0;
-        bulk_load(sLD + (s * 2 + 0) * BM, p.neg_Lsc + row, BM * 4, bar);
-        bulk_load(sLD + (s * 2 + 1) * BM, p.neg_D + row, BM * 4, bar);
-        // dO into its single buffer, once step i-1's dV product has read it
-        if (i >= 1 && !MBAR_WAIT(&bars->do_empty, (i - 1) & 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars->do_full, Tr::Q_TILE);
-#pragma unroll
-        for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sdO + c * Tr::Q_CHUNK, &tmdO, &bars->do_full, c * 64, q0, bh);
+          for (int c = 0; c < D / 64; ++c)
+            tma_load_3d(sdO + c * Tr::Q_CHUNK, &tmdO, &bars->do_full, c * 64, q0, bh);
+        }
+        g += n_q;
       }
       // Drain every issued load before the CTA may exit.
-      for (int i = max(0, n_q - 2); i < n_q; ++i)
-        MBAR_WAIT(&bars->q_full[i & 1], (i >> 1) & 1, abort_flag);
-      if (n_q > 0) MBAR_WAIT(&bars->do_full, (n_q - 1) & 1, abort_flag);
-      MBAR_WAIT(&bars->kv_full, 0, abort_flag);
+      for (int gs = max(0, g - 2); gs < g; ++gs)
+        MBAR_WAIT(&bars->q_full[gs & 1], (gs >> 1) & 1, abort_flag);
+      if (g > 0) MBAR_WAIT(&bars->do_full, (g - 1) & 1, abort_flag);
     }
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<Tr::REGS_OTHER>();
     if (lane == 0) {
-      const uint32_t aK = smem_u32(sK), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
+      const uint32_t aK0 = smem_u32(sK0), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
       const uint32_t colS = tmem + Tr::COL_S, colDP = tmem + Tr::COL_DP;
       const uint32_t colDV = tmem + Tr::COL_DV, colDK = tmem + Tr::COL_DK;
       // Operand descriptors are built once; inside the unrolled loops each
       // MMA only adds a compile-time offset (16-byte units).
-      const uint64_t dK_k = sw128_desc(aK, 16, 1024), dV_k = sw128_desc(aV, 16, 1024);
-      const uint64_t dK_mn = sw128_desc(aK, Tr::KV_CHUNK, 1024);
+      const uint64_t dK_k0 = sw128_desc(aK0, 16, 1024), dV_k = sw128_desc(aV, 16, 1024);
+      const uint64_t dK_mn0 = sw128_desc(aK0, Tr::KV_CHUNK, 1024);
       const uint64_t dQ_k0 = sw128_desc(aQ, 16, 1024), dO_k = sw128_desc(adO, 16, 1024);
       const uint64_t dQ_mn0 = sw128_desc(aQ, Tr::Q_CHUNK, 1024);
       const uint64_t dO_mn = sw128_desc(adO, Tr::Q_CHUNK, 1024);
       const uint64_t dS_mn = sw128_desc(adS, Tr::BN * 128, 1024);
       const uint64_t dS_k = sw128_desc(adS, 16, 1024);
       auto stg = [](uint64_t d0, int s) { return d0 + uint64_t(s) * uint64_t(Tr::Q_TILE >> 4); };
+      auto kbuf = [](uint64_t d0, int b) { return d0 + uint64_t(b) * uint64_t(Tr::KV_TILE >> 4); };
 
       // Sᵀ (or dPᵀ) = X[128 keys × D] · Y[BM × D]ᵀ, both K-major.
       auto mma_st = [&](uint32_t dcol, uint64_t dx, uint64_t dy) {
@@ -321,16 +406,16 @@ __global__ void __launch_bounds__(512, 1)
           mma_ss<false>(dcol, dx + oa, dy + ob, Tr::IDESC_ST, ks > 0);
         }
       };
-      // dV or dK [128 × D] += A[128 × BM] (TMEM) · Y[BM × D] (MN-major).
-      // A (Pᵀ or dSᵀ, bf16 pairs) was written by the two compute
-      // warpgroups, each into the first half of the columns it had read, so
-      // k-step ks sits at column (ks / kPerWg)·CWC + (ks % kPerWg)·8.
-      auto mma_grad = [&](uint32_t dcol, uint32_t acol, uint64_t dy, bool acc) {
+      // dV [128 × D] += Pᵀ[128 × BM] (TMEM) · dO[BM × D] (MN-major).  Pᵀ
+      // (pairs of the input type) was written by the two compute warpgroups,
+      // each into the first half of the columns it had read, so k-step ks
+      // sits at column (ks / kPerWg)·CWC + (ks % kPerWg)·8.
+      auto mma_dv = [&](bool acc) {
         constexpr int kPerWg = CWC / 16;
 #pragma unroll
         for (int ks = 0; ks < BM / 16; ++ks)
-          mma_ts<false>(dcol, acol + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
-                        dy + uint64_t(ks * 128), Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
+          mma_ts<false>(colDV, colS + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
+                        dO_mn + uint64_t(ks * 128), Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
       };
       // dK [128 × D] += dSᵀ [128 keys × BM] (shared memory, K-major: key rows of
       // BM query values in 64-column blocks) · Q [BM × D] (MN-major).
@@ -344,77 +429,119 @@ __global__ void __launch_bounds__(512, 1)
       };
       // dQᵀ [D × BM] = Kᵀ · dSᵀ  (d = 128), or dQ [BM × D] = dS · K (d = 64);
       // both operands MN-major, K dimension = the 128 keys.
-      auto mma_dq = [&](uint32_t dcol) {
+      auto mma_dq = [&](uint64_t dkmn) {
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / 16; ++ks) {
           const uint64_t o = uint64_t(ks * 128);
           if constexpr (Tr::DQ_T)
-            mma_ss<false>(dcol, dK_mn + o, dS_mn + o, Tr::IDESC_DQ, ks > 0);
+            mma_ss<false>(colDP, dkmn + o, dS_mn + o, Tr::IDESC_DQ, ks > 0);
           else
-            mma_ss<false>(dcol, dS_mn + o, dK_mn + o, Tr::IDESC_DQ, ks > 0);
+            mma_ss<false>(colDP, dS_mn + o, dkmn + o, Tr::IDESC_DQ, ks > 0);
         }
       };
 
-      bool ok = MBAR_WAIT(&bars->kv_full, 0, abort_flag);
-      if (ok && n_q > 0)
-        ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && MBAR_WAIT(&bars->do_full, 0, abort_flag);
-      tc_fence_after();
-      BTRACE(15001);  // K, V, Q0, dO0 landed
-      if (ok && n_q > 0) {
-        mma_st(colS, dK_k, dQ_k0);
-        tc_commit(&bars->s_full);
-        mma_st(colDP, dV_k, dO_k);
-        tc_commit(&bars->dp_full);
-      }
-      // Per step i: dV (needs Pᵀ_i), then the next Sᵀ into the same columns
-      // (in issue order after dV read them), dK (needs dSᵀ_i), dQ into the
-      // dPᵀ columns (after dK read dSᵀ_i), and last the next dPᵀ, once the
-      // dQ warpgroup has drained dQ_i from those columns.
-      for (int i = 0; i < n_q && ok; ++i) {
-        const int s = i & 1;
-        const bool more = i + 1 < n_q;
-        ok = MBAR_WAIT(&bars->p_ready, i & 1, abort_flag);
-        tc_fence_after();
-        if (!ok) break;
-        BTRACE(2000 + i);
-        mma_grad(colDV, colS, dO_mn, i > 0);
-        tc_commit(&bars->do_empty);
-        BTRACE(3000 + i);
-        if (more) {
-          ok = MBAR_WAIT(&bars->q_full[s ^ 1], ((i + 1) >> 1) & 1, abort_flag);
-          tc_fence_after();
-          if (!ok) break;
-          mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
-          tc_commit(&bars->s_full);
-        }
-        BTRACE(1000 + i);
-        ok = MBAR_WAIT(&bars->ds_ready, i & 1, abort_flag);
-        tc_fence_after();
-        if (!ok) break;
-        BTRACE(4000 + i);
-        // dQ first (into the dPᵀ columns, which the compute warpgroups have
-        // read), so warpgroup 2 drains it while the tensor core runs dK.
-        mma_dq(colDP);
-        tc_commit(&bars->dq_full);
-        mma_dk(stg(dQ_mn0, s), i > 0);
-        tc_commit(&bars->q_empty[s]);
-        tc_commit(&bars->ds_free);
-        if (!more) tc_commit(&bars->dkv_done);
-        BTRACE(5000 + i);
+      bool ok = true;
+      int g = 0, it = 0;
+      for (int j; ok && take_item(it, j); ++it) {
+        int bh, kb, i0, n_q;
+        item(j, bh, kb, i0, n_q);
+        (void)bh;
+        (void)i0;
 #ifdef FA_TRACE
-        if (trace_on) tc_commit(&bars->watch);
+        const bool trace_on = trace_cta && it == 0;
 #endif
-        if (more) {
-          ok = MBAR_WAIT(&bars->dq_empty, i & 1, abort_flag) &&
-               MBAR_WAIT(&bars->do_full, (i + 1) & 1, abort_flag);
+        const int b = it & 1;
+        const uint64_t dK_k = kbuf(dK_k0, b), dK_mn = kbuf(dK_mn0, b);
+        ok = MBAR_WAIT(&bars->k_full[b], (it >> 1) & 1, abort_flag);
+        if (ok && n_q > 0)
+          ok = MBAR_WAIT(&bars->q_full[g & 1], (g >> 1) & 1, abort_flag) &&
+               MBAR_WAIT(&bars->do_full, g & 1, abort_flag);
+        tc_fence_after();
+        if (!ok) break;
+        BTRACE(15001);
+#ifdef FA_TRACE
+        btrace(trace_cta && it < 200, 19000 + it);  // item: K, Q0, dO0 landed
+#endif
+        if (n_q > 0) {
+          mma_st(colS, dK_k, stg(dQ_k0, g & 1));
+          tc_commit(&bars->s_full);
+          // dPᵀ(0) needs V, and the previous item's last dQ out of the dPᵀ columns
+          ok = MBAR_WAIT(&bars->v_full, it & 1, abort_flag);
+          if (ok && g > 0) ok = MBAR_WAIT(&bars->dq_empty, (g - 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
           mma_st(colDP, dV_k, dO_k);
           tc_commit(&bars->dp_full);
-          BTRACE(6000 + i);
+          if (n_q == 1) tc_commit(&bars->v_free);  // the item's last dPᵀ
+        } else {
+          ok = MBAR_WAIT(&bars->v_full, it & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          tc_commit(&bars->v_free);
         }
+        // dV and dK restart from zero: the previous item's epilogue must
+        // have read them.
+        if (it > 0) {
+          ok = MBAR_WAIT(&bars->dkv_free, (it - 1) & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+        }
+        // Per step: dV (needs Pᵀ), the next Sᵀ into the same columns (in
+        // issue order after dV read them), dQ into the dPᵀ columns (read by
+        // the compute warpgroups by then), dK, and last the next dPᵀ, once
+        // warpgroup 2 has drained dQ from those columns.
+        for (int i = 0; i < n_q; ++i) {
+          const int gs = g + i, s = gs & 1;
+          const bool more = i + 1 < n_q;
+          ok = MBAR_WAIT(&bars->p_ready, gs & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          BTRACE(2000 + i);
+          mma_dv(i > 0);
+          tc_commit(&bars->do_empty);
+          BTRACE(3000 + i);
+          if (more) {
+            ok = MBAR_WAIT(&bars->q_full[s ^ 1], ((gs + 1) >> 1) & 1, abort_flag);
+            tc_fence_after();
+            if (!ok) break;
+            mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
+            tc_commit(&bars->s_full);
+          }
+          BTRACE(1000 + i);
+          ok = MBAR_WAIT(&bars->ds_ready, gs & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          BTRACE(4000 + i);
+#ifdef FA_TRACE
+          btrace(trace_cta && gs < 2000, 20000 + gs);  // got dS of global step gs
+#endif
+          // dQ first, so warpgroup 2 drains it while the tensor core runs dK.
+          mma_dq(dK_mn);
+          tc_commit(&bars->dq_full);
+          if (!more) tc_commit(&bars->k_free[b]);  // the item's last product reading K
+          mma_dk(stg(dQ_mn0, s), i > 0);
+          tc_commit(&bars->q_empty[s]);
+          tc_commit(&bars->ds_free);
+          BTRACE(5000 + i);
+          if (more) {
+            ok = MBAR_WAIT(&bars->dq_empty, gs & 1, abort_flag) &&
+                 MBAR_WAIT(&bars->do_full, (gs + 1) & 1, abort_flag);
+            tc_fence_after();
+            if (!ok) break;
+            mma_st(colDP, dV_k, dO_k);
+            tc_commit(&bars->dp_full);
+            if (i + 2 == n_q) tc_commit(&bars->v_free);  // the item's last dPᵀ
+            BTRACE(6000 + i);
+          }
+        }
+        if (!ok) break;
+        if (n_q == 0) tc_commit(&bars->k_free[b]);
+        tc_commit(&bars->dkv_done);  // after the item's last dK (or at once if it has no steps)
+#ifdef FA_TRACE
+        btrace(trace_cta && it < 200, 19200 + it);  // item: last products issued
+#endif
+        g += n_q;
       }
-      if (n_q == 0) tc_commit(&bars->dkv_done);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ P / dS (thread = key)
@@ -424,184 +551,119 @@ __global__ void __launch_bounds__(512, 1)
     const int cw = warp >> 2;
     const int quad = warp & 3;
     const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
-    const int key = key0 + kr;
-    const bool key_live = key < p.Nk;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const float sl2 = p.scale_log2;
     const float scale = p.scale;
-    const int qmin = key - off;  // first query row that sees this key
     const uint32_t tS = tmem + lane_off + Tr::COL_S;
     const uint32_t tDP = tmem + lane_off + Tr::COL_DP;
     bool ok = true;
-    for (int i = 0; i < n_q; ++i) {
-      const int s = i & 1;
-      const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
-      // −L·log2e and −D of this warpgroup's query columns (16-byte aligned)
-      const float4* sL4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 0) * BM + cw * CWC);
-      const float4* sD4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 1) * BM + cw * CWC);
-      // ---- P = exp2(S·c − L·log2e), causal / ragged masking
-      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, i & 1, abort_flag));
-      tc_fence_after();
-      if (!ok) break;
+    int g = 0, it = 0;
+    for (int j; ok && __all_sync(0xffffffffu, take_item(it, j)); ++it) {
+      int bh, kb, i0, n_q;
+      item(j, bh, kb, i0, n_q);
 #ifdef FA_TRACE
-      btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // got S
+      const bool trace_on = trace_cta && it == 0;
 #endif
-      const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
-      uint32_t Pk[CWC / 2];  // P as packed pairs of the input type
-      const uint64_t c2 = pk2(sl2, sl2);
-      // Load the warpgroup's CWC columns at once (one TMEM round trip), then
-      // 32 at a time: exponentiate, pack to pairs of the input type, store Pᵀ
-      // back to TMEM into the columns this warpgroup has read (the other
-      // warpgroup may still be reading its own half).  The packed P stays in
-      // registers for dS, so dS uses the same rounded P as the dV product.
-      uint32_t u[CWC];
-#pragma unroll
-      for (int c = 0; c < CWC; c += 32)
-        tmem_ld32(tS + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
-      tmem_ld_wait();
+      const int key0 = kb * Tr::BN;
+      const int key = key0 + kr;
+      const bool key_live = key < p.Nk;
+      const int qmin = key - off;  // first query row that sees this key
+      for (int i = 0; i < n_q; ++i) {
+        const int gs = g + i, s = gs & 1;
+        const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
+        // −L·log2e and −D of this warpgroup's query columns (16-byte aligned)
+        const float4* sL4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 0) * BM + cw * CWC);
+        const float4* sD4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 1) * BM + cw * CWC);
+        // ---- P = exp2(S·c − L·log2e), causal / ragged masking
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, gs & 1, abort_flag));
+        tc_fence_after();
+        if (!ok) break;
 #ifdef FA_TRACE
-      btrace(trace_on && lane == 0, 17000 + (cw * 4 + quad) * 20 + i);  // S in registers
+        btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // got S
+        btrace(trace_cta && warp == 0 && lane == 0 && i == 0 && it < 200, 19800 + it);  // item: first S
 #endif
+        const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
+        uint32_t Pk[CWC / 2];  // P as packed pairs of the input type
+        const uint64_t c2 = pk2(sl2, sl2);
+        // Load the warpgroup's CWC columns at once (one TMEM round trip), then
+        // 32 at a time: exponentiate, pack to pairs of the input type, store Pᵀ
+        // back to TMEM into the columns this warpgroup has read (the other
+        // warpgroup may still be reading its own half).  The packed P stays in
+        // registers for dS, so dS uses the same rounded P as the dV product.
+        uint32_t u[CWC];
 #pragma unroll
-      for (int c = 0; c < CWC; c += 32) {
+        for (int c = 0; c < CWC; c += 32)
+          tmem_ld32(tS + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
+        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 nl = sL4[(c + e) >> 2];
+        for (int c = 0; c < CWC; c += 32) {
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int q = c + e + 2 * h2;
-            const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2,
-                                        h2 ? pk2(nl.z, nl.w) : pk2(nl.x, nl.y)));
-            float p0 = ex2(x.x), p1 = ex2(x.y);
-            if (need_mask) {
-              if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
-              if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
+          for (int e = 0; e < 32; e += 4) {
+            const float4 nl = sL4[(c + e) >> 2];
+#pragma unroll
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int q = c + e + 2 * h2;
+              const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2,
+                                          h2 ? pk2(nl.z, nl.w) : pk2(nl.x, nl.y)));
+              float p0 = ex2(x.x), p1 = ex2(x.y);
+              if (need_mask) {
+                if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
+                if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;
+              }
+              Pk[q >> 1] = ElemTraits<T>::pack2(p0, p1);
             }
-            Pk[q >> 1] = ElemTraits<T>::pack2(p0, p1);
           }
+          tmem_st16(tS + cw * CWC + c / 2, Pk + (c >> 1));
         }
-        tmem_st16(tS + cw * CWC + c / 2, Pk + (c >> 1));
-      }
-      tmem_st_wait();
-      tc_fence_before();
-#ifdef FA_TRACE
-      btrace(trace_on && lane == 0, 12000 + (cw * 4 + quad) * 20 + i);  // P done
-#endif
-      mbar_arrive(&bars->p_ready);
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars->p_ready);
 
-      // ---- dS = P ∘ (dP − D) · scale, to TMEM (A operand of dK += dSᵀ Q)
-      // and to shared memory for the dQ product (row = key, BM query values
-      // contiguous, 128-byte swizzled, 64 values per column block).
-      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dp_full, i & 1, abort_flag));
-      if (ok && i >= 1)
-        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (i - 1) & 1, abort_flag));
-      tc_fence_after();
-      if (!ok) break;
-#ifdef FA_TRACE
-      btrace(trace_on && lane == 0, 11000 + (cw * 4 + quad) * 20 + i);  // dP seen, dS buffer free
-#endif
-      const uint64_t sc2 = pk2(scale, scale);
+        // ---- dS = P ∘ (dP − D) · scale, to shared memory (row = key, BM
+        // query values contiguous, 128-byte swizzled, 64 values per column
+        // block): the A operand of dK += dSᵀ Q and an operand of dQ.
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dp_full, gs & 1, abort_flag));
+        if (ok && gs >= 1)
+          ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (gs - 1) & 1, abort_flag));
+        tc_fence_after();
+        if (!ok) break;
+        const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
-      for (int c = 0; c < CWC; c += 32) {
-        // one 32-column TMEM load per chunk (measured faster here than
-        // loading all CWC columns before the arithmetic)
-        tmem_ld32(tDP + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
-        tmem_ld_wait();
-        uint32_t w[16];
+        for (int c = 0; c < CWC; c += 32) {
+          // one 32-column TMEM load per chunk (measured faster here than
+          // loading all CWC columns before the arithmetic)
+          tmem_ld32(tDP + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
+          tmem_ld_wait();
+          uint32_t w[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 4) {
-          const float4 nd = sD4[(c + e) >> 2];
+          for (int e = 0; e < 32; e += 4) {
+            const float4 nd = sD4[(c + e) >> 2];
 #pragma unroll
-          for (int h2 = 0; h2 < 2; ++h2) {
-            const int q = c + e + 2 * h2;
-            const uint64_t t = fadd2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])),
-                                     h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
-            const float2 pq = ElemTraits<T>::unpack2(Pk[q >> 1]);
-            const float2 ds = upk2(fmul2(t, fmul2(pk2(pq.x, pq.y), sc2)));
-            w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
+            for (int h2 = 0; h2 < 2; ++h2) {
+              const int q = c + e + 2 * h2;
+              const uint64_t t = fadd2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])),
+                                       h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
+              const float2 pq = ElemTraits<T>::unpack2(Pk[q >> 1]);
+              const float2 ds = upk2(fmul2(t, fmul2(pk2(pq.x, pq.y), sc2)));
+              w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
+            }
+          }
+#pragma unroll
+          for (int c16 = 0; c16 < 4; ++c16) {
+            const int col = cw * CWC + c + c16 * 8;  // first query column of this 16-byte chunk
+            const int blk = col >> 6, ch = (col >> 3) & 7;
+            *reinterpret_cast<uint4*>(sdS + blk * (Tr::BN * 128) + kr * 128 + ((ch ^ (kr & 7)) << 4)) =
+                make_uint4(w[c16 * 4], w[c16 * 4 + 1], w[c16 * 4 + 2], w[c16 * 4 + 3]);
           }
         }
-#pragma unroll
-        for (int c16 = 0; c16 < 4; ++c16) {
-          const int col = cw * CWC + c + c16 * 8;  // first query column of this 16-byte chunk
-          const int blk = col >> 6, ch = (col >> 3) & 7;
-          *reinterpret_cast<uint4*>(sdS + blk * (Tr::BN * 128) + kr * 128 + ((ch ^ (kr & 7)) << 4)) =
-              make_uint4(w[c16 * 4], w[c16 * 4 + 1], w[c16 * 4 + 2], w[c16 * 4 + 3]);
-        }
-      }
+        fence_async_smem();
+        tc_fence_before();
 #ifdef FA_TRACE
-      btrace(trace_on && lane == 0, 18000 + (cw * 4 + quad) * 20 + i);  // dS computed and issued
+        btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
 #endif
-      fence_async_smem();
-      tc_fence_before();
-#ifdef FA_TRACE
-      btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
-      btrace(trace_on && lane == 0, 13000 + (cw * 4 + quad) * 20 + i);
-#endif
-      mbar_arrive(&bars->ds_ready);
-    }
-    // ---- dK, dV of the tile: TMEM → registers (packed to the dtype) → shared
-    // memory → TMA tensor stores.  The Q stages are free by now: dV goes to
-    // stage 0 and dK to stage 1, each as D/64 blocks of BN rows × 128 bytes,
-    // 128-byte swizzled like the loads; warpgroup cw stages columns
-    // [cw·D/2, (cw+1)·D/2).  The tensor maps clip rows past Nk.
-    if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dkv_done, 0, abort_flag));
-    tc_fence_after();
-#ifdef FA_TRACE
-    btrace(trace_on && lane == 0, 14000 + (cw * 4 + quad));  // dK, dV complete in TMEM
-#endif
-    // Stage one matrix's columns of this warpgroup (zeros if the tile saw no query).
-    auto stage_out = [&](int which) {
-      const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV) + cw * (D / 2);
-      uint8_t* stage = sQ + which * Tr::Q_TILE;
-#pragma unroll
-      for (int c = 0; c < D / 2; c += 32) {
-        uint32_t v[32];
-        tmem_ld32(tcol + c, v);
-        tmem_ld_wait();
-#pragma unroll
-        for (int c8 = 0; c8 < 32; c8 += 8) {
-          const int col = cw * (D / 2) + c + c8;  // first column of this 16-byte chunk
-          const int blk = col >> 6, ch = (col >> 3) & 7;
-          uint4 x = make_uint4(0u, 0u, 0u, 0u);
-          if (n_q > 0) {
-            x.x = ElemTraits<T>::pack2(__uint_as_float(v[c8]), __uint_as_float(v[c8 + 1]));
-            x.y = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 2]), __uint_as_float(v[c8 + 3]));
-            x.z = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 4]), __uint_as_float(v[c8 + 5]));
-            x.w = ElemTraits<T>::pack2(__uint_as_float(v[c8 + 6]), __uint_as_float(v[c8 + 7]));
-          }
-          *reinterpret_cast<uint4*>(stage + blk * Tr::KV_CHUNK + kr * 128 + ((ch ^ (kr & 7)) << 4)) = x;
-        }
+        mbar_arrive(&bars->ds_ready);
       }
-      fence_async_smem();
-    };
-    if constexpr (D == 128) {
-      // Warpgroup cw owns column block cw of both matrices: it stores dV's
-      // block while it stages dK's.
-      const bool elected = kr == 0;
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
-        if (ok) stage_out(which);
-        ok = named_bar_and(2 + cw, 128, ok);
-        if (ok && elected) {
-          tma_store_3d(which ? &tmdK : &tmdV, sQ + which * Tr::Q_TILE + cw * Tr::KV_CHUNK, cw * 64,
-                       key0, bh);
-          bulk_commit();
-        }
-      }
-      if (elected) bulk_wait_read0();  // the staging must outlive TMA's reads
-    } else {
-      if (ok) {
-        stage_out(0);
-        stage_out(1);
-      }
-      // Both warpgroups share the one column block: one thread stores it.
-      if (named_bar_and(2, 256, ok) && threadIdx.x == 0) {
-        tma_store_3d(&tmdV, sQ, 0, key0, bh);
-        tma_store_3d(&tmdK, sQ + Tr::Q_TILE, 0, key0, bh);
-        bulk_commit();
-        bulk_wait_read0();
-      }
+      g += n_q;
     }
   } else {
     // ------------------------------------------------------------ dQ (warpgroup 2)
@@ -612,80 +674,132 @@ __global__ void __launch_bounds__(512, 1)
     const uint32_t tQ = tmem + lane_off + Tr::COL_DP;  // dQ of the step sits in the dPᵀ columns
     const bool leader = (warp == 8 && lane == 0);
     bool ok = true;
-    for (int i = 0; i < n_q; ++i) {
-      const int q0 = (i0 + i) * BM;
-      ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full, i & 1, abort_flag));
-      tc_fence_after();
-      if (!ok) break;
-#ifdef FA_TRACE
-      btrace(trace_on && leader, 9000 + i);  // dQ ready seen
-#endif
-      if constexpr (Tr::DQ_T) {
-        // thread = d index r, TMEM column q = query row q0 + q.  All BM
-        // columns come to registers first, so the dPᵀ columns are released
-        // after one TMEM round trip; then for each q a warp adds 32
-        // consecutive floats (one 128-byte line) of the fp32 accumulator
-        // (mode 1), or stores them into this K/V block's partial (mode 2).
-        uint32_t v[BM];
+    int g = 0, it = 0;
+    for (int j; ok && named_bar_and(1, 128, take_item(it, j)); ++it) {
+      int bh, kb, i0, n_q;
+      item(j, bh, kb, i0, n_q);
+      for (int i = 0; i < n_q; ++i) {
+        const int gs = g + i;
+        const int q0 = (i0 + i) * BM;
+        ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dq_full, gs & 1, abort_flag));
+        tc_fence_after();
+        if (!ok) break;
+        if constexpr (Tr::DQ_T) {
+          // thread = d index r, TMEM column q = query row q0 + q.  All BM
+          // columns come to registers first, so the dPᵀ columns are released
+          // after one TMEM round trip; then for each q a warp adds 32
+          // consecutive floats (one 128-byte line) of the fp32 accumulator
+          // (mode 1), or stores them into this K/V block's partial (mode 2).
+          uint32_t v[BM];
 #pragma unroll
-        for (int c = 0; c < BM; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
-        float* dst = p.dq_mode == 2
-                         ? p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D + r
-                         : p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D + r;
-        if (p.dq_mode == 2) {
-#pragma unroll
-          for (int q = 0; q < BM; ++q) dst[q * D] = __uint_as_float(v[q]);
-        } else {
-#pragma unroll
-          for (int q = 0; q < BM; ++q) red_add_f32(dst + q * D, __uint_as_float(v[q]));
-        }
-      } else {
-        uint32_t v[D];  // thread = query row r: its D values
-#pragma unroll
-        for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
-        tmem_ld_wait();
-        tc_fence_before();
-        mbar_arrive(&bars->dq_empty);  // the dP columns may take the next dPᵀ
-        // The previous bulk operation must have finished reading the staging buffer.
-        if (leader) bulk_wait_read0();
-        named_bar(1, 128);
-        // write the row's D values, rotating the 16-byte chunk order by lane
-        // to spread shared-memory banks
-#pragma unroll
-        for (int cc = 0; cc < D / 4; ++cc) {
-          const int c4 = (cc + lane) % (D / 4);
-          float4 x;
-          x.x = __uint_as_float(v[c4 * 4 + 0]);
-          x.y = __uint_as_float(v[c4 * 4 + 1]);
-          x.z = __uint_as_float(v[c4 * 4 + 2]);
-          x.w = __uint_as_float(v[c4 * 4 + 3]);
-          *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
-        }
-        fence_async_smem();
-        named_bar(1, 128);
-        if (leader) {
+          for (int c = 0; c < BM; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
+          float* dst = p.dq_mode == 2
+                           ? p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D + r
+                           : p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D + r;
           if (p.dq_mode == 2) {
-            float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
-            bulk_store(dst, sdQ, Tr::DQ_STAGE);
+#pragma unroll
+            for (int q = 0; q < BM; ++q) dst[q * D] = __uint_as_float(v[q]);
           } else {
-            float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
-            bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+#pragma unroll
+            for (int q = 0; q < BM; ++q) red_add_f32(dst + q * D, __uint_as_float(v[q]));
           }
-          bulk_commit();
+        } else {
+          uint32_t v[D];  // thread = query row r: its D values
+#pragma unroll
+          for (int c = 0; c < D; c += 32) tmem_ld32(tQ + c, *reinterpret_cast<uint32_t(*)[32]>(v + c));
+          tmem_ld_wait();
+          tc_fence_before();
+          mbar_arrive(&bars->dq_empty);  // the dP columns may take the next dPᵀ
+          // The previous bulk operation must have finished reading the staging buffer.
+          if (leader) bulk_wait_read0();
+          named_bar(1, 128);
+          // write the row's D values, rotating the 16-byte chunk order by lane
+          // to spread shared-memory banks
+#pragma unroll
+          for (int cc = 0; cc < D / 4; ++cc) {
+            const int c4 = (cc + lane) % (D / 4);
+            float4 x;
+            x.x = __uint_as_float(v[c4 * 4 + 0]);
+            x.y = __uint_as_float(v[c4 * 4 + 1]);
+            x.z = __uint_as_float(v[c4 * 4 + 2]);
+            x.w = __uint_as_float(v[c4 * 4 + 3]);
+            *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
+          }
+          fence_async_smem();
+          named_bar(1, 128);
+          if (leader) {
+            if (p.dq_mode == 2) {
+              float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
+              bulk_store(dst, sdQ, Tr::DQ_STAGE);
+            } else {
+              float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
+              bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+            }
+            bulk_commit();
+          }
         }
       }
+      if (!ok) break;
+      // ---- dK, dV of the item (thread = key row r): out of TMEM 32 columns
+      // at a time, packed to the dtype, straight to global memory.  This
+      // warpgroup is otherwise idle until the next item's first dQ, so the
+      // compute warpgroups go on to the next item's P at once; the
+      // accumulators are released after the last TMEM load.
+      ok = named_bar_and(1, 128, MBAR_WAIT(&bars->dkv_done, it & 1, abort_flag));
+      tc_fence_after();
+      if (!ok) break;
+      {
+        const int key = kb * Tr::BN + r;
+        const bool live = key < p.Nk;
+        const size_t rowoff = (size_t(bh) * p.Nk + (live ? key : 0)) * D;
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV);
+          T* out = reinterpret_cast<T*>(which ? p.dK : p.dV) + rowoff;
+#pragma unroll
+          for (int c = 0; c < D; c += 32) {
+            uint32_t v[32];
+            tmem_ld32(tcol + c, v);
+            tmem_ld_wait();
+            if (which == 1 && c + 32 == D) {
+              tc_fence_before();
+              mbar_arrive(&bars->dkv_free);
+            }
+            if (live) {
+#pragma unroll
+              for (int e = 0; e < 32; e += 8) {
+                uint4 x = make_uint4(0u, 0u, 0u, 0u);
+                if (n_q > 0) {
+                  x.x = ElemTraits<T>::pack2(__uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+                  x.y = ElemTraits<T>::pack2(__uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+                  x.z = ElemTraits<T>::pack2(__uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+                  x.w = ElemTraits<T>::pack2(__uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+                }
+                *reinterpret_cast<uint4*>(out + c + e) = x;
+              }
+            }
+          }
+        }
+      }
+      g += n_q;
     }
     if (leader) bulk_wait0();
   }
 
 #ifdef FA_TRACE
-  btrace(trace_on && lane == 0, 14100 + warp);  // warp finished
+  btrace(trace_cta && lane == 0, 14100 + warp);  // warp finished
 #endif
   tc_fence_before();
   __syncthreads();
+#ifdef FA_TRACE
+  if (threadIdx.x == 0 && blockIdx.x < 1024) {
+    g_cta_times[2][blockIdx.x] = (long long)globaltimer_ns();
+    g_cta_times[3][blockIdx.x] = clock64();
+  }
+#endif
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -703,6 +817,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
   const int bh = blockIdx.y;
   const int q = blockIdx.x * RPB + g;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.item_ctr = 0;
   if (q >= p.Nq_pad) return;
   float dsum = 0.f;
   float lsc = INFINITY;
@@ -905,8 +1020,10 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
     e = cudaEventRecord(a.ev_start, a.stream);
     if (e != cudaSuccess) return e;
   }
-  kern<<<dim3(p.n_kblocks * BH), Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(
-      a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK, a.tmdV, p);
+  // persistent: one CTA per SM (or per work item, if fewer)
+  const int grid = std::min(p.n_kblocks * BH, sm_count());
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK,
+                                                        a.tmdV, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.ev_stop) {
@@ -940,6 +1057,10 @@ FA_ERROR_ACCESSOR(take_error_bwd)
 
 #ifdef FA_TRACE
 }  // namespace fa
+extern "C" int fa_cta_times_read(long long* out) {
+  cudaMemcpyFromSymbol(out, fa::g_cta_times, sizeof(fa::g_cta_times));
+  return 4 * 1024;
+}
 extern "C" int fa_btrace_read(long long* out, int max) {
   const int n = max < 32768 ? max : 32768;
   cudaMemcpyFromSymbol(out, fa::g_btrace, sizeof(long long) * n);

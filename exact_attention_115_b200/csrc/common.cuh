@@ -46,7 +46,10 @@ static __device__ int g_fa_site = 0;
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 
 // Bits OR-ed into the error word by kernels.
-enum : int { kErrTimeout = 1 };
+enum : int {
+  kErrTimeout = 1,  // a bounded wait expired
+  kErrLayout = 2,   // a kernel found its dynamic shared memory misaligned and did nothing
+};
 
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -45,6 +45,7 @@ struct BwdParams {
   float* neg_D;    // [B*H, Nq_pad] -rowsum(dO * O), padded rows zero
   float* neg_Lsc;  // [B*H, Nq_pad] -L * log2(e), padded rows -inf
   float* dQacc;   // [B*H, Nq_pad, d] fp32 (mode 1) or [nkv, B*H, Nq_pad, d] (mode 2)
+  int* item_ctr;  // work items handed out beyond the first wave (zeroed by the preprocess)
   int B, H, Nq, Nk, Nq_pad;
   float scale;        // softmax scale
   float scale_log2;   // scale * log2(e)
@@ -62,6 +63,9 @@ struct BwdLaunch {
 };
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a);
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count();
 
 // Heads per launch-order group: as many as keep the bytes one head's CTAs
 // share (K and V in the forward; Q, dO, the fp32 dQ accumulator, L and D in
