@@ -19,8 +19,12 @@
 // buffers, dQ accumulator cleared), bwd_main (below), bwd_dq_finalise
 // (sum / convert).
 //
-// bwd_main, B200 design.  One CTA per (K/V block of 128 keys, head), issued
-// heaviest first within groups of heads.  A step handles BM = 128 query rows.
+// bwd_main, B200 design.  Persistent: one CTA per SM takes work items (a K/V
+// block of 128 keys of one head) from a global counter, heaviest first within
+// groups of heads, each when its previous item is one step from the end; K is
+// double buffered so the next item's K loads while the current item runs, V
+// is reloaded once the current item's last dPᵀ has read it.  A step handles
+// BM = 128 query rows of the item.
 // The two score-like products are computed transposed (keys on TMEM lanes):
 // Sᵀ = K Qᵀ and dPᵀ = V dOᵀ, so that the thread owning key row k holds
 // Pᵀ[k, :] and dSᵀ[k, :].  Pᵀ goes back to TMEM as the A operand of
@@ -33,11 +37,12 @@
 //            with one bulk reduce-add (cp.reduce.async.bulk .add.f32).
 // Roles (512 threads, setmaxnreg split 136 / 136 / 104 registers):
 //   warpgroups 0 and 1: thread = key row; warpgroup c computes P and dS for
-//                query columns [64c, 64c + 64) of each step, and writes half
-//                of the final dK/dV columns;
+//                query columns [64c, 64c + 64) of each step;
 //   warpgroup 2: moves dQ of the step from TMEM to the fp32 accumulator,
-//                and writes each work item's dK and dV;
-//   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: TMA producer.
+//                and writes each work item's dK and dV (so the compute
+//                warpgroups go straight on to the next item);
+//   warp 12: tcgen05.mma issuer, TMEM owner; warp 13: Q / dO producer;
+//   warp 14: work-item scheduler and K / V loads.
 // TMEM (512 columns): Sᵀ | dPᵀ | dV | dK (128, 128, d, d).  Per step the
 // MMA order is dV, next Sᵀ, dQ, dK, next dPᵀ: dQ lands in the dPᵀ columns
 // (read by then), warpgroup 2 drains it while dK runs, and the next dPᵀ
