@@ -41,6 +41,7 @@ SIGNATURES = {
     "fa_bwd_set_timing_events": (_I, [_VP, _VP]),
     "fa_last_timeout_site": (_I, []),
     "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "fa_selftest_wait_timeout": (_I, [ctypes.c_uint, _VP]),
     "fa_version": (ctypes.c_char_p, []),
 }
 
@@ -235,6 +236,13 @@ def set_bwd_timing_events(start=None, stop=None) -> None:
         lib().fa_bwd_set_timing_events(None, None)
     else:
         lib().fa_bwd_set_timing_events(start.cuda_event, stop.cuda_event)
+
+
+def selftest_wait_timeout(limit_us: int = 20000, device=None) -> int:
+    """Enqueue the failure-detection self-test (a bounded wait that runs out
+    after ``limit_us``); returns the launch status.  The next status() reads
+    FA_ERR_TIMEOUT."""
+    return int(lib().fa_selftest_wait_timeout(int(limit_us), _stream(device)))
 
 
 def version() -> str:

@@ -359,6 +359,13 @@ int fa_bwd_set_timing_events(void* start, void* stop) {
 
 int fa_last_timeout_site(void) { return g_last_site; }
 
+int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
+  if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID;
+  return launch_selftest_wait(1000ull * limit_us, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? FA_OK
+             : FA_ERR_CUDA;
+}
+
 const char* fa_version(void) { return "fa-b200 0.1 (sm_100a)"; }
 
 }  // extern "C"

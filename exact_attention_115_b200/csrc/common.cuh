@@ -132,13 +132,14 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t* bar, uint32_t pari
 // Returns false (and leaves the CTA aborted) on timeout or if the CTA was
 // already aborted by another thread.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int site = 0) {
+                                          int site = 0,
+                                          unsigned long long limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_sleep(bar, parity)) return true;
   const unsigned long long t0 = globaltimer_ns();
   for (;;) {
     if (mbar_try_wait_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicOr(&g_fa_error, kErrTimeout);
       atomicCAS(&g_fa_site, 0, site);

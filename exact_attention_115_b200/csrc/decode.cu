@@ -242,6 +242,26 @@ cudaError_t decode_scratch_ptr(void** out) {
   return cudaSuccess;
 }
 
+// Failure-detection self-test: one thread waits, through the same bounded
+// wait the kernels use, on an mbarrier that nothing ever arrives at; after
+// limit_ns it records a timeout (error word + site) and returns.
+__global__ void selftest_wait_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, FA_SITE_BASE + __LINE__, limit_ns);
+}
+
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream) {
+  selftest_wait_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
+
 FA_ERROR_ACCESSOR(take_error_decode)
 
 }  // namespace fa

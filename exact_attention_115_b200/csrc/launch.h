@@ -104,6 +104,7 @@ cudaError_t decode_scratch_ptr(void** out);
 cudaError_t take_error_fwd(int* word, int* site);
 cudaError_t take_error_bwd(int* word, int* site);
 cudaError_t take_error_decode(int* word, int* site);
+cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 
 // Sets the dynamic shared-memory limit of `kernel` on the current device once.
 cudaError_t set_smem_once(const void* kernel, int bytes);

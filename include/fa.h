@@ -134,14 +134,16 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
 int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
                       int Nk, int d, float scale, int dtype, int num_splits, void* stream);
 
-/* Synchronises `stream`, then returns and clears the device error word:/* Synchronises `stream`, then returns and clears the device error word:
+/* Synchronises `stream`, then returns and clears the device error word:
  * FA_OK, FA_ERR_TIMEOUT if a kernel's bounded wait expired, FA_ERR_CUDA if
- * the stream reports a CUDA error. */
+ * the stream reports a CUDA error or a kernel found its shared memory
+ * misaligned (it then did nothing). */
 int fa_status(void* stream);
 
 /* Diagnostic: identifies the first kernel wait that timed out among those
  * fa_status has reported (10000 + line in the forward kernel file, 20000 +
- * line in the backward file); 0 if none has.  No counterpart on the pages. */
+ * line in the backward file, 30000 + line in the decode file); 0 if none
+ * has.  No counterpart on the pages. */
 int fa_last_timeout_site(void);
 
 /* Measurement hook (no counterpart on the pages, which only say to profile
@@ -152,6 +154,16 @@ int fa_last_timeout_site(void);
  * cudaEventElapsedTime.  The events are created and owned by the caller.
  * Pass NULLs to switch it off.  Process-wide; returns FA_OK. */
 int fa_bwd_set_timing_events(void* start, void* stop);
+
+/* Failure-detection self-test (no counterpart on the pages).  Enqueues on
+ * `stream` one thread that waits, through the kernels' own bounded wait, on
+ * a barrier nothing arrives at, for `limit_us` microseconds (1..1000000),
+ * then records a timeout as any kernel wait would: the next fa_status
+ * returns FA_ERR_TIMEOUT and fa_last_timeout_site names that wait (30000 +
+ * line).  Nothing faults or traps; the context stays usable.  Returns
+ * FA_ERR_INVALID for a limit out of range, else FA_OK (FA_ERR_CUDA if the
+ * launch fails). */
+int fa_selftest_wait_timeout(unsigned int limit_us, void* stream);
 
 /* Library version string (static storage). */
 const char* fa_version(void);

@@ -134,3 +134,9 @@ def test_python_binding_refuses_cpu_tensors(lib):
         fa.forward(q, q, q)
     with pytest.raises(ValueError):
         fa.decode(q[:, :, :1], q, q)
+
+
+def test_selftest_rejects_limits_out_of_range(lib):
+    # validated before anything is enqueued, so no GPU is needed
+    assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
+    assert lib.fa_selftest_wait_timeout(1000001, None) == fa.FA_ERR_INVALID
