@@ -34,6 +34,9 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I,
                     _VP, _SZ, _VP]),
+    "fa_fwd_strided": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I,
+                            _F, _I, _VP]),
+    "fa_bwd_strided": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
     "fa_set_bwd_dq_mode": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
@@ -80,12 +83,27 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"unsupported dtype {t.dtype}")
 
 
-def _check(name, t, shape=None, dtype=None):
+class Layout(ctypes.Structure):
+    """fa_layout: element strides (batch, head, row) of a [B, H, N, d] tensor."""
+    _fields_ = [("b", ctypes.c_longlong), ("h", ctypes.c_longlong), ("n", ctypes.c_longlong)]
+
+
+def _layout(t) -> Layout:
+    s = t.stride()
+    return Layout(s[0], s[1], s[2])
+
+
+def _check(name, t, shape=None, dtype=None, strided=False):
+    """Validate a tensor argument; ``strided`` allows any strides with the
+    last (d) dimension contiguous, else the tensor must be contiguous."""
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if not t.is_cuda:
         raise ValueError(f"{name} must be on a CUDA device (no CPU path exists)")
-    if not t.is_contiguous():
+    if strided:
+        if t.dim() != 4 or t.stride(-1) != 1:
+            raise ValueError(f"{name} must be [B, H, N, d] with the d dimension contiguous")
+    elif not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
@@ -103,24 +121,35 @@ def _raise(fn, code):
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
-    """O, L = attention(q, k, v).  Returns (O [B,H,Nq,d] q.dtype, L [B,H,Nq] fp32)."""
-    _check("q", q)
+    """O, L = attention(q, k, v).  q, k, v (and out) are [B, H, N, d] with any
+    strides whose d dimension is contiguous (a [B, N, H, d] tensor viewed
+    with .transpose(1, 2) works as is).  Returns (O [B,H,Nq,d] q.dtype,
+    L [B,H,Nq] fp32 contiguous)."""
+    _check("q", q, strided=True)
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
-    _check("k", k, (B, H, Nk, d), q.dtype)
-    _check("v", v, (B, H, Nk, d), q.dtype)
+    _check("k", k, (B, H, Nk, d), q.dtype, strided=True)
+    _check("v", v, (B, H, Nk, d), q.dtype, strided=True)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if out is None:
-        out = torch.empty_like(q)
+        out = torch.empty((B, H, Nq, d), dtype=q.dtype, device=q.device)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    _check("out", out, q.shape, q.dtype)
+    _check("out", out, (B, H, Nq, d), q.dtype, strided=True)
     _check("lse", lse, (B, H, Nq), torch.float32)
-    rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                      B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                      _stream(q.device))
-    _raise("fa_fwd", rc)
+    if q.is_contiguous() and k.is_contiguous() and v.is_contiguous() and out.is_contiguous():
+        rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                          lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                          _dtype_code(q), _stream(q.device))
+        _raise("fa_fwd", rc)
+        return out, lse
+    lq, lk, lv, lo = _layout(q), _layout(k), _layout(v), _layout(out)
+    rc = lib().fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv),
+                              ctypes.byref(lo), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                              _dtype_code(q), _stream(q.device))
+    _raise("fa_fwd_strided", rc)
     return out, lse
 
 
@@ -140,29 +169,41 @@ def set_bwd_dq_mode(mode: int) -> int:
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace=None):
     """dQ, dK, dV of attention given the forward's O and L and the upstream dO."""
-    _check("q", q)
+    _check("q", q, strided=True)
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
     for name, t, n in (("k", k, Nk), ("v", v, Nk), ("o", o, Nq), ("do", do, Nq)):
-        _check(name, t, (B, H, n, d), q.dtype)
+        _check(name, t, (B, H, n, d), q.dtype, strided=True)
     _check("lse", lse, (B, H, Nq), torch.float32)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    dq = torch.empty_like(q) if dq is None else dq
-    dk = torch.empty_like(k) if dk is None else dk
-    dv = torch.empty_like(v) if dv is None else dv
-    for name, t, ref in (("dq", dq, q), ("dk", dk, k), ("dv", dv, v)):
-        _check(name, t, ref.shape, q.dtype)
+    dev = q.device
+    dq = torch.empty((B, H, Nq, d), dtype=q.dtype, device=dev) if dq is None else dq
+    dk = torch.empty((B, H, Nk, d), dtype=q.dtype, device=dev) if dk is None else dk
+    dv = torch.empty((B, H, Nk, d), dtype=q.dtype, device=dev) if dv is None else dv
+    for name, t, n in (("dq", dq, Nq), ("dk", dk, Nk), ("dv", dv, Nk)):
+        _check(name, t, (B, H, n, d), q.dtype, strided=True)
     need = bwd_workspace_bytes(B, H, Nq, Nk, d, q.dtype)
     if workspace is None:
-        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+        workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     _check("workspace", workspace)
-    rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                      lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                      B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                      workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                      _stream(q.device))
-    _raise("fa_bwd", rc)
+    ts = (q, k, v, o, do, dq, dk, dv)
+    if all(t.is_contiguous() for t in ts):
+        rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                          B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
+                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                          _stream(dev))
+        _raise("fa_bwd", rc)
+        return dq, dk, dv
+    lays = [_layout(t) for t in ts]
+    rc = lib().fa_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d,
+                              int(bool(causal)), float(scale), _dtype_code(q),
+                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                              _stream(dev))
+    _raise("fa_bwd_strided", rc)
     return dq, dk, dv
 
 

@@ -48,21 +48,47 @@ CUtensorMapDataType tma_type(int dtype) {
   }
 }
 
-// 3-D map over a contiguous [BH, N, d] tensor: x = d (innermost), y = row,
-// z = batch·head.  The box is one 128-byte swizzled column block of
-// `box_rows` rows; rows past N read as zero.
-bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int BH, int box_rows) {
+// Tensor map over a [B, H, N, d] tensor with element strides l (d
+// contiguous).  When batches are exactly H heads apart (l.b == H·l.h, as in a
+// contiguous tensor) heads and batches merge into one index: a 3-D map
+// (x = d, y = row, z = b·H + h); otherwise a 4-D map (x, y, z = h, w = b),
+// and *is4d says which.  The box is one 128-byte swizzled column block of
+// `box_rows` rows; rows past N read as zero (and stores there are dropped).
+bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int H, int B,
+              const fa_layout& l, int box_rows, bool* is4d) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const int es = elem_size(dtype);
-  cuuint64_t dims[3] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(BH)};
-  cuuint64_t strides[2] = {cuuint64_t(d) * es, cuuint64_t(N) * d * es};
-  cuuint32_t box[3] = {cuuint32_t(128 / es), cuuint32_t(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = enc(m, tma_type(dtype), 3, const_cast<void*>(ptr), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+  const bool merge = l.b == (long long)H * l.h;
+  *is4d = !merge;
+  cuuint64_t dims[4] = {cuuint64_t(d), cuuint64_t(N), cuuint64_t(merge ? B * H : H), cuuint64_t(B)};
+  cuuint64_t strides[3] = {cuuint64_t(l.n) * es, cuuint64_t(l.h) * es, cuuint64_t(l.b) * es};
+  cuuint32_t box[4] = {cuuint32_t(128 / es), cuuint32_t(box_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, tma_type(dtype), merge ? 3 : 4, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+fa_layout contiguous_layout(int H, int N, int d) {
+  return fa_layout{(long long)H * N * d, (long long)N * d, (long long)d};
+}
+
+bool is_contiguous(const fa_layout& l, int H, int N, int d) {
+  const fa_layout c = contiguous_layout(H, N, d);
+  return l.b == c.b && l.h == c.h && l.n == c.n;
+}
+
+// Strides the kernels accept: non-negative, each a multiple of 16 bytes (the
+// tensor-map rule; it also keeps every row 16-byte aligned).
+bool valid_layout(const fa_layout* l, int dtype) {
+  if (!l) return false;
+  const long long es = elem_size(dtype);
+  const long long v[3] = {l->b, l->h, l->n};
+  for (long long x : v)
+    if (x < 0 || (x * es) % 16 != 0 || x * es >= (1ll << 40)) return false;
+  return true;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -159,22 +185,35 @@ using namespace fa;
 
 extern "C" {
 
-int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
-           int Nk, int d, int causal, float scale, int dtype, void* stream) {
+int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* L,
+                   const fa_layout* lq, const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
+                   int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
+                   void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(L))
     return FA_ERR_INVALID;
+  if (!valid_layout(lq, dtype) || !valid_layout(lk, dtype) || !valid_layout(lv, dtype) ||
+      !valid_layout(lo, dtype))
+    return FA_ERR_INVALID;
   if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
+  // the fp32 path stages its tiles with plain loads of contiguous tensors
+  if (dtype == FA_FP32 && !(is_contiguous(*lq, H, Nq, d) && is_contiguous(*lk, H, Nk, d) &&
+                            is_contiguous(*lv, H, Nk, d) && is_contiguous(*lo, H, Nq, d)))
+    return FA_ERR_UNSUPPORTED;
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
   if (int64_t((Nq + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
-  if (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, 128) || !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) ||
-      !make_map(&a.tmV, V, dtype, d, Nk, BH, 128) || !make_map(&a.tmO, O, dtype, d, Nq, BH, 128))
+  bool m4[4];
+  if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
+      !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
+      !make_map(&a.tmV, V, dtype, d, Nk, H, B, *lv, 128, &m4[2]) ||
+      !make_map(&a.tmO, O, dtype, d, Nq, H, B, *lo, 128, &m4[3]))
     return FA_ERR_CUDA;
+  for (int i = 0; i < 4; ++i) a.params.map4d |= int(m4[i]) << i;
   a.params.Q = Q;
   a.params.K = K;
   a.params.V = V;
@@ -192,6 +231,13 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
   return launch_fwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
+           int Nk, int d, int causal, float scale, int dtype, void* stream) {
+  const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
+  return fa_fwd_strided(Q, K, V, O, L, &lq, &lk, &lk, &lq, B, H, Nq, Nk, d, causal, scale, dtype,
+                        stream);
+}
+
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
   if (check_common(B, H, Nq, Nk, d, 1.0f, dtype) != FA_OK) return 0;
   return bwd_layout(B, H, Nq, Nk, d, effective_dq_mode(B, H, Nq, Nk, d)).total;
@@ -204,15 +250,26 @@ int fa_set_bwd_dq_mode(int mode) {
   return prev;
 }
 
-int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-           const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
-           int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
+                   const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
+                   const fa_layout* ldo, const fa_layout* ldq, const fa_layout* ldk,
+                   const fa_layout* ldv, int B, int H, int Nq, int Nk, int d, int causal,
+                   float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return FA_ERR_INVALID;
+  const fa_layout* lays[] = {lq, lk, lv, lo, ldo, ldq, ldk, ldv};
+  for (const fa_layout* l : lays)
+    if (!valid_layout(l, dtype)) return FA_ERR_INVALID;
   if (dtype == FA_FP32 && d != 64) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_FP32) {  // the CUDA-core fp32 path reads and writes contiguous tensors
+    const int rows[] = {Nq, Nk, Nk, Nq, Nq, Nq, Nk, Nk};
+    for (int i = 0; i < 8; ++i)
+      if (!is_contiguous(*lays[i], H, rows[i], d)) return FA_ERR_UNSUPPORTED;
+  }
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
   // grids: (rows, B·H) for the per-row kernels, one CTA per (K/V block, head)
   if (int64_t(B) * H > 65535 || int64_t((Nk + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
@@ -225,10 +282,14 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   std::memset(&a, 0, sizeof(a));
   const int bm = bwd_block_rows(d);
   // (the fp32 path stages its operands without TMA)
+  bool m4[6] = {false, false, false, false, false, false};
   if (dtype != FA_FP32 &&
-      (!make_map(&a.tmQ, Q, dtype, d, Nq, BH, bm) || !make_map(&a.tmdO, dO, dtype, d, Nq, BH, bm) ||
-       !make_map(&a.tmK, K, dtype, d, Nk, BH, 128) || !make_map(&a.tmV, V, dtype, d, Nk, BH, 128) ||
-       !make_map(&a.tmdK, dK, dtype, d, Nk, BH, 128) || !make_map(&a.tmdV, dV, dtype, d, Nk, BH, 128)))
+      (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, bm, &m4[0]) ||
+       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
+       !make_map(&a.tmV, V, dtype, d, Nk, H, B, *lv, 128, &m4[2]) ||
+       !make_map(&a.tmdO, dO, dtype, d, Nq, H, B, *ldo, bm, &m4[4]) ||
+       !make_map(&a.tmdK, dK, dtype, d, Nk, H, B, *ldk, 128, &m4[3]) ||
+       !make_map(&a.tmdV, dV, dtype, d, Nk, H, B, *ldv, 128, &m4[5])))
     return FA_ERR_CUDA;
   BwdParams& p = a.params;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;
@@ -244,10 +305,25 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
   p.n_kblocks = (Nk + 127) / 128;
   p.dq_mode = mode;
   p.head_group = head_group_for(size_t(p.Nq_pad) * (size_t(d) * (2 * elem_size(dtype) + 4) + 8), BH);
+  auto to_strides = [](const fa_layout* l) { return Strides{l->b, l->h, l->n}; };
+  p.s_o = to_strides(lo);
+  p.s_do = to_strides(ldo);
+  p.s_dq = to_strides(ldq);
+  p.s_dk = to_strides(ldk);
+  p.s_dv = to_strides(ldv);
+  for (int i = 0; i < 6; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dK 3, dO 4, dV 5
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;
   return launch_bwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+           const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
+           int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+  const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
+  return fa_bwd_strided(Q, K, V, O, dO, L, dQ, dK, dV, &lq, &lk, &lk, &lq, &lq, &lq, &lk, &lk, B,
+                        H, Nq, Nk, d, causal, scale, dtype, workspace, ws_bytes, stream);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {

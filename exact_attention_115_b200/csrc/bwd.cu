@@ -190,7 +190,9 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
   n = max(0, nt - i0);
 }
 
-template <typename T, int D, bool CAUSAL>
+// GEN: some tensor has a general layout (4-D tensor maps or plain strided
+// accesses); otherwise every access uses the contiguous [B·H, N, d] form.
+template <typename T, int D, bool CAUSAL, bool GEN>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -326,14 +328,16 @@ __global__ void __launch_bounds__(512, 1)
         mbar_arrive_expect_tx(&bars->k_full[b], Tr::KV_TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sK0 + b * Tr::KV_TILE + c * Tr::KV_CHUNK, &tmK, &bars->k_full[b], c * 64, key0, bh);
+          tma_load_bh(sK0 + b * Tr::KV_TILE + c * Tr::KV_CHUNK, &tmK, GEN && ((p.map4d >> 1) & 1),
+                      &bars->k_full[b], c * 64, key0, bh, p.H);
 #ifdef FA_TRACE
         btrace(trace_cta && it < 200, 19400 + it);  // item: V load issued
 #endif
         mbar_arrive_expect_tx(&bars->v_full, Tr::KV_TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
-          tma_load_3d(sV + c * Tr::KV_CHUNK, &tmV, &bars->v_full, c * 64, key0, bh);
+          tma_load_bh(sV + c * Tr::KV_CHUNK, &tmV, GEN && ((p.map4d >> 2) & 1), &bars->v_full, c * 64, key0, bh,
+                      p.H);
       }
       // Drain every issued load before the CTA may exit (it items loaded).
       for (int k = max(0, it - 2); k < it; ++k)
@@ -361,7 +365,8 @@ __global__ void __launch_bounds__(512, 1)
           mbar_arrive_expect_tx(bar, Tr::Q_TILE + 2 * BM * 4);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, bar, c * 64, q0, bh);
+            tma_load_bh(sQ + s * Tr::Q_TILE + c * Tr::Q_CHUNK, &tmQ, GEN && (p.map4d & 1), bar, c * 64, q0, bh,
+                        p.H);
           const size_t row = size_t(bh) * p.Nq_pad + q0;
           bulk_load(sLD + (s * 2 + 0) * BM, p.neg_Lsc + row, BM * 4, bar);
           bulk_load(sLD + (s * 2 + 1) * BM, p.neg_D + row, BM * 4, bar);
@@ -373,7 +378,8 @@ __global__ void __launch_bounds__(512, 1)
           mbar_arrive_expect_tx(&bars->do_full, Tr::Q_TILE);
 #pragma unroll
           for (int c = 0; c < D / 64; ++c)
-            tma_load_3d(sdO + c * Tr::Q_CHUNK, &tmdO, &bars->do_full, c * 64, q0, bh);
+            tma_load_bh(sdO + c * Tr::Q_CHUNK, &tmdO, GEN && ((p.map4d >> 4) & 1), &bars->do_full, c * 64, q0, bh,
+                        p.H);
         }
         g += n_q;
       }
@@ -759,11 +765,12 @@ __global__ void __launch_bounds__(512, 1)
       {
         const int key = kb * Tr::BN + r;
         const bool live = key < p.Nk;
-        const size_t rowoff = (size_t(bh) * p.Nk + (live ? key : 0)) * D;
+        const int krow = live ? key : 0;
 #pragma unroll
         for (int which = 0; which < 2; ++which) {
           const uint32_t tcol = tmem + lane_off + (which ? Tr::COL_DK : Tr::COL_DV);
-          T* out = reinterpret_cast<T*>(which ? p.dK : p.dV) + rowoff;
+          T* out = reinterpret_cast<T*>(which ? p.dK : p.dV) +
+                   row_offset<GEN, D>(which ? p.s_dk : p.s_dv, bh, p.H, p.Nk, krow);
 #pragma unroll
           for (int c = 0; c < D; c += 32) {
             uint32_t v[32];
@@ -815,7 +822,7 @@ __global__ void __launch_bounds__(512, 1)
 // rows, so their P is 0), stored negated so the main kernel adds them; in
 // mode 1 the fp32 dQ accumulator is cleared.
 // A group of D/8 lanes handles one row (8 elements per lane).
-template <typename T, int D>
+template <typename T, int D, bool GEN>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;  // rows per block
@@ -827,9 +834,10 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   float dsum = 0.f;
   float lsc = INFINITY;
   if (q < p.Nq) {
-    const size_t off = (size_t(bh) * p.Nq + q) * D + sl * 8;
-    const uint4 a = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.O) + off);
-    const uint4 c = *reinterpret_cast<const uint4*>(reinterpret_cast<const T*>(p.dO) + off);
+    const T* orow = reinterpret_cast<const T*>(p.O) + row_offset<GEN, D>(p.s_o, bh, p.H, p.Nq, q);
+    const T* dorow = reinterpret_cast<const T*>(p.dO) + row_offset<GEN, D>(p.s_do, bh, p.H, p.Nq, q);
+    const uint4 a = *reinterpret_cast<const uint4*>(orow + sl * 8);
+    const uint4 c = *reinterpret_cast<const uint4*>(dorow + sl * 8);
     const uint32_t aw[4] = {a.x, a.y, a.z, a.w}, cw[4] = {c.x, c.y, c.z, c.w};
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
@@ -854,7 +862,7 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
 }
 
 // dQ = Σ (dQ accumulator or per-K/V-block partials), cast to the dtype.
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool GEN>
 __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;
@@ -887,7 +895,8 @@ __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   o.y = ElemTraits<T>::pack2(acc[2], acc[3]);
   o.z = ElemTraits<T>::pack2(acc[4], acc[5]);
   o.w = ElemTraits<T>::pack2(acc[6], acc[7]);
-  *reinterpret_cast<uint4*>(reinterpret_cast<T*>(p.dQ) + (size_t(bh) * p.Nq + q) * D + sl * 8) = o;
+  T* dqrow = reinterpret_cast<T*>(p.dQ) + row_offset<GEN, D>(p.s_dq, bh, p.H, p.Nq, q);
+  *reinterpret_cast<uint4*>(dqrow + sl * 8) = o;
 }
 
 // fp32 backward on the CUDA cores (fp32 inputs only; a parity path, not a
@@ -999,16 +1008,16 @@ static cudaError_t launch_bwd_fp32(const BwdLaunch& a) {
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool GEN>
 static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   using Tr = BwdTraits<T, D>;
   const BwdParams& p = a.params;
   constexpr int RPB = 256 / (D / 8);
   const int BH = p.B * p.H;
-  bwd_preprocess_kernel<T, D><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  bwd_preprocess_kernel<T, D, GEN><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kern = bwd_main_kernel<T, D, CAUSAL>;
+  auto kern = bwd_main_kernel<T, D, CAUSAL, GEN>;
   e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc draws on the registers the CTA was launched with: refuse
@@ -1035,15 +1044,24 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
     e = cudaEventRecord(a.ev_stop, a.stream);
     if (e != cudaSuccess) return e;
   }
-  bwd_dq_finalise_kernel<T, D, CAUSAL><<<dim3((p.Nq + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  bwd_dq_finalise_kernel<T, D, CAUSAL, GEN><<<dim3((p.Nq + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
   return cudaGetLastError();
 }
 
 int bwd_block_rows(int d) { (void)d; return 128; }
 
 cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
-#define FA_BWD_CASE(TY, DD) \
-  return causal ? launch_bwd_t<TY, DD, true>(a) : launch_bwd_t<TY, DD, false>(a);
+  const BwdParams& p = a.params;
+  const bool gen = p.map4d != 0 || !contiguous_strides(p.s_o, p.H, p.Nq, d) ||
+                   !contiguous_strides(p.s_do, p.H, p.Nq, d) ||
+                   !contiguous_strides(p.s_dq, p.H, p.Nq, d) ||
+                   !contiguous_strides(p.s_dk, p.H, p.Nk, d) ||
+                   !contiguous_strides(p.s_dv, p.H, p.Nk, d);
+#define FA_BWD_CASE(TY, DD)                                                        \
+  return causal ? (gen ? launch_bwd_t<TY, DD, true, true>(a)                       \
+                       : launch_bwd_t<TY, DD, true, false>(a))                     \
+                : (gen ? launch_bwd_t<TY, DD, false, true>(a)                      \
+                       : launch_bwd_t<TY, DD, false, false>(a));
   if (dtype == FA_BF16) {
     if (d == 64) FA_BWD_CASE(__nv_bfloat16, 64)
     if (d == 128) FA_BWD_CASE(__nv_bfloat16, 128)

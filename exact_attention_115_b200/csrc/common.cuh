@@ -193,6 +193,26 @@ __device__ __forceinline__ bool named_bar_and(int id, int count, bool pred) {
   return r != 0;
 }
 
+// 4-D tiled load of one box (x = element in the row, y = row, z = head,
+// w = batch): attention tensors with arbitrary batch / head / row strides.
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar, int x,
+                                            int y, int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, const void* src, int x, int y,
+                                             int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+
 // Tiled store of one box from shared memory (bulk-group completion: the
 // caller commits and waits on the group before reusing `src` or exiting).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y,
@@ -202,6 +222,24 @@ __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void*
           reinterpret_cast<uint64_t>(map)),
       "r"(smem_u32(src)), "r"(x), "r"(y), "r"(z)
       : "memory");
+}
+
+// A [B, H, N, d] tensor's box at (x, row, head-and-batch index bh): through a
+// 3-D map (d, N, B·H) when the layout lets heads and batches merge into one
+// index, else a 4-D map (d, N, H, B).
+__device__ __forceinline__ void tma_load_bh(void* dst, const CUtensorMap* map, bool map4d,
+                                            uint64_t* bar, int x, int y, int bh, int H) {
+  if (map4d)
+    tma_load_4d(dst, map, bar, x, y, bh % H, bh / H);
+  else
+    tma_load_3d(dst, map, bar, x, y, bh);
+}
+__device__ __forceinline__ void tma_store_bh(const CUtensorMap* map, bool map4d, const void* src,
+                                             int x, int y, int bh, int H) {
+  if (map4d)
+    tma_store_4d(map, src, x, y, bh % H, bh / H);
+  else
+    tma_store_3d(map, src, x, y, bh);
 }
 
 // ------------------------------------------------------------------ tcgen05

@@ -189,7 +189,9 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
   }
 }
 
-template <typename T, int D, bool CAUSAL>
+// GEN: some tensor map is 4-D (a layout whose heads and batches do not merge
+// into one index); otherwise every map is the 3-D (d, N, B·H) form.
+template <typename T, int D, bool CAUSAL, bool GEN>
 __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -285,7 +287,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
         mbar_arrive_expect_tx(bar, Tr::TILE);
 #pragma unroll
         for (int c = 0; c < Tr::DC; ++c)
-          tma_load_3d(dst + c * Tr::CHUNK, map, bar, c * Tr::AW, row, bh);
+          tma_load_bh(dst + c * Tr::CHUNK, map, GEN && ((p.map4d >> which) & 1), bar, c * Tr::AW, row, bh, p.H);
       }
     };
     auto load_kv = [&](int i) {  // i-th K/V tile in consumption order: K0 V0 K1 V1 ...
@@ -636,7 +638,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       if (named_bar_and(1 + t, 128, ok) && r == 0) {
 #pragma unroll
         for (int blk = 0; blk < Tr::DC; ++blk)
-          tma_store_3d(&tmO, smem + t * Tr::TILE + blk * Tr::CHUNK, blk * Tr::AW, tile_first_row, bh);
+          tma_store_bh(&tmO, GEN && ((p.map4d >> 3) & 1), smem + t * Tr::TILE + blk * Tr::CHUNK, blk * Tr::AW,
+                       tile_first_row, bh, p.H);
         bulk_commit();
         bulk_wait_read0();
       }
@@ -653,10 +656,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL>
+template <typename T, int D, bool CAUSAL, bool GEN>
 static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   using Tr = FwdTraits<T, D>;
-  auto kern = fwd_kernel<T, D, CAUSAL>;
+  auto kern = fwd_kernel<T, D, CAUSAL, GEN>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg redistributes the registers the CTA was launched with; refuse
@@ -679,16 +682,18 @@ int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
 int fwd_rows_per_cta(int dtype, int d) { return 128 * fwd_tiles(dtype == FA_FP32, d); }
 
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
-#define FA_FWD_CASE(TY, DD)                                                      \
-  return causal ? launch_fwd_t<TY, DD, true>(a) : launch_fwd_t<TY, DD, false>(a);
+  const bool gen = a.params.map4d != 0;  // only 4-D tensor maps differ: every access is TMA
+#define FA_FWD_CASE(TY, DD)                                                                       \
+  return causal ? (gen ? launch_fwd_t<TY, DD, true, true>(a) : launch_fwd_t<TY, DD, true, false>(a)) \
+                : (gen ? launch_fwd_t<TY, DD, false, true>(a) : launch_fwd_t<TY, DD, false, false>(a));
   if (dtype == FA_BF16) {
     if (d == 64) FA_FWD_CASE(__nv_bfloat16, 64)
     if (d == 128) FA_FWD_CASE(__nv_bfloat16, 128)
   } else if (dtype == FA_FP16) {
     if (d == 64) FA_FWD_CASE(__half, 64)
     if (d == 128) FA_FWD_CASE(__half, 128)
-  } else if (dtype == FA_FP32) {
-    if (d == 64) FA_FWD_CASE(float, 64)
+  } else if (dtype == FA_FP32) {  // contiguous only (the host rejects other layouts)
+    if (d == 64) return causal ? launch_fwd_t<float, 64, true, false>(a) : launch_fwd_t<float, 64, false, false>(a);
   }
 #undef FA_FWD_CASE
   return cudaErrorInvalidValue;

@@ -7,6 +7,25 @@
 
 namespace fa {
 
+// Element strides of one [B, H, N, d] attention tensor (d contiguous).
+struct Strides {
+  long long b, h, n;
+};
+
+inline bool contiguous_strides(const Strides& s, int H, int N, int d) {
+  return s.n == d && s.h == (long long)N * d && s.b == (long long)H * N * d;
+}
+
+// Element offset of row n of head bh = b·H + h: the general strided form, or
+// the contiguous [B·H, N, D] one when GEN is false.
+template <bool GEN, int D>
+__host__ __device__ __forceinline__ long long row_offset(const Strides& s, int bh, int H, int N, int n) {
+  if constexpr (GEN)
+    return (bh / H) * s.b + (bh % H) * s.h + n * s.n;
+  else
+    return ((long long)bh * N + n) * D;
+}
+
 struct FwdParams {
   const void* Q;  // raw inputs (read directly only by the fp32 path)
   const void* K;
@@ -17,6 +36,7 @@ struct FwdParams {
   float scale_log2;  // scale * log2(e)
   int n_qblocks;     // ceil(Nq / fwd_rows_per_cta): one CTA per block of query rows
   int head_group;    // heads per launch-order group (see head_group_for)
+  int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
 };
 
 struct FwdLaunch {
@@ -52,6 +72,8 @@ struct BwdParams {
   int n_kblocks;      // ceil(Nk / 128)
   int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials
   int head_group;     // heads per launch-order group (see head_group_for)
+  Strides s_o, s_do, s_dq, s_dk, s_dv;  // plain (non-TMA) accesses; Q, K, V, dO go through tensor maps
+  int map4d;  // bit per tensor map (Q 0, K 1, V 2, dK 3, dO 4, dV 5): 4-D (d, N, H, B), else 3-D (d, N, B·H)
 };
 
 struct BwdLaunch {

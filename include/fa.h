@@ -68,6 +68,26 @@ typedef enum {
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
            int Nk, int d, int causal, float scale, int dtype, void* stream);
 
+/* Element strides of one attention tensor viewed as [B, H, N, d], the d
+ * elements of a row contiguous: b between batches, h between heads, n between
+ * rows.  A contiguous [B, H, N, d] tensor has {H·N·d, N·d, d}; a [B, N, H, d]
+ * tensor (sequence before head) has {N·H·d, d, H·d}.  Each stride times the
+ * element size must be a non-negative multiple of 16 bytes.  The 51CTO notes,
+ * section "Sequence Parallel": the backward kernel shown there takes a batch,
+ * head, row and column stride for every tensor it touches. */
+typedef struct {
+  long long b, h, n;
+} fa_layout;
+
+/* fa_fwd for tensors with arbitrary strides (one fa_layout each for Q, K, V
+ * and O; L stays contiguous [B, H, Nq]).  fa_fwd is this call with contiguous
+ * layouts.  Layout errors: FA_ERR_INVALID; a non-contiguous fp32 tensor:
+ * FA_ERR_UNSUPPORTED (the fp32 path reads contiguous tensors). */
+int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* L,
+                   const fa_layout* lq, const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
+                   int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
+                   void* stream);
+
 /* Bytes of device workspace fa_bwd needs for this problem (0 on invalid
  * arguments).  The workspace holds D = rowsum(dO ∘ O) [B,H,Nq] and the fp32
  * dQ accumulator; its contents on entry do not matter. */
@@ -81,6 +101,16 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype);
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
            const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* fa_bwd for tensors with arbitrary strides (layouts of Q, K, V, O, dO, dQ,
+ * dK, dV in that order; L stays contiguous).  fa_bwd is this call with
+ * contiguous layouts.  Errors as for fa_fwd_strided and fa_bwd. */
+int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
+                   const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
+                   const fa_layout* ldo, const fa_layout* ldq, const fa_layout* ldk,
+                   const fa_layout* ldv, int B, int H, int Nq, int Nk, int d, int causal,
+                   float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* How fa_bwd reduces the dQ contributions of the different K/V blocks:
  *   0 = automatic (the measured faster strategy for the shape),

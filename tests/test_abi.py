@@ -140,3 +140,22 @@ def test_selftest_rejects_limits_out_of_range(lib):
     # validated before anything is enqueued, so no GPU is needed
     assert lib.fa_selftest_wait_timeout(0, None) == fa.FA_ERR_INVALID
     assert lib.fa_selftest_wait_timeout(1000001, None) == fa.FA_ERR_INVALID
+
+
+def test_strided_entry_points_validate_layouts(lib):
+    L = fa.Layout
+    good, bad = L(2 * 64 * 64, 64 * 64, 64), L(2 * 64 * 64, 64 * 64, 3)  # 3 elements: not 16-byte aligned
+    P = 4096  # any 16-byte-aligned non-null address: the call returns before touching memory
+    args = (1, 2, 64, 64, 64, 0, 0.125)
+    r = ctypes.byref
+    assert lib.fa_fwd_strided(P, P, P, P, P, r(bad), r(good), r(good), r(good), *args, fa.FA_BF16,
+                              None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_strided(P, P, P, P, P, None, r(good), r(good), r(good), *args, fa.FA_BF16,
+                              None) == fa.FA_ERR_INVALID
+    # fp32 reads contiguous tensors only
+    nc = L(2 * 64 * 64, 64, 2 * 64)
+    assert lib.fa_fwd_strided(P, P, P, P, P, r(nc), r(good), r(good), r(good), *args, fa.FA_FP32,
+                              None) == fa.FA_ERR_UNSUPPORTED
+    lays = [r(good)] * 8
+    assert lib.fa_bwd_strided(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, P,
+                              1 << 30, None) == fa.FA_ERR_INVALID
