@@ -3,6 +3,7 @@
 Only the tests, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
 legs may import this package.  It shares no code with the CUDA library.
 """
+from . import philox  # noqa: F401
 from .attention import (  # noqa: F401
     attention_backward,
     attention_decode,

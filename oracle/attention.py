@@ -16,6 +16,14 @@ primitive:
   dS = P ∘ dP, dQ = dS K, dK = dSᵀ Q.  The page omits transposes, the scale
   and the −D term of the softmax Jacobian; this file writes the exact gradient
   of O = softmax(scale·Q Kᵀ) V (D = rowsum(dO ∘ O)).
+* Same notes, section "算法的改进": the note under the V1/V2 forward and
+  backward figures says the V1 algorithm also carries mask and dropout steps.
+  The figures did not survive, so where dropout acts is a reading: on the
+  normalised weights P, so the product uses P ∘ Z · s instead of P, where Z is
+  a 0/1 keep mask and s = 1 / (keep probability); L stays the logsumexp of
+  the undropped scores.  The backward is the exact gradient for that fixed Z:
+  dP = (dO Vᵀ) ∘ Z · s and D = rowsum(dO ∘ O) with the dropped O.  The mask
+  is an input here (``keep_fn``); ``oracle/philox.py`` draws it.
 * Same notes, section "Sequence Parallel" (last paragraph, Flash-Decoding):
   split K/V along the sequence, compute each part's softmax, then a reduction
   rescales and adds the parts.  ``decode_split_combine`` restates that.
@@ -122,8 +130,13 @@ def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None):
     return p, L
 
 
-def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None):
-    """O [r, d] and L [r] for query rows of one head (see ``head_probs``)."""
+def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None, keep_fn=None,
+                 kscale: float = 1.0):
+    """O [r, d] and L [r] for query rows of one head (see ``head_probs``).
+
+    With dropout, ``keep_fn(rows, cols)`` gives the boolean keep mask at
+    absolute query rows / key columns and ``kscale`` the factor on kept
+    weights: O = (P ∘ Z · kscale) V."""
     q = _f64(q)
     k = _f64(k)
     v = _f64(v)
@@ -138,31 +151,49 @@ def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None):
     for c0 in range(0, r, _ROW_CHUNK):
         c1 = min(r, c0 + _ROW_CHUNK)
         p, l = head_probs(q[c0:c1], k, scale, causal, rows[c0:c1], nq_total)
+        if keep_fn is not None:
+            p = p * keep_fn(rows[c0:c1], np.arange(k.shape[0])) * kscale
         O[c0:c1] = p @ v
         L[c0:c1] = l
     return O, L
 
 
-def attention_forward(Q, K, V, scale: float, causal: bool = False):
-    """O [B,H,Nq,d] and L [B,H,Nq] (float64) for [B,H,N,d] inputs."""
+def _dropout_fn(dropout, bh):
+    """(keep_fn, kscale) of head index bh for dropout = (p, seed, offset)."""
+    if dropout is None:
+        return None, 1.0
+    from . import philox
+
+    p, seed, offset = dropout
+    return (lambda r, c: philox.keep_mask(bh, r, c, p, seed, offset)), philox.keep_scale(p)
+
+
+def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None):
+    """O [B,H,Nq,d] and L [B,H,Nq] (float64) for [B,H,N,d] inputs.
+    ``dropout`` = (p, seed, offset) applies the Philox keep mask of
+    ``oracle/philox.py`` to head index b·H + h."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, H, Nq, d = Q.shape
     O = np.empty((B, H, Nq, V.shape[3]))
     L = np.empty((B, H, Nq))
     for b in range(B):
         for h in range(H):
-            O[b, h], L[b, h] = head_forward(Q[b, h], K[b, h], V[b, h], scale, causal)
+            fn, ks = _dropout_fn(dropout, b * H + h)
+            O[b, h], L[b, h] = head_forward(Q[b, h], K[b, h], V[b, h], scale, causal,
+                                            keep_fn=fn, kscale=ks)
     return O, L
 
 
 # --------------------------------------------------------------------------
 # Backward: the exact gradient of O = softmax(scale Q Kᵀ [masked]) V.
 # --------------------------------------------------------------------------
-def head_backward(q, k, v, do, scale: float, causal: bool):
+def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale: float = 1.0):
     """dQ, dK, dV, D for one head (all query rows), float64.
 
     D_i = Σ_c dO_ic O_ic; dP = dO Vᵀ; dS = P ∘ (dP − D); dV = Pᵀ dO;
-    dQ = scale · dS K; dK = scale · dSᵀ Q.
+    dQ = scale · dS K; dK = scale · dSᵀ Q.  With dropout (``keep_fn``, see
+    ``head_forward``) the products that see P ∘ Z · kscale are O and dV, and
+    dP = (dO Vᵀ) ∘ Z · kscale.
     """
     q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
     nq = q.shape[0]
@@ -174,19 +205,22 @@ def head_backward(q, k, v, do, scale: float, causal: bool):
     for c0 in range(0, nq, _ROW_CHUNK):
         c1 = min(nq, c0 + _ROW_CHUNK)
         p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq)
-        o = p @ v
+        z = 1.0 if keep_fn is None else keep_fn(rows_all[c0:c1], np.arange(k.shape[0])) * kscale
+        pz = p * z
+        o = pz @ v
         Di = (do[c0:c1] * o).sum(axis=1)
-        dp = do[c0:c1] @ v.T
+        dp = (do[c0:c1] @ v.T) * z
         ds = p * (dp - Di[:, None])
-        dv += p.T @ do[c0:c1]
+        dv += pz.T @ do[c0:c1]
         dk += scale * (ds.T @ q[c0:c1])
         dq[c0:c1] = scale * (ds @ k)
         D[c0:c1] = Di
     return dq, dk, dv, D
 
 
-def attention_backward(Q, K, V, dO, scale: float, causal: bool = False):
-    """dQ, dK, dV ([B,H,N,d]) and D ([B,H,Nq]) in float64."""
+def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=None):
+    """dQ, dK, dV ([B,H,N,d]) and D ([B,H,Nq]) in float64 (``dropout`` as in
+    ``attention_forward``)."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     B, H = Q.shape[:2]
     dQ = np.empty_like(Q)
@@ -195,12 +229,14 @@ def attention_backward(Q, K, V, dO, scale: float, causal: bool = False):
     D = np.empty(Q.shape[:3])
     for b in range(B):
         for h in range(H):
+            fn, ks = _dropout_fn(dropout, b * H + h)
             dQ[b, h], dK[b, h], dV[b, h], D[b, h] = head_backward(
-                Q[b, h], K[b, h], V[b, h], dO[b, h], scale, causal)
+                Q[b, h], K[b, h], V[b, h], dO[b, h], scale, causal, keep_fn=fn, kscale=ks)
     return dQ, dK, dV, D
 
 
-def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows):
+def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows, keep_fn=None,
+                       kscale: float = 1.0):
     """The same gradient as ``head_backward`` at selected rows only.
 
     Returns (dQ[q_rows], dK[k_rows], dV[k_rows], D[q_rows]).  dK/dV of a key
@@ -217,17 +253,20 @@ def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows):
     for c0 in range(0, nq, _ROW_CHUNK):
         c1 = min(nq, c0 + _ROW_CHUNK)
         p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq)
-        o = p @ v
+        z = 1.0 if keep_fn is None else keep_fn(rows_all[c0:c1], np.arange(k.shape[0])) * kscale
+        o = (p * z) @ v
         Di = (do[c0:c1] * o).sum(axis=1)
+        zc = 1.0 if keep_fn is None else z[:, k_rows]
         pc = p[:, k_rows]
-        dpc = do[c0:c1] @ v[k_rows].T
+        dpc = (do[c0:c1] @ v[k_rows].T) * zc
         dsc = pc * (dpc - Di[:, None])
-        dv += pc.T @ do[c0:c1]
+        dv += (pc * zc).T @ do[c0:c1]
         dk += scale * (dsc.T @ q[c0:c1])
     p, _ = head_probs(q[q_rows], k, scale, causal, q_rows, nq)
-    o = p @ v
+    z = 1.0 if keep_fn is None else keep_fn(q_rows, np.arange(k.shape[0])) * kscale
+    o = (p * z) @ v
     Dq = (do[q_rows] * o).sum(axis=1)
-    dp = do[q_rows] @ v.T
+    dp = (do[q_rows] @ v.T) * z
     ds = p * (dp - Dq[:, None])
     dq = scale * (ds @ k)
     return dq, dk, dv, Dq
