@@ -34,9 +34,8 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I,
                     _VP, _SZ, _VP]),
-    "fa_fwd_strided": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I,
-                            _F, _I, _VP]),
-    "fa_bwd_strided": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _SZ, _VP]),
+    "fa_fwd_ex": (_I, [_VP] * 9 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP]),
+    "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _SZ, _VP]),
     "fa_set_bwd_dq_mode": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
@@ -88,6 +87,18 @@ class Layout(ctypes.Structure):
     _fields_ = [("b", ctypes.c_longlong), ("h", ctypes.c_longlong), ("n", ctypes.c_longlong)]
 
 
+class Dropout(ctypes.Structure):
+    """fa_dropout: drop probability, generator seed and counter offset."""
+    _fields_ = [("p", ctypes.c_float), ("seed", ctypes.c_ulonglong), ("offset", ctypes.c_uint)]
+
+
+def _dropout(p, seed, offset):
+    """A Dropout for the C call, or None when p == 0."""
+    if p == 0:
+        return None
+    return Dropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF)
+
+
 def _layout(t) -> Layout:
     s = t.stride()
     return Layout(s[0], s[1], s[2])
@@ -120,10 +131,13 @@ def _raise(fn, code):
         raise FAError(fn, code)
 
 
-def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None):
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
     """O, L = attention(q, k, v).  q, k, v (and out) are [B, H, N, d] with any
     strides whose d dimension is contiguous (a [B, N, H, d] tensor viewed
-    with .transpose(1, 2) works as is).  Returns (O [B,H,Nq,d] q.dtype,
+    with .transpose(1, 2) works as is).  ``dropout_p`` > 0 drops attention
+    weights with the keep mask that ``seed`` and ``offset`` select (pass the
+    same three to ``backward``).  Returns (O [B,H,Nq,d] q.dtype,
     L [B,H,Nq] fp32 contiguous)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
@@ -138,18 +152,19 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
     _check("out", out, (B, H, Nq, d), q.dtype, strided=True)
     _check("lse", lse, (B, H, Nq), torch.float32)
-    if q.is_contiguous() and k.is_contiguous() and v.is_contiguous() and out.is_contiguous():
+    dr = _dropout(dropout_p, seed, offset)
+    if dr is None and all(t.is_contiguous() for t in (q, k, v, out)):
         rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
                           _dtype_code(q), _stream(q.device))
         _raise("fa_fwd", rc)
         return out, lse
     lq, lk, lv, lo = _layout(q), _layout(k), _layout(v), _layout(out)
-    rc = lib().fa_fwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                              lse.data_ptr(), ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv),
-                              ctypes.byref(lo), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
-                              _dtype_code(q), _stream(q.device))
-    _raise("fa_fwd_strided", rc)
+    rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                         ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
+                         B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
+                         None if dr is None else ctypes.byref(dr), _stream(q.device))
+    _raise("fa_fwd_ex", rc)
     return out, lse
 
 
@@ -167,8 +182,10 @@ def set_bwd_dq_mode(mode: int) -> int:
 
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
-             dq=None, dk=None, dv=None, workspace=None):
-    """dQ, dK, dV of attention given the forward's O and L and the upstream dO."""
+             dq=None, dk=None, dv=None, workspace=None, dropout_p: float = 0.0, seed: int = 0,
+             offset: int = 0):
+    """dQ, dK, dV of attention given the forward's O and L and the upstream dO
+    (and the forward's ``dropout_p``, ``seed`` and ``offset``)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -188,7 +205,8 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
         workspace = torch.empty(need, dtype=torch.uint8, device=dev)
     _check("workspace", workspace)
     ts = (q, k, v, o, do, dq, dk, dv)
-    if all(t.is_contiguous() for t in ts):
+    dr = _dropout(dropout_p, seed, offset)
+    if dr is None and all(t.is_contiguous() for t in ts):
         rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
@@ -197,13 +215,13 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
         _raise("fa_bwd", rc)
         return dq, dk, dv
     lays = [_layout(t) for t in ts]
-    rc = lib().fa_bwd_strided(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                              dv.data_ptr(), *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d,
-                              int(bool(causal)), float(scale), _dtype_code(q),
-                              workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                              _stream(dev))
-    _raise("fa_bwd_strided", rc)
+    rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
+                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                         *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d, int(bool(causal)),
+                         float(scale), _dtype_code(q), None if dr is None else ctypes.byref(dr),
+                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         _stream(dev))
+    _raise("fa_bwd_ex", rc)
     return dq, dk, dv
 
 

@@ -179,16 +179,36 @@ int sm_count() {
   return n_sm[dev];
 }
 
+// Dropout parameters from the C struct: FA_OK with *out filled (t4 = 0 when
+// there is no dropout), or FA_ERR_INVALID for a probability outside [0, 1)
+// or one that keeps nothing after rounding.  The keep threshold is
+// T = round((1 − p)·256), computed in double from the float p.
+int dropout_params(const fa_dropout* dr, DropoutParams* out) {
+  std::memset(out, 0, sizeof(*out));
+  if (!dr || dr->p == 0.0f) return FA_OK;
+  const double pd = dr->p;
+  if (!(pd >= 0.0 && pd < 1.0)) return FA_ERR_INVALID;  // also rejects NaN
+  const long t = std::lrint((1.0 - pd) * 256.0);
+  if (t < 1) return FA_ERR_INVALID;
+  if (t >= 256) return FA_OK;  // rounds to keeping everything: no dropout
+  out->k0 = uint32_t(dr->seed & 0xFFFFFFFFull);
+  out->k1 = uint32_t(dr->seed >> 32);
+  out->offset = dr->offset;
+  out->t4 = uint32_t(t) * 0x01010101u;
+  out->scale = float(256.0 / double(t));
+  return FA_OK;
+}
+
 }  // namespace fa
 
 using namespace fa;
 
 extern "C" {
 
-int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* L,
-                   const fa_layout* lq, const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
-                   int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
-                   void* stream) {
+int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
+              const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
+              int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
+              void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
@@ -204,9 +224,14 @@ int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* 
     return FA_ERR_UNSUPPORTED;
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
   if (int64_t((Nq + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid
+  DropoutParams drop;
+  st = dropout_params(dropout, &drop);
+  if (st != FA_OK) return st;
+  if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
+  a.params.drop = drop;
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
@@ -234,8 +259,8 @@ int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* 
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
            int Nk, int d, int causal, float scale, int dtype, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
-  return fa_fwd_strided(Q, K, V, O, L, &lq, &lk, &lk, &lq, B, H, Nq, Nk, d, causal, scale, dtype,
-                        stream);
+  return fa_fwd_ex(Q, K, V, O, L, &lq, &lk, &lk, &lq, B, H, Nq, Nk, d, causal, scale, dtype, nullptr,
+                   stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
@@ -250,12 +275,12 @@ int fa_set_bwd_dq_mode(int mode) {
   return prev;
 }
 
-int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                   const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
-                   const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
-                   const fa_layout* ldo, const fa_layout* ldq, const fa_layout* ldk,
-                   const fa_layout* ldv, int B, int H, int Nq, int Nk, int d, int causal,
-                   float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
+int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+              const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
+              const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
+              const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
+              int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
+              void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
@@ -273,6 +298,10 @@ int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, c
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
   // grids: (rows, B·H) for the per-row kernels, one CTA per (K/V block, head)
   if (int64_t(B) * H > 65535 || int64_t((Nk + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  DropoutParams drop;
+  st = dropout_params(dropout, &drop);
+  if (st != FA_OK) return st;
+  if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int mode = effective_dq_mode(B, H, Nq, Nk, d);
   const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
@@ -312,6 +341,7 @@ int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, c
   p.s_dk = to_strides(ldk);
   p.s_dv = to_strides(ldv);
   for (int i = 0; i < 6; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dK 3, dO 4, dV 5
+  p.drop = drop;
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;
@@ -322,8 +352,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            const float* L, void* dQ, void* dK, void* dV, int B, int H, int Nq, int Nk, int d,
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
-  return fa_bwd_strided(Q, K, V, O, dO, L, dQ, dK, dV, &lq, &lk, &lk, &lq, &lq, &lq, &lk, &lk, B,
-                        H, Nq, Nk, d, causal, scale, dtype, workspace, ws_bytes, stream);
+  return fa_bwd_ex(Q, K, V, O, dO, L, dQ, dK, dV, &lq, &lk, &lk, &lq, &lq, &lq, &lk, &lk, B, H, Nq,
+                   Nk, d, causal, scale, dtype, nullptr, workspace, ws_bytes, stream);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {

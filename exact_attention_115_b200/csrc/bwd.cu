@@ -52,6 +52,7 @@
 #include <algorithm>
 
 #include "common.cuh"
+#include "dropout.cuh"
 #include "launch.h"
 
 namespace fa {
@@ -192,7 +193,8 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
 
 // GEN: some tensor has a general layout (4-D tensor maps or plain strided
 // accesses); otherwise every access uses the contiguous [B·H, N, d] form.
-template <typename T, int D, bool CAUSAL, bool GEN>
+// DROP: the forward dropped weights; the compute warps redraw its keep mask.
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -585,6 +587,14 @@ __global__ void __launch_bounds__(512, 1)
         // −L·log2e and −D of this warpgroup's query columns (16-byte aligned)
         const float4* sL4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 0) * BM + cw * CWC);
         const float4* sD4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 1) * BM + cw * CWC);
+        // Dropout: keep bytes of this key for query columns q0 .. q0 + CWC − 1
+        // (column pair q, q + 1 in keep[q / 4], bytes q % 4 and up), drawn
+        // before S arrives.
+        uint32_t keep[DROP ? CWC / 4 : 1];
+        if constexpr (DROP) {
+#pragma unroll
+          for (int g16 = 0; g16 < CWC / 16; ++g16) keep16_col(p.drop, bh, key, q0 + 16 * g16, keep + 4 * g16);
+        }
         // ---- P = exp2(S·c − L·log2e), causal / ragged masking
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, gs & 1, abort_flag));
         tc_fence_after();
@@ -624,7 +634,19 @@ __global__ void __launch_bounds__(512, 1)
               Pk[q >> 1] = ElemTraits<T>::pack2(p0, p1);
             }
           }
-          tmem_st16(tS + cw * CWC + c / 2, Pk + (c >> 1));
+          if constexpr (DROP) {
+            // the dV product sees the dropped weights (its 256/T factor is
+            // applied in the epilogue); dS below needs the undropped P
+            uint32_t pm[16];
+#pragma unroll
+            for (int w = 0; w < 16; ++w) {
+              const int pi = (c >> 1) + w;  // pair index: columns 2·pi, 2·pi + 1
+              pm[w] = Pk[pi] & keep_pair_mask(keep[pi >> 1], (2 * pi) & 3);
+            }
+            tmem_st16(tS + cw * CWC + c / 2, pm);
+          } else {
+            tmem_st16(tS + cw * CWC + c / 2, Pk + (c >> 1));
+          }
         }
         tmem_st_wait();
         tc_fence_before();
@@ -652,8 +674,18 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int q = c + e + 2 * h2;
-              const uint64_t t = fadd2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])),
-                                       h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
+              uint64_t t;
+              if constexpr (DROP) {
+                // dP ∘ Z · 256/T − D
+                const uint32_t sb = __float_as_uint(p.drop.scale);
+                const uint64_t z = pk2(__uint_as_float(keep_word_mask(keep[q >> 2], q & 3) & sb),
+                                       __uint_as_float(keep_word_mask(keep[q >> 2], (q & 3) + 1) & sb));
+                t = ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), z,
+                          h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
+              } else {
+                t = fadd2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])),
+                          h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
+              }
               const float2 pq = ElemTraits<T>::unpack2(Pk[q >> 1]);
               const float2 ds = upk2(fmul2(t, fmul2(pk2(pq.x, pq.y), sc2)));
               w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
@@ -779,6 +811,10 @@ __global__ void __launch_bounds__(512, 1)
             if (which == 1 && c + 32 == D) {
               tc_fence_before();
               mbar_arrive(&bars->dkv_free);
+            }
+            if (DROP && which == 0) {  // dV: the kept weights' 256/T factor
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * p.drop.scale);
             }
             if (live) {
 #pragma unroll
@@ -1008,7 +1044,7 @@ static cudaError_t launch_bwd_fp32(const BwdLaunch& a) {
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL, bool GEN>
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false>
 static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   using Tr = BwdTraits<T, D>;
   const BwdParams& p = a.params;
@@ -1017,7 +1053,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   bwd_preprocess_kernel<T, D, GEN><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kern = bwd_main_kernel<T, D, CAUSAL, GEN>;
+  auto kern = bwd_main_kernel<T, D, CAUSAL, GEN, DROP>;
   e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc draws on the registers the CTA was launched with: refuse
@@ -1057,11 +1093,18 @@ cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
                    !contiguous_strides(p.s_dq, p.H, p.Nq, d) ||
                    !contiguous_strides(p.s_dk, p.H, p.Nk, d) ||
                    !contiguous_strides(p.s_dv, p.H, p.Nk, d);
+  const bool drop = p.drop.t4 != 0;
+  // dropout runs in the general-layout variant only (one extra build per shape)
 #define FA_BWD_CASE(TY, DD)                                                        \
-  return causal ? (gen ? launch_bwd_t<TY, DD, true, true>(a)                       \
-                       : launch_bwd_t<TY, DD, true, false>(a))                     \
-                : (gen ? launch_bwd_t<TY, DD, false, true>(a)                      \
-                       : launch_bwd_t<TY, DD, false, false>(a));
+  {                                                                                \
+    if (drop)                                                                      \
+      return causal ? launch_bwd_t<TY, DD, true, true, true>(a)                    \
+                    : launch_bwd_t<TY, DD, false, true, true>(a);                  \
+    return causal ? (gen ? launch_bwd_t<TY, DD, true, true>(a)                     \
+                         : launch_bwd_t<TY, DD, true, false>(a))                   \
+                  : (gen ? launch_bwd_t<TY, DD, false, true>(a)                    \
+                         : launch_bwd_t<TY, DD, false, false>(a));                 \
+  }
   if (dtype == FA_BF16) {
     if (d == 64) FA_BWD_CASE(__nv_bfloat16, 64)
     if (d == 128) FA_BWD_CASE(__nv_bfloat16, 128)

@@ -29,6 +29,7 @@
 // are done) with TMA tensor stores.
 #define FA_SITE_BASE 10000
 #include "common.cuh"
+#include "dropout.cuh"
 #include "launch.h"
 
 namespace fa {
@@ -191,7 +192,8 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 
 // GEN: some tensor map is 4-D (a layout whose heads and batches do not merge
 // into one index); otherwise every map is the 3-D (d, N, B·H) form.
-template <typename T, int D, bool CAUSAL, bool GEN>
+// DROP: dropout on P (16-bit types only), masks drawn in the softmax warps.
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP>
 __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -551,6 +553,13 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       } else {
 #pragma unroll
         for (int c = 0; c < Tr::BN; c += 64) {
+          // Dropout: keep bytes of this row's columns k0 + c .. k0 + c + 63
+          // (pair e of the half sits in keep[e / 2], bytes 2·(e % 2) and up).
+          uint32_t keep[DROP ? 16 : 1];
+          if constexpr (DROP) {
+#pragma unroll
+            for (int g = 0; g < 4; ++g) keep16_row(p.drop, bh, qi, k0 + c + 16 * g, keep + 4 * g);
+          }
           uint32_t u[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
@@ -563,6 +572,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
             const float2 pr = ElemTraits<T>::unpack2(u[e]);
             sum2[q] = fadd2(sum2[q], pk2(pe.x, pe.y));
             sum2_p[q] = fadd2(sum2_p[q], pk2(pr.x, pr.y));
+            // the product sees the dropped weights; the sums above do not
+            if constexpr (DROP) u[e] &= keep_pair_mask(keep[e / 2], (2 * e) & 3);
           }
           tmem_st32(tS + c / 2, u);
         }
@@ -585,7 +596,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
     if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
     tc_fence_after();
     if (ok) {
-      const float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;
+      float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;
+      if constexpr (DROP) inv *= p.drop.scale;  // kept weights scaled by 256 / T
       const bool live = qi < p.Nq;
       if constexpr (TF32) {
         float* orow = reinterpret_cast<float*>(p.O) + (size_t(bh) * p.Nq + (live ? qi : 0)) * D;
@@ -656,10 +668,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL, bool GEN>
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false>
 static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   using Tr = FwdTraits<T, D>;
-  auto kern = fwd_kernel<T, D, CAUSAL, GEN>;
+  auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg redistributes the registers the CTA was launched with; refuse
@@ -683,16 +695,23 @@ int fwd_rows_per_cta(int dtype, int d) { return 128 * fwd_tiles(dtype == FA_FP32
 
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
   const bool gen = a.params.map4d != 0;  // only 4-D tensor maps differ: every access is TMA
-#define FA_FWD_CASE(TY, DD)                                                                       \
-  return causal ? (gen ? launch_fwd_t<TY, DD, true, true>(a) : launch_fwd_t<TY, DD, true, false>(a)) \
-                : (gen ? launch_fwd_t<TY, DD, false, true>(a) : launch_fwd_t<TY, DD, false, false>(a));
+  const bool drop = a.params.drop.t4 != 0;
+  // dropout runs in the general-layout variant only (one extra build per shape)
+#define FA_FWD_CASE(TY, DD)                                                                      \
+  {                                                                                              \
+    if (drop)                                                                                    \
+      return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
+                    : launch_fwd_t<TY, DD, false, true, true>(a);                                \
+    return causal ? (gen ? launch_fwd_t<TY, DD, true, true>(a) : launch_fwd_t<TY, DD, true, false>(a)) \
+                  : (gen ? launch_fwd_t<TY, DD, false, true>(a) : launch_fwd_t<TY, DD, false, false>(a)); \
+  }
   if (dtype == FA_BF16) {
     if (d == 64) FA_FWD_CASE(__nv_bfloat16, 64)
     if (d == 128) FA_FWD_CASE(__nv_bfloat16, 128)
   } else if (dtype == FA_FP16) {
     if (d == 64) FA_FWD_CASE(__half, 64)
     if (d == 128) FA_FWD_CASE(__half, 128)
-  } else if (dtype == FA_FP32) {  // contiguous only (the host rejects other layouts)
+  } else if (dtype == FA_FP32) {  // contiguous, no dropout (the host rejects the rest)
     if (d == 64) return causal ? launch_fwd_t<float, 64, true, false>(a) : launch_fwd_t<float, 64, false, false>(a);
   }
 #undef FA_FWD_CASE

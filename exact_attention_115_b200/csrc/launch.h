@@ -26,6 +26,14 @@ __host__ __device__ __forceinline__ long long row_offset(const Strides& s, int b
     return ((long long)bh * N + n) * D;
 }
 
+// Dropout of the attention weights (see dropout.cuh); t4 == 0 means none.
+struct DropoutParams {
+  uint32_t k0, k1;  // Philox key: the seed's low and high words
+  uint32_t offset;  // Philox counter word 3
+  uint32_t t4;      // keep threshold T (1..255) in each of the four bytes
+  float scale;      // 256 / T, applied to the kept weights
+};
+
 struct FwdParams {
   const void* Q;  // raw inputs (read directly only by the fp32 path)
   const void* K;
@@ -37,6 +45,7 @@ struct FwdParams {
   int n_qblocks;     // ceil(Nq / fwd_rows_per_cta): one CTA per block of query rows
   int head_group;    // heads per launch-order group (see head_group_for)
   int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
+  DropoutParams drop;
 };
 
 struct FwdLaunch {
@@ -74,6 +83,7 @@ struct BwdParams {
   int head_group;     // heads per launch-order group (see head_group_for)
   Strides s_o, s_do, s_dq, s_dk, s_dv;  // plain (non-TMA) accesses; Q, K, V, dO go through tensor maps
   int map4d;  // bit per tensor map (Q 0, K 1, V 2, dK 3, dO 4, dV 5): 4-D (d, N, H, B), else 3-D (d, N, B·H)
+  DropoutParams drop;
 };
 
 struct BwdLaunch {

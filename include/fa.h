@@ -79,14 +79,38 @@ typedef struct {
   long long b, h, n;
 } fa_layout;
 
+/* Dropout of the attention weights.  The study notes on FlashAttention V1/V2
+ * (51CTO), section "算法的改进", mention the dropout steps of the V1
+ * algorithm; the library applies them to the normalised weights:
+ * O = (P ∘ Z · 256/T) V with Z a 0/1 keep mask, while L stays the logsumexp
+ * of the undropped scores.  The keep threshold is T = round((1 − p)·256)
+ * (computed in double from the float p), so a weight survives with
+ * probability T/256.  Z is drawn inside the kernels by the counter-based
+ * generator Philox4x32-10 (Salmon et al., "Parallel Random Numbers: As Easy
+ * as 1, 2, 3", SC'11): 4×4 blocks of the [Nq, Nk] weights of head index
+ * bh = b·H + h, block (query rows 4r.., keys 4c..) from counter
+ * (c, r, bh, offset) and key (seed low word, seed high word); word i of the
+ * output belongs to query row 4r + i and byte j of that word (least
+ * significant first) to key 4c + j; a weight is kept iff its byte is below T.
+ * The backward redraws the same Z from the same seed and offset, so the two
+ * calls must get the same fa_dropout. */
+typedef struct {
+  float p;                 /* probability of dropping a weight, in [0, 1); 0 = none */
+  unsigned long long seed; /* generator key */
+  unsigned int offset;     /* counter word 3: a separate stream per call */
+} fa_dropout;
+
 /* fa_fwd for tensors with arbitrary strides (one fa_layout each for Q, K, V
- * and O; L stays contiguous [B, H, Nq]).  fa_fwd is this call with contiguous
- * layouts.  Layout errors: FA_ERR_INVALID; a non-contiguous fp32 tensor:
- * FA_ERR_UNSUPPORTED (the fp32 path reads contiguous tensors). */
-int fa_fwd_strided(const void* Q, const void* K, const void* V, void* O, float* L,
-                   const fa_layout* lq, const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
-                   int B, int H, int Nq, int Nk, int d, int causal, float scale, int dtype,
-                   void* stream);
+ * and O; L stays contiguous [B, H, Nq]) and optional dropout (NULL or p = 0:
+ * none).  fa_fwd is this call with contiguous layouts and no dropout.
+ * Layout errors and a dropout probability outside [0, 1) (or one that keeps
+ * nothing after rounding): FA_ERR_INVALID; a non-contiguous fp32 tensor or
+ * fp32 with dropout: FA_ERR_UNSUPPORTED (the fp32 path reads contiguous
+ * tensors and has no dropout). */
+int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
+              const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
+              int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
+              void* stream);
 
 /* Bytes of device workspace fa_bwd needs for this problem (0 on invalid
  * arguments).  The workspace holds D = rowsum(dO ∘ O) [B,H,Nq] and the fp32
@@ -103,14 +127,18 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* fa_bwd for tensors with arbitrary strides (layouts of Q, K, V, O, dO, dQ,
- * dK, dV in that order; L stays contiguous).  fa_bwd is this call with
- * contiguous layouts.  Errors as for fa_fwd_strided and fa_bwd. */
-int fa_bwd_strided(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                   const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
-                   const fa_layout* lk, const fa_layout* lv, const fa_layout* lo,
-                   const fa_layout* ldo, const fa_layout* ldq, const fa_layout* ldk,
-                   const fa_layout* ldv, int B, int H, int Nq, int Nk, int d, int causal,
-                   float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
+ * dK, dV in that order; L stays contiguous) and the forward's dropout (the
+ * same fa_dropout as the forward call, or NULL).  With dropout the gradient
+ * is the exact one for the drawn Z: dV = (P ∘ Z · s)ᵀ dO,
+ * dP = (dO Vᵀ) ∘ Z · s, dS = P ∘ (dP − D), s = 256/T.  fa_bwd is this call
+ * with contiguous layouts and no dropout.  Errors as for fa_fwd_ex and
+ * fa_bwd. */
+int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+              const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
+              const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
+              const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
+              int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
+              void* workspace, size_t ws_bytes, void* stream);
 
 /* How fa_bwd reduces the dQ contributions of the different K/V blocks:
  *   0 = automatic (the measured faster strategy for the shape),

@@ -142,20 +142,45 @@ def test_selftest_rejects_limits_out_of_range(lib):
     assert lib.fa_selftest_wait_timeout(1000001, None) == fa.FA_ERR_INVALID
 
 
-def test_strided_entry_points_validate_layouts(lib):
+def test_ex_entry_points_validate_layouts(lib):
     L = fa.Layout
     good, bad = L(2 * 64 * 64, 64 * 64, 64), L(2 * 64 * 64, 64 * 64, 3)  # 3 elements: not 16-byte aligned
     P = 4096  # any 16-byte-aligned non-null address: the call returns before touching memory
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
-    assert lib.fa_fwd_strided(P, P, P, P, P, r(bad), r(good), r(good), r(good), *args, fa.FA_BF16,
-                              None) == fa.FA_ERR_INVALID
-    assert lib.fa_fwd_strided(P, P, P, P, P, None, r(good), r(good), r(good), *args, fa.FA_BF16,
-                              None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, r(bad), r(good), r(good), r(good), *args, fa.FA_BF16,
+                         None, None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, None, r(good), r(good), r(good), *args, fa.FA_BF16,
+                         None, None) == fa.FA_ERR_INVALID
     # fp32 reads contiguous tensors only
     nc = L(2 * 64 * 64, 64, 2 * 64)
-    assert lib.fa_fwd_strided(P, P, P, P, P, r(nc), r(good), r(good), r(good), *args, fa.FA_FP32,
-                              None) == fa.FA_ERR_UNSUPPORTED
+    assert lib.fa_fwd_ex(P, P, P, P, P, r(nc), r(good), r(good), r(good), *args, fa.FA_FP32,
+                         None, None) == fa.FA_ERR_UNSUPPORTED
     lays = [r(good)] * 8
-    assert lib.fa_bwd_strided(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, P,
-                              1 << 30, None) == fa.FA_ERR_INVALID
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, None, P,
+                         1 << 30, None) == fa.FA_ERR_INVALID
+
+
+@pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, float("nan"), 0.999])
+def test_ex_entry_points_reject_bad_dropout(lib, p):
+    """A probability outside [0, 1), or one that rounds to keeping nothing
+    (T = round((1 - p)·256) = 0), is invalid; checked before any launch."""
+    good = fa.Layout(2 * 64 * 64, 64 * 64, 64)
+    P = 4096
+    args = (1, 2, 64, 64, 64, 0, 0.125)
+    r = ctypes.byref
+    dr = fa.Dropout(p, 1, 0)
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_BF16, r(dr),
+                         None) == fa.FA_ERR_INVALID
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *[r(good)] * 8, *args, fa.FA_BF16, r(dr), P,
+                         1 << 30, None) == fa.FA_ERR_INVALID
+
+
+def test_fp32_has_no_dropout(lib):
+    good = fa.Layout(2 * 64 * 64, 64 * 64, 64)
+    P = 4096
+    args = (1, 2, 64, 64, 64, 0, 0.125)
+    r = ctypes.byref
+    dr = fa.Dropout(0.1, 1, 0)
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_FP32, r(dr),
+                         None) == fa.FA_ERR_UNSUPPORTED
