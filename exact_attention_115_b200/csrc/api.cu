@@ -191,8 +191,15 @@ int dropout_params(const fa_dropout* dr, DropoutParams* out) {
   const long t = std::lrint((1.0 - pd) * 256.0);
   if (t < 1) return FA_ERR_INVALID;
   if (t >= 256) return FA_OK;  // rounds to keeping everything: no dropout
-  out->k0 = uint32_t(dr->seed & 0xFFFFFFFFull);
-  out->k1 = uint32_t(dr->seed >> 32);
+  // Philox4x32-10 key schedule: round r uses the seed's words plus r times
+  // the Weyl constants (mod 2^32); computed once here, read by every draw.
+  uint32_t k0 = uint32_t(dr->seed & 0xFFFFFFFFull), k1 = uint32_t(dr->seed >> 32);
+  for (int r = 0; r < 10; ++r) {
+    out->rk[r][0] = k0;
+    out->rk[r][1] = k1;
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
   out->offset = dr->offset;
   out->t4 = uint32_t(t) * 0x01010101u;
   out->scale = float(256.0 / double(t));

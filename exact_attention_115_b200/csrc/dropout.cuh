@@ -23,16 +23,17 @@
 
 namespace fa {
 
-// Philox4x32-10: ten rounds of two 32×32→64 products and a key-mixed swap,
-// the key advancing by the Weyl constants between rounds.
-__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+// Philox4x32-10: ten rounds of two 32×32→64 products and a key-mixed swap.
+// The round keys (the seed advanced by the Weyl constants, rk[r]) come
+// precomputed from the host, so a round is two wide products and two
+// three-way XORs.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const uint32_t (&rk)[10][2]) {
 #pragma unroll
   for (int r = 0; r < 10; ++r) {
-    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
-    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
-    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
-    k0 += 0x9E3779B9u;
-    k1 += 0xBB67AE85u;
+    const uint64_t p0 = uint64_t(0xD2511F53u) * c.x;
+    const uint64_t p1 = uint64_t(0xCD9E8D57u) * c.z;
+    c = make_uint4(uint32_t(p1 >> 32) ^ c.y ^ rk[r][0], uint32_t(p1),
+                   uint32_t(p0 >> 32) ^ c.w ^ rk[r][1], uint32_t(p0));
   }
   return c;
 }
@@ -78,7 +79,7 @@ __device__ __forceinline__ void keep16_row(const DropoutParams& d, int bh, int r
   const int m = row & 3;
   const uint4 w = philox4x32_10(make_uint4(uint32_t(col0 / 4 + m), uint32_t(row >> 2), uint32_t(bh),
                                            d.offset),
-                                d.k0, d.k1);
+                                d.rk);
   out[0] = w.x; out[1] = w.y; out[2] = w.z; out[3] = w.w;  // block m, word i ↔ row 4·rb + i
   lane4_transpose(out, m);  // out[n] = word m (this row) of block n
 #pragma unroll
@@ -94,7 +95,7 @@ __device__ __forceinline__ void keep16_col(const DropoutParams& d, int bh, int k
   const int m = key & 3;
   const uint4 w = philox4x32_10(make_uint4(uint32_t(key >> 2), uint32_t(row0 / 4 + m), uint32_t(bh),
                                            d.offset),
-                                d.k0, d.k1);
+                                d.rk);
   out[0] = w.x; out[1] = w.y; out[2] = w.z; out[3] = w.w;  // block m: word i ↔ row, byte j ↔ key
   byte4_transpose(out);      // out[j]: byte i ↔ row 4·rb + i, for key 4·cb + j
   lane4_transpose(out, m);   // out[n] = block n's word for this key

@@ -28,10 +28,10 @@ __host__ __device__ __forceinline__ long long row_offset(const Strides& s, int b
 
 // Dropout of the attention weights (see dropout.cuh); t4 == 0 means none.
 struct DropoutParams {
-  uint32_t k0, k1;  // Philox key: the seed's low and high words
-  uint32_t offset;  // Philox counter word 3
-  uint32_t t4;      // keep threshold T (1..255) in each of the four bytes
-  float scale;      // 256 / T, applied to the kept weights
+  uint32_t rk[10][2];  // Philox round keys: the seed's (low, high) words plus r·(Weyl constants)
+  uint32_t offset;     // Philox counter word 3
+  uint32_t t4;         // keep threshold T (1..255) in each of the four bytes
+  float scale;         // 256 / T, applied to the kept weights
 };
 
 struct FwdParams {
