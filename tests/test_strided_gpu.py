@@ -1,5 +1,5 @@
-"""GPU parity for tensors with arbitrary strides (fa_fwd_strided /
-fa_bwd_strided through the Python binding): [B, N, H, d] ("sequence before
+"""GPU parity for tensors with arbitrary strides (fa_fwd_ex / fa_bwd_ex
+through the Python binding): [B, N, H, d] ("sequence before
 head"), slices of a fused [B, N, 3, H, d] QKV projection, rows padded past
 d (heads and batches still merge into one tensor-map index, but the plain
 accesses need the strides) and a mix of these in one call.  The
