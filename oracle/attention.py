@@ -33,8 +33,16 @@ Readings where the pages are silent (each also listed in the design notes):
 * causal masking is bottom-right aligned: key j is visible to query i iff
   j <= i + (Nk - Nq).  For Nq == Nk this is the plain lower triangle.
 * L is the natural-log logsumexp of the scaled, masked scores of a row.
-* a row with no visible key (only possible in a split of the decode) has
-  O = 0 and L = -inf.
+* a row with no visible key (a split of the decode, or a key-padding mask
+  that hides every key) has O = 0 and L = -inf.
+* key padding (``kv_len``): batch element b sees only keys j < kv_len[b]
+  (an additive 0 / -inf mask over keys, ANDed with the causal mask, whose
+  alignment still uses the full Nq and Nk).  The FlashAttention1 post
+  (CSDN), section "引言/动机", lists the fused chain as matmul, scale, mask,
+  softmax, so a mask acts on the scaled scores before the softmax; the
+  51CTO notes' background list names custom masks as a reason to write
+  one's own kernel.  Which masks is not fixed; this one is the padding of
+  batched sequences of different lengths.
 
 Everything is float64.  Inputs are whatever the caller passes (normally the
 storage-dtype values the GPU sees, upcast exactly).  Rows are processed in
@@ -101,12 +109,13 @@ def tiled_softmax_then_matmul(s_row, V) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Forward: the plain definition, per (batch, head), rows in chunks.
 # --------------------------------------------------------------------------
-def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None):
+def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None, nk_valid=None):
     """P (softmax rows) and L for the given query rows of one head.
 
     q: [r, d] the query rows, k: [Nk, d].  ``rows`` are the absolute indices
     of those query rows (needed for the causal mask) and ``nq_total`` the
-    head's full query length.  Returns (P [r, Nk], L [r]).
+    head's full query length; keys j >= ``nk_valid`` are masked (key
+    padding).  Returns (P [r, Nk], L [r]).
     """
     q = _f64(q)
     k = _f64(k)
@@ -119,6 +128,8 @@ def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None):
     s = scale * (q @ k.T)
     if causal:
         s = np.where(causal_visible(nq_total, nk, rows), s, -np.inf)
+    if nk_valid is not None:
+        s = np.where(np.arange(nk)[None, :] < nk_valid, s, -np.inf)
     m = s.max(axis=1, keepdims=True)
     empty = ~np.isfinite(m)  # row with no visible key
     m = np.where(empty, 0.0, m)
@@ -131,7 +142,7 @@ def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None):
 
 
 def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None, keep_fn=None,
-                 kscale: float = 1.0):
+                 kscale: float = 1.0, nk_valid=None):
     """O [r, d] and L [r] for query rows of one head (see ``head_probs``).
 
     With dropout, ``keep_fn(rows, cols)`` gives the boolean keep mask at
@@ -150,7 +161,7 @@ def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None, 
     L = np.empty(r)
     for c0 in range(0, r, _ROW_CHUNK):
         c1 = min(r, c0 + _ROW_CHUNK)
-        p, l = head_probs(q[c0:c1], k, scale, causal, rows[c0:c1], nq_total)
+        p, l = head_probs(q[c0:c1], k, scale, causal, rows[c0:c1], nq_total, nk_valid)
         if keep_fn is not None:
             p = p * keep_fn(rows[c0:c1], np.arange(k.shape[0])) * kscale
         O[c0:c1] = p @ v
@@ -168,10 +179,11 @@ def _dropout_fn(dropout, bh):
     return (lambda r, c: philox.keep_mask(bh, r, c, p, seed, offset)), philox.keep_scale(p)
 
 
-def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None):
+def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None, kv_len=None):
     """O [B,H,Nq,d] and L [B,H,Nq] (float64) for [B,H,N,d] inputs.
     ``dropout`` = (p, seed, offset) applies the Philox keep mask of
-    ``oracle/philox.py`` to head index b·H + h."""
+    ``oracle/philox.py`` to head index b·H + h; ``kv_len`` (B integers)
+    hides keys j >= kv_len[b] of batch element b."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, H, Nq, d = Q.shape
     O = np.empty((B, H, Nq, V.shape[3]))
@@ -180,14 +192,16 @@ def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None)
         for h in range(H):
             fn, ks = _dropout_fn(dropout, b * H + h)
             O[b, h], L[b, h] = head_forward(Q[b, h], K[b, h], V[b, h], scale, causal,
-                                            keep_fn=fn, kscale=ks)
+                                            keep_fn=fn, kscale=ks,
+                                            nk_valid=None if kv_len is None else int(kv_len[b]))
     return O, L
 
 
 # --------------------------------------------------------------------------
 # Backward: the exact gradient of O = softmax(scale Q Kᵀ [masked]) V.
 # --------------------------------------------------------------------------
-def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale: float = 1.0):
+def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale: float = 1.0,
+                  nk_valid=None):
     """dQ, dK, dV, D for one head (all query rows), float64.
 
     D_i = Σ_c dO_ic O_ic; dP = dO Vᵀ; dS = P ∘ (dP − D); dV = Pᵀ dO;
@@ -204,7 +218,7 @@ def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale:
     rows_all = np.arange(nq)
     for c0 in range(0, nq, _ROW_CHUNK):
         c1 = min(nq, c0 + _ROW_CHUNK)
-        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq)
+        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq, nk_valid)
         z = 1.0 if keep_fn is None else keep_fn(rows_all[c0:c1], np.arange(k.shape[0])) * kscale
         pz = p * z
         o = pz @ v
@@ -218,9 +232,10 @@ def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale:
     return dq, dk, dv, D
 
 
-def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=None):
-    """dQ, dK, dV ([B,H,N,d]) and D ([B,H,Nq]) in float64 (``dropout`` as in
-    ``attention_forward``)."""
+def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=None,
+                       kv_len=None):
+    """dQ, dK, dV ([B,H,N,d]) and D ([B,H,Nq]) in float64 (``dropout`` and
+    ``kv_len`` as in ``attention_forward``)."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     B, H = Q.shape[:2]
     dQ = np.empty_like(Q)
@@ -231,12 +246,13 @@ def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=
         for h in range(H):
             fn, ks = _dropout_fn(dropout, b * H + h)
             dQ[b, h], dK[b, h], dV[b, h], D[b, h] = head_backward(
-                Q[b, h], K[b, h], V[b, h], dO[b, h], scale, causal, keep_fn=fn, kscale=ks)
+                Q[b, h], K[b, h], V[b, h], dO[b, h], scale, causal, keep_fn=fn, kscale=ks,
+                nk_valid=None if kv_len is None else int(kv_len[b]))
     return dQ, dK, dV, D
 
 
 def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows, keep_fn=None,
-                       kscale: float = 1.0):
+                       kscale: float = 1.0, nk_valid=None):
     """The same gradient as ``head_backward`` at selected rows only.
 
     Returns (dQ[q_rows], dK[k_rows], dV[k_rows], D[q_rows]).  dK/dV of a key
@@ -252,7 +268,7 @@ def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows, 
     rows_all = np.arange(nq)
     for c0 in range(0, nq, _ROW_CHUNK):
         c1 = min(nq, c0 + _ROW_CHUNK)
-        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq)
+        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq, nk_valid)
         z = 1.0 if keep_fn is None else keep_fn(rows_all[c0:c1], np.arange(k.shape[0])) * kscale
         o = (p * z) @ v
         Di = (do[c0:c1] * o).sum(axis=1)
@@ -262,7 +278,7 @@ def head_backward_rows(q, k, v, do, scale: float, causal: bool, q_rows, k_rows, 
         dsc = pc * (dpc - Di[:, None])
         dv += (pc * zc).T @ do[c0:c1]
         dk += scale * (dsc.T @ q[c0:c1])
-    p, _ = head_probs(q[q_rows], k, scale, causal, q_rows, nq)
+    p, _ = head_probs(q[q_rows], k, scale, causal, q_rows, nq, nk_valid)
     z = 1.0 if keep_fn is None else keep_fn(q_rows, np.arange(k.shape[0])) * kscale
     o = (p * z) @ v
     Dq = (do[q_rows] * o).sum(axis=1)

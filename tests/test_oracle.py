@@ -329,3 +329,59 @@ def test_decode_matches_sdpa():
     O, L = oracle.attention_decode(Q, K, V, 0.25)
     want, _ = _sdpa(Q, K, V, 0.25, False)
     assert np.max(np.abs(O - want)) <= 1e-13
+
+
+# --------------------------------------------------------------------------
+# Key padding (kv_len): pinned by the truncated problem it must equal.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_padding_matches_torch_autograd(causal):
+    """Hiding keys j >= kv_len[b] against torch float64 SDPA with the same
+    boolean mask (padding AND bottom-right causal with the full Nk), forward
+    and autograd gradients; the hidden keys get zero dK and dV."""
+    rng = _rng(500)
+    B, H, Nq, Nk, d = 3, 2, 7, 11, 4
+    Q, dO = rng.standard_normal((B, H, Nq, d)), rng.standard_normal((B, H, Nq, d))
+    K, V = rng.standard_normal((B, H, Nk, d)), rng.standard_normal((B, H, Nk, d))
+    kv_len = [11, 9, 6]
+    O, L = oracle.attention_forward(Q, K, V, 0.5, causal, kv_len=kv_len)
+    dQ, dK, dV, _ = oracle.attention_backward(Q, K, V, dO, 0.5, causal, kv_len=kv_len)
+    j = np.arange(Nk)[None, None, None, :]
+    vis = j < np.array(kv_len)[:, None, None, None]
+    if causal:
+        vis = vis & (j <= np.arange(Nq)[None, None, :, None] + (Nk - Nq))
+    q, k, v = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.tensor(vis),
+                                                         scale=0.5)
+    o.backward(torch.tensor(dO))
+    assert np.max(np.abs(O - o.detach().numpy())) <= 1e-12
+    for got, want in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        assert np.max(np.abs(got - want.numpy())) <= 1e-11
+    for b, n in enumerate(kv_len):
+        assert np.all(dK[b, :, n:] == 0) and np.all(dV[b, :, n:] == 0)
+
+
+def test_key_padding_full_length_is_no_mask_and_zero_length_is_empty():
+    rng = _rng(501)
+    Q, K, V, dO = (rng.standard_normal((2, 1, 5, 3)) for _ in range(4))
+    O0, L0 = oracle.attention_forward(Q, K, V, 0.4, False)
+    O1, L1 = oracle.attention_forward(Q, K, V, 0.4, False, kv_len=[5, 5])
+    assert np.array_equal(O0, O1) and np.array_equal(L0, L1)
+    O2, L2 = oracle.attention_forward(Q, K, V, 0.4, False, kv_len=[0, 5])
+    assert np.all(O2[0] == 0) and np.all(np.isneginf(L2[0]))
+    assert np.array_equal(O2[1], O0[1])
+    g = oracle.attention_backward(Q, K, V, dO, 0.4, False, kv_len=[0, 5])
+    for x in g[:3]:
+        assert np.all(x[0] == 0)
+
+
+def test_key_padding_matches_torch_sdpa_bool_mask():
+    rng = _rng(502)
+    B, H, N, d = 2, 2, 33, 8
+    Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    kv_len = [20, 33]
+    mask = torch.tensor(np.arange(N)[None, None, None, :] < np.array(kv_len)[:, None, None, None])
+    o = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(Q), torch.tensor(K), torch.tensor(V), attn_mask=mask, scale=0.3)
+    O, _ = oracle.attention_forward(Q, K, V, 0.3, False, kv_len=kv_len)
+    assert np.max(np.abs(O - o.numpy())) <= 1e-12
