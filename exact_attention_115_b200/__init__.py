@@ -34,8 +34,9 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I,
                     _VP, _SZ, _VP]),
-    "fa_fwd_ex": (_I, [_VP] * 9 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP]),
-    "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _SZ, _VP]),
+    "fa_fwd_ex": (_I, [_VP] * 9 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP]),
+    "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _SZ,
+                                               _VP]),
     "fa_set_bwd_dq_mode": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
@@ -99,6 +100,18 @@ def _dropout(p, seed, offset):
     return Dropout(float(p), int(seed) & 0xFFFFFFFFFFFFFFFF, int(offset) & 0xFFFFFFFF)
 
 
+def _kv_len_ptr(kv_len, B, device):
+    """Device pointer of a key-padding length tensor (int32 [B] on the
+    tensors' device), or None."""
+    if kv_len is None:
+        return None
+    if not isinstance(kv_len, torch.Tensor) or kv_len.dtype != torch.int32:
+        raise TypeError("kv_len must be an int32 torch.Tensor")
+    if kv_len.device != device or tuple(kv_len.shape) != (B,) or not kv_len.is_contiguous():
+        raise ValueError(f"kv_len must be a contiguous [B={B}] tensor on {device}")
+    return kv_len.data_ptr()
+
+
 def _layout(t) -> Layout:
     s = t.stride()
     return Layout(s[0], s[1], s[2])
@@ -132,12 +145,13 @@ def _raise(fn, code):
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-            dropout_p: float = 0.0, seed: int = 0, offset: int = 0):
+            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, kv_len=None):
     """O, L = attention(q, k, v).  q, k, v (and out) are [B, H, N, d] with any
     strides whose d dimension is contiguous (a [B, N, H, d] tensor viewed
     with .transpose(1, 2) works as is).  ``dropout_p`` > 0 drops attention
     weights with the keep mask that ``seed`` and ``offset`` select (pass the
-    same three to ``backward``).  Returns (O [B,H,Nq,d] q.dtype,
+    same three to ``backward``).  ``kv_len`` (int32 [B] on the device) hides
+    keys j >= kv_len[b] of batch element b.  Returns (O [B,H,Nq,d] q.dtype,
     L [B,H,Nq] fp32 contiguous)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
@@ -153,7 +167,8 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     _check("out", out, (B, H, Nq, d), q.dtype, strided=True)
     _check("lse", lse, (B, H, Nq), torch.float32)
     dr = _dropout(dropout_p, seed, offset)
-    if dr is None and all(t.is_contiguous() for t in (q, k, v, out)):
+    kvl = _kv_len_ptr(kv_len, B, q.device)
+    if dr is None and kvl is None and all(t.is_contiguous() for t in (q, k, v, out)):
         rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
                           _dtype_code(q), _stream(q.device))
@@ -163,7 +178,7 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                          ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
                          B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                         None if dr is None else ctypes.byref(dr), _stream(q.device))
+                         None if dr is None else ctypes.byref(dr), kvl, _stream(q.device))
     _raise("fa_fwd_ex", rc)
     return out, lse
 
@@ -183,9 +198,9 @@ def set_bwd_dq_mode(mode: int) -> int:
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace=None, dropout_p: float = 0.0, seed: int = 0,
-             offset: int = 0):
+             offset: int = 0, kv_len=None):
     """dQ, dK, dV of attention given the forward's O and L and the upstream dO
-    (and the forward's ``dropout_p``, ``seed`` and ``offset``)."""
+    (and the forward's ``dropout_p``, ``seed``, ``offset`` and ``kv_len``)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -206,7 +221,8 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     _check("workspace", workspace)
     ts = (q, k, v, o, do, dq, dk, dv)
     dr = _dropout(dropout_p, seed, offset)
-    if dr is None and all(t.is_contiguous() for t in ts):
+    kvl = _kv_len_ptr(kv_len, B, dev)
+    if dr is None and kvl is None and all(t.is_contiguous() for t in ts):
         rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
@@ -219,7 +235,7 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                          *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d, int(bool(causal)),
                          float(scale), _dtype_code(q), None if dr is None else ctypes.byref(dr),
-                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         kvl, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                          _stream(dev))
     _raise("fa_bwd_ex", rc)
     return dq, dk, dv

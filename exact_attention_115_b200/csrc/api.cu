@@ -215,7 +215,7 @@ extern "C" {
 int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              void* stream) {
+              const int* kv_len, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
@@ -235,10 +235,13 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   st = dropout_params(dropout, &drop);
   if (st != FA_OK) return st;
   if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID;
+  if (kv_len && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
   a.params.drop = drop;
+  a.params.kv_len = kv_len;
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
@@ -267,7 +270,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
            int Nk, int d, int causal, float scale, int dtype, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
   return fa_fwd_ex(Q, K, V, O, L, &lq, &lk, &lk, &lq, B, H, Nq, Nk, d, causal, scale, dtype, nullptr,
-                   stream);
+                   nullptr, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
@@ -287,7 +290,7 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
               const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
               int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              void* workspace, size_t ws_bytes, void* stream) {
+              const int* kv_len, void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
@@ -309,6 +312,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   st = dropout_params(dropout, &drop);
   if (st != FA_OK) return st;
   if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID;
+  if (kv_len && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int mode = effective_dq_mode(B, H, Nq, Nk, d);
   const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
@@ -349,6 +354,7 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   p.s_dv = to_strides(ldv);
   for (int i = 0; i < 6; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dK 3, dO 4, dV 5
   p.drop = drop;
+  p.kv_len = kv_len;
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;
@@ -360,7 +366,7 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
   return fa_bwd_ex(Q, K, V, O, dO, L, dQ, dK, dV, &lq, &lk, &lk, &lq, &lq, &lq, &lk, &lk, B, H, Nq,
-                   Nk, d, causal, scale, dtype, nullptr, workspace, ws_bytes, stream);
+                   Nk, d, causal, scale, dtype, nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {

@@ -220,10 +220,12 @@ __global__ void __launch_bounds__(512, 1)
 
   // Work item j: (K/V block kb, head bh) in the grouped order (causal: the
   // first key blocks are seen by the most query tiles) and its query-tile
-  // range [i0, i0 + n_q).
+  // range [i0, i0 + n_q).  A block wholly past the batch element's key
+  // padding length has no steps (its dK and dV rows are written as zeros).
   auto item = [&](int j, int& bh, int& kb, int& i0, int& n_q) {
     grouped_order(j, p.B * p.H, p.n_kblocks, p.head_group, bh, kb);
     q_tile_range<BM, CAUSAL>(kb, p.Nq, p.Nk, i0, n_q);
+    if (p.kv_len && kb * Tr::BN >= keys_of(p.kv_len, bh, p.H, p.Nk)) n_q = 0;
   };
   // The it-th work item of this CTA, as the scheduler published it in the
   // item ring; false after the last one (or on abort).
@@ -579,7 +581,7 @@ __global__ void __launch_bounds__(512, 1)
 #endif
       const int key0 = kb * Tr::BN;
       const int key = key0 + kr;
-      const bool key_live = key < p.Nk;
+      const bool key_live = key < keys_of(p.kv_len, bh, p.H, p.Nk);
       const int qmin = key - off;  // first query row that sees this key
       for (int i = 0; i < n_q; ++i) {
         const int gs = g + i, s = gs & 1;

@@ -242,6 +242,12 @@ __device__ __forceinline__ void tma_store_bh(const CUtensorMap* map, bool map4d,
     tma_store_3d(map, src, x, y, bh);
 }
 
+// Keys visible to head index bh = b·H + h: all Nk, or the key-padding length
+// kv_len[b] clamped to [0, Nk].
+__device__ __forceinline__ int keys_of(const int* kv_len, int bh, int H, int Nk) {
+  return kv_len ? min(max(__ldg(kv_len + bh / H), 0), Nk) : Nk;
+}
+
 // ------------------------------------------------------------------ tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(

@@ -217,14 +217,17 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 #ifdef FA_TRACE
   const bool trace_on = blockIdx.x == 0;
 #endif
-  const int off = p.Nk - p.Nq;  // bottom-right causal alignment
+  const int off = p.Nk - p.Nq;  // bottom-right causal alignment (full Nk)
+  const int nk = keys_of(p.kv_len, bh, p.H, p.Nk);  // keys this batch element sees
 
-  int kv_end = p.Nk;
+  int kv_end = nk;
   if (CAUSAL) {
     const int q_last = min(q_row0 + 128 * Tr::TILES - 1, p.Nq - 1);
-    kv_end = min(p.Nk, q_last + off + 1);
+    kv_end = min(nk, q_last + off + 1);
   }
-  const int n_kv = (kv_end + Tr::BN - 1) / Tr::BN;
+  // at least one (then fully masked) tile, so that every role runs its loop
+  // once and an empty row still ends with O = 0 and L = -inf
+  const int n_kv = max(1, (kv_end + Tr::BN - 1) / Tr::BN);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < 2; ++i) {
@@ -481,10 +484,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       tmem_ld_wait();
       float* s = reinterpret_cast<float*>(&su[0][0]);
       const int k0 = j * Tr::BN;
-      const bool tail = k0 + Tr::BN > p.Nk;
+      const bool tail = k0 + Tr::BN > nk;
       const bool diag = CAUSAL && (k0 + Tr::BN - 1 > tile_first_row + off);
       if (tail || diag) {
-        int lim = p.Nk - k0;
+        int lim = nk - k0;
         if (CAUSAL) lim = min(lim, qi + off + 1 - k0);
 #pragma unroll
         for (int c = 0; c < Tr::BN; ++c)
@@ -596,7 +599,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
     if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
     tc_fence_after();
     if (ok) {
-      float inv = row_sum_p > 0.f ? 1.f / row_sum_p : 0.f;
+      // A row whose every score was masked (m_ref still -inf) has O = 0: the
+      // FMA-pipe exponentials leave it tiny but nonzero weights otherwise.
+      float inv = (row_sum_p > 0.f && m_ref != -INFINITY) ? 1.f / row_sum_p : 0.f;
       if constexpr (DROP) inv *= p.drop.scale;  // kept weights scaled by 256 / T
       const bool live = qi < p.Nq;
       if constexpr (TF32) {

@@ -46,6 +46,7 @@ struct FwdParams {
   int head_group;    // heads per launch-order group (see head_group_for)
   int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
+  const int* kv_len;  // key padding: keys of batch element b are [0, kv_len[b]); null = all Nk
 };
 
 struct FwdLaunch {
@@ -84,6 +85,7 @@ struct BwdParams {
   Strides s_o, s_do, s_dq, s_dk, s_dv;  // plain (non-TMA) accesses; Q, K, V, dO go through tensor maps
   int map4d;  // bit per tensor map (Q 0, K 1, V 2, dK 3, dO 4, dV 5): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
+  const int* kv_len;  // key padding, as in FwdParams
 };
 
 struct BwdLaunch {

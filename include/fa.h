@@ -100,9 +100,21 @@ typedef struct {
   unsigned int offset;     /* counter word 3: a separate stream per call */
 } fa_dropout;
 
-/* fa_fwd for tensors with arbitrary strides (one fa_layout each for Q, K, V
- * and O; L stays contiguous [B, H, Nq]) and optional dropout (NULL or p = 0:
- * none).  fa_fwd is this call with contiguous layouts and no dropout.
+/* Key padding (`kv_len`, for fa_fwd_ex and fa_bwd_ex): NULL, or a DEVICE
+ * array of B int32 lengths; batch element b then sees only keys
+ * j < kv_len[b] (values are clamped to [0, Nk] on the device).  It is the
+ * additive 0 / -inf mask of batched sequences padded to Nk, ANDed with the
+ * causal mask, whose bottom-right alignment still uses the full Nq and Nk.
+ * The FlashAttention1 post (CSDN), section "引言/动机", lists the fused chain
+ * as matmul, scale, mask, softmax: the mask acts on the scaled scores before
+ * the softmax.  A row that sees no key gets O = 0 and L = -inf; keys past
+ * the length get dK = dV = 0.  The pointer must be 4-byte aligned
+ * (FA_ERR_INVALID); fp32 has no key padding (FA_ERR_UNSUPPORTED).
+ *
+ * fa_fwd for tensors with arbitrary strides (one fa_layout each for Q, K, V
+ * and O; L stays contiguous [B, H, Nq]), optional dropout (NULL or p = 0:
+ * none) and optional key padding.  fa_fwd is this call with contiguous
+ * layouts, no dropout and no padding.
  * Layout errors and a dropout probability outside [0, 1) (or one that keeps
  * nothing after rounding): FA_ERR_INVALID; a non-contiguous fp32 tensor or
  * fp32 with dropout: FA_ERR_UNSUPPORTED (the fp32 path reads contiguous
@@ -110,7 +122,7 @@ typedef struct {
 int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              void* stream);
+              const int* kv_len, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for this problem (0 on invalid
  * arguments).  The workspace holds D = rowsum(dO ∘ O) [B,H,Nq] and the fp32
@@ -127,18 +139,18 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream);
 
 /* fa_bwd for tensors with arbitrary strides (layouts of Q, K, V, O, dO, dQ,
- * dK, dV in that order; L stays contiguous) and the forward's dropout (the
- * same fa_dropout as the forward call, or NULL).  With dropout the gradient
+ * dK, dV in that order; L stays contiguous), the forward's dropout (the
+ * same fa_dropout as the forward call, or NULL) and its key padding.  With dropout the gradient
  * is the exact one for the drawn Z: dV = (P ∘ Z · s)ᵀ dO,
  * dP = (dO Vᵀ) ∘ Z · s, dS = P ∘ (dP − D), s = 256/T.  fa_bwd is this call
- * with contiguous layouts and no dropout.  Errors as for fa_fwd_ex and
- * fa_bwd. */
+ * with contiguous layouts, no dropout and no padding.  Errors as for
+ * fa_fwd_ex and fa_bwd. */
 int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
               const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
               const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
               int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              void* workspace, size_t ws_bytes, void* stream);
+              const int* kv_len, void* workspace, size_t ws_bytes, void* stream);
 
 /* How fa_bwd reduces the dQ contributions of the different K/V blocks:
  *   0 = automatic (the measured faster strategy for the shape),

@@ -149,16 +149,16 @@ def test_ex_entry_points_validate_layouts(lib):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     assert lib.fa_fwd_ex(P, P, P, P, P, r(bad), r(good), r(good), r(good), *args, fa.FA_BF16,
-                         None, None) == fa.FA_ERR_INVALID
+                         None, None, None) == fa.FA_ERR_INVALID
     assert lib.fa_fwd_ex(P, P, P, P, P, None, r(good), r(good), r(good), *args, fa.FA_BF16,
-                         None, None) == fa.FA_ERR_INVALID
+                         None, None, None) == fa.FA_ERR_INVALID
     # fp32 reads contiguous tensors only
     nc = L(2 * 64 * 64, 64, 2 * 64)
     assert lib.fa_fwd_ex(P, P, P, P, P, r(nc), r(good), r(good), r(good), *args, fa.FA_FP32,
-                         None, None) == fa.FA_ERR_UNSUPPORTED
+                         None, None, None) == fa.FA_ERR_UNSUPPORTED
     lays = [r(good)] * 8
-    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, None, P,
-                         1 << 30, None) == fa.FA_ERR_INVALID
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, None, None,
+                         P, 1 << 30, None) == fa.FA_ERR_INVALID
 
 
 @pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, float("nan"), 0.999])
@@ -170,10 +170,10 @@ def test_ex_entry_points_reject_bad_dropout(lib, p):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     dr = fa.Dropout(p, 1, 0)
-    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_BF16, r(dr),
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_BF16, r(dr), None,
                          None) == fa.FA_ERR_INVALID
-    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *[r(good)] * 8, *args, fa.FA_BF16, r(dr), P,
-                         1 << 30, None) == fa.FA_ERR_INVALID
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *[r(good)] * 8, *args, fa.FA_BF16, r(dr), None,
+                         P, 1 << 30, None) == fa.FA_ERR_INVALID
 
 
 def test_fp32_has_no_dropout(lib):
@@ -182,5 +182,20 @@ def test_fp32_has_no_dropout(lib):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     dr = fa.Dropout(0.1, 1, 0)
-    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_FP32, r(dr),
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_FP32, r(dr), None,
+                         None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_key_padding_pointer_checks(lib):
+    good = fa.Layout(2 * 64 * 64, 64 * 64, 64)
+    P = 4096
+    args = (1, 2, 64, 64, 64, 0, 0.125)
+    r = ctypes.byref
+    lays4, lays8 = [r(good)] * 4, [r(good)] * 8
+    # a misaligned length array is invalid; fp32 has no key padding
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, P + 2,
+                         None) == fa.FA_ERR_INVALID
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *lays8, *args, fa.FA_BF16, None, P + 2, P,
+                         1 << 30, None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_FP32, None, P,
                          None) == fa.FA_ERR_UNSUPPORTED
