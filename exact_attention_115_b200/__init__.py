@@ -40,6 +40,7 @@ SIGNATURES = {
     "fa_set_bwd_dq_mode": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
+    "fa_decode_ex": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _SZ, _VP]),
     "fa_status": (_I, [_VP]),
     "fa_bwd_set_timing_events": (_I, [_VP, _VP]),
     "fa_last_timeout_site": (_I, []),
@@ -246,8 +247,10 @@ def decode_workspace_bytes(B, H, Nk, d, num_splits=0) -> int:
 
 
 def decode(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, lse=None,
-           workspace=None):
-    """Split-KV decode: q [B,H,1,d], k/v [B,H,Nk,d] -> (O [B,H,1,d], L [B,H,1])."""
+           workspace=None, kv_len=None):
+    """Split-KV decode: q [B,H,1,d], k/v [B,H,Nk,d] -> (O [B,H,1,d], L [B,H,1]).
+    ``kv_len`` (int32 [B] on the device) limits batch element b to its first
+    kv_len[b] keys (a padded KV cache)."""
     _check("q", q)
     B, H, one, d = q.shape
     if one != 1:
@@ -262,11 +265,19 @@ def decode(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, l
     need = decode_workspace_bytes(B, H, Nk, d, num_splits)
     if workspace is None:
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
-    rc = lib().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                         B, H, Nk, d, float(scale), _dtype_code(q), int(num_splits),
-                         workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                         _stream(q.device))
-    _raise("fa_decode", rc)
+    kvl = _kv_len_ptr(kv_len, B, q.device)
+    if kvl is None:
+        rc = lib().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
+                             int(num_splits), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(q.device))
+        _raise("fa_decode", rc)
+        return out, lse
+    rc = lib().fa_decode_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
+                            B, H, Nk, d, float(scale), _dtype_code(q), int(num_splits), kvl,
+                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                            _stream(q.device))
+    _raise("fa_decode_ex", rc)
     return out, lse
 
 

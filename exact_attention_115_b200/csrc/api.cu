@@ -379,13 +379,14 @@ size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {
   return round_up(size_t(BH) * s * d * sizeof(float), 256) + round_up(size_t(BH) * s * 4, 256);
 }
 
-int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nk,
-              int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
-              void* stream) {
+int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
+                 int Nk, int d, float scale, int dtype, int num_splits, const int* kv_len,
+                 void* workspace, size_t ws_bytes, void* stream) {
   int st = check_common(B, H, 1, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   if (num_splits < 0) return FA_ERR_INVALID;
+  if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID;
   const void* ptrs[] = {Q, K, V, O, L};
   for (const void* p : ptrs)
     if (!p || !aligned16(p)) return FA_ERR_INVALID;
@@ -408,9 +409,18 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
   p.splits = s;
   p.keys_per_split = kps;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.H = H;
+  p.kv_len = kv_len;
   return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FA_OK
              : FA_ERR_CUDA;
+}
+
+int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nk,
+              int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
+              void* stream) {
+  return fa_decode_ex(Q, K, V, O, L, B, H, Nk, d, scale, dtype, num_splits, nullptr, workspace,
+                      ws_bytes, stream);
 }
 
 int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
@@ -448,6 +458,8 @@ int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, floa
   p.splits = s;
   p.keys_per_split = kps;
   p.scale_log2 = scale * 1.4426950408889634f;
+  p.H = H;
+  p.kv_len = nullptr;
   return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? FA_OK
              : FA_ERR_CUDA;

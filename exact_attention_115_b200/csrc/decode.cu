@@ -69,8 +69,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LPK, sl = lane % LPK;  // key slot in the warp, lane in the group
 
+  // this part's keys, cut at the batch element's key-padding length (a part
+  // past it is empty: L_part = -inf, weight 0 in the combine)
   const int k_begin = part * p.keys_per_split;
-  const int k_end = min(p.Nk, k_begin + p.keys_per_split);
+  const int k_end = min(keys_of(p.kv_len, bh, p.H, p.Nk), k_begin + p.keys_per_split);
 
   // q slice, pre-multiplied by scale·log2(e) so scores come out in log2 units.
   float q[8];

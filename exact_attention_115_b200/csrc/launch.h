@@ -126,6 +126,8 @@ struct DecodeParams {
   float* Lpart;  // [B*H, S] natural-log logsumexp of each part (-inf if empty)
   int BH, Nk, splits, keys_per_split;
   float scale_log2;
+  int H;
+  const int* kv_len;  // key padding (keys [0, kv_len[b]) of batch element b); null = all Nk
 };
 
 cudaError_t launch_decode(int dtype, int d, const DecodeParams& p, cudaStream_t s);

@@ -174,6 +174,18 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
               int d, float scale, int dtype, int num_splits, void* workspace, size_t ws_bytes,
               void* stream);
 
+/* fa_decode with key padding: `kv_len` is NULL or a DEVICE array of B int32
+ * lengths (4-byte aligned), and the query of batch element b attends to keys
+ * j < kv_len[b] only (clamped to [0, Nk]): a KV cache whose sequences are
+ * padded to Nk.  Parts past a length are empty and get weight 0 in the
+ * combine; a length of 0 gives O = 0 and L = -inf.  The mask acts on the
+ * scaled scores before the softmax (the FlashAttention1 post (CSDN),
+ * section "引言/动机": matmul, scale, mask, softmax).  The workspace is
+ * fa_decode's. */
+int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
+                 int Nk, int d, float scale, int dtype, int num_splits, const int* kv_len,
+                 void* workspace, size_t ws_bytes, void* stream);
+
 /* fa_decode_noalloc: the split-KV decode of fa_decode for callers that
  * cannot allocate device memory.  The pages have no counterpart for it.
  *

@@ -325,6 +325,7 @@ def decode_split_combine(q, k, v, scale: float, num_splits: int):
     return O, L
 
 
-def attention_decode(Q, K, V, scale: float):
-    """Decode forward (Nq = 1, no mask): O [B,H,1,d], L [B,H,1]."""
-    return attention_forward(Q, K, V, scale, causal=False)
+def attention_decode(Q, K, V, scale: float, kv_len=None):
+    """Decode forward (Nq = 1, no causal mask; ``kv_len`` as in
+    ``attention_forward``): O [B,H,1,d], L [B,H,1]."""
+    return attention_forward(Q, K, V, scale, causal=False, kv_len=kv_len)

@@ -199,3 +199,12 @@ def test_key_padding_pointer_checks(lib):
                          1 << 30, None) == fa.FA_ERR_INVALID
     assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_FP32, None, P,
                          None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_decode_ex_checks_the_length_pointer(lib):
+    P = 4096
+    # a misaligned key-length array is invalid (checked before any launch)
+    assert lib.fa_decode_ex(P, P, P, P, P, 1, 2, 64, 64, 0.125, fa.FA_BF16, 0, P + 2, P, 1 << 20,
+                            None) == fa.FA_ERR_INVALID
+    assert lib.fa_decode_ex(P, P, P, P, P, 1, 2, 64, 64, 0.125, fa.FA_FP32, 0, None, P, 1 << 20,
+                            None) == fa.FA_ERR_UNSUPPORTED

@@ -385,3 +385,20 @@ def test_key_padding_matches_torch_sdpa_bool_mask():
         torch.tensor(Q), torch.tensor(K), torch.tensor(V), attn_mask=mask, scale=0.3)
     O, _ = oracle.attention_forward(Q, K, V, 0.3, False, kv_len=kv_len)
     assert np.max(np.abs(O - o.numpy())) <= 1e-12
+
+
+def test_decode_key_padding_matches_sdpa():
+    rng = _rng(503)
+    B, H, Nk, d = 3, 2, 50, 8
+    Q = rng.standard_normal((B, H, 1, d))
+    K, V = rng.standard_normal((B, H, Nk, d)), rng.standard_normal((B, H, Nk, d))
+    kv_len = [50, 17, 1]
+    mask = torch.tensor(np.arange(Nk)[None, None, None, :] < np.array(kv_len)[:, None, None, None])
+    o = torch.nn.functional.scaled_dot_product_attention(
+        torch.tensor(Q), torch.tensor(K), torch.tensor(V), attn_mask=mask, scale=0.35)
+    O, L = oracle.attention_decode(Q, K, V, 0.35, kv_len=kv_len)
+    assert np.max(np.abs(O - o.numpy())) <= 1e-12
+    s = 0.35 * np.einsum("bhqd,bhkd->bhqk", Q, K)
+    for b, n in enumerate(kv_len):
+        ref = np.log(np.exp(s[b, :, :, :n]).sum(-1))
+        assert np.max(np.abs(L[b] - ref)) <= 1e-12
