@@ -242,6 +242,46 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     return dq, dk, dv
 
 
+class _Attention(torch.autograd.Function):
+    """forward() / backward() of this module as one autograd node.  Saves
+    q, k, v, O and L (not P); the backward recomputes P in the kernel."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal, scale, dropout_p, seed, offset, kv_len):
+        O, L = forward(q, k, v, causal=causal, scale=scale, dropout_p=dropout_p, seed=seed,
+                       offset=offset, kv_len=kv_len)
+        ctx.save_for_backward(q, k, v, O, L)
+        ctx.args = (causal, scale, dropout_p, seed, offset, kv_len)
+        ctx.mark_non_differentiable(L)
+        return O, L
+
+    @staticmethod
+    def backward(ctx, dO, dL):
+        q, k, v, O, L = ctx.saved_tensors
+        causal, scale, dropout_p, seed, offset, kv_len = ctx.args
+        if dO.stride(-1) != 1:
+            dO = dO.contiguous()
+        dq, dk, dv = backward(q, k, v, O, dO, L, causal=causal, scale=scale, dropout_p=dropout_p,
+                              seed=seed, offset=offset, kv_len=kv_len)
+        return dq, dk, dv, None, None, None, None, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale: float | None = None, dropout_p: float = 0.0,
+              seed: int | None = None, offset: int = 0, kv_len=None):
+    """Differentiable O = attention(q, k, v) for [B, H, N, d] CUDA tensors
+    (any strides with d contiguous), through forward() and backward().  With
+    dropout and no ``seed``, one is drawn from torch's default CPU generator
+    (so torch.manual_seed makes runs repeatable); the backward reuses it.
+    Returns O only (L is kept for the backward)."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(q.shape[-1])
+    if dropout_p > 0 and seed is None:
+        seed = int(torch.randint(0, 2**62, (1,)).item())
+    O, _ = _Attention.apply(q, k, v, bool(causal), float(scale), float(dropout_p),
+                            0 if seed is None else int(seed), int(offset), kv_len)
+    return O
+
+
 def decode_workspace_bytes(B, H, Nk, d, num_splits=0) -> int:
     return int(lib().fa_decode_workspace_bytes(B, H, Nk, d, num_splits))
 
