@@ -1,6 +1,7 @@
 // C ABI of the attention library: argument checks, TMA descriptor set-up,
 // workspace layout and kernel launches.  No device memory is allocated here
 // and nothing synchronises except fa_status.
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -15,9 +16,9 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-int g_dq_mode = 0;  // 0 auto, 1 reduce-add, 2 partial buffers
+std::atomic<int> g_dq_mode{0};  // 0 auto, 1 reduce-add, 2 partial buffers
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_bwd_set_timing_events
-int g_last_site = 0;  // fa_last_timeout_site
+std::atomic<int> g_last_site{0};  // fa_last_timeout_site
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -108,7 +109,8 @@ size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int bwd_pad_rows(int Nq) { return int(round_up(size_t(Nq), 128)); }
 
 int effective_dq_mode(int B, int H, int Nq, int Nk, int d) {
-  if (g_dq_mode != 0) return g_dq_mode;
+  const int forced = g_dq_mode.load();
+  if (forced != 0) return forced;
   (void)B; (void)H; (void)Nq; (void)Nk; (void)d;
   return 1;  // reduce-add: measured faster (partials cost nkv× the dQ traffic)
 }
@@ -151,7 +153,8 @@ int decode_keys_per_split(int Nk, int splits) {
 cudaError_t set_smem_once(const void* kernel, int bytes) {
   static std::mutex mu;
   static int done_n[kMaxDevices] = {0};
-  static const void* done_k[kMaxDevices][64];
+  constexpr int kTracked = 128;  // more than the kernel variants of the library
+  static const void* done_k[kMaxDevices][kTracked];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -161,7 +164,7 @@ cudaError_t set_smem_once(const void* kernel, int bytes) {
     for (int i = 0; i < done_n[dev]; ++i)
       if (done_k[dev][i] == kernel) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  if (e == cudaSuccess && track && done_n[dev] < 64) done_k[dev][done_n[dev]++] = kernel;
+  if (e == cudaSuccess && track && done_n[dev] < kTracked) done_k[dev][done_n[dev]++] = kernel;
   return e;
 }
 
@@ -280,8 +283,7 @@ size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
 
 int fa_set_bwd_dq_mode(int mode) {
   if (mode < 0 || mode > 2) return FA_ERR_INVALID;
-  const int prev = g_dq_mode;
-  g_dq_mode = mode;
+  const int prev = g_dq_mode.exchange(mode);
   return prev;
 }
 
@@ -488,7 +490,7 @@ int fa_bwd_set_timing_events(void* start, void* stop) {
   return FA_OK;
 }
 
-int fa_last_timeout_site(void) { return g_last_site; }
+int fa_last_timeout_site(void) { return g_last_site.load(); }
 
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID;
