@@ -2,7 +2,7 @@
 j < kv_len[b]) in fa_fwd_ex / fa_bwd_ex against the fp64 oracle.
 
 Lengths cover the full length, a single key, tile edges ± 1, lengths past
-Nk (clamped) and zero (every row of that batch element sees no key:
+Nk and below zero (clamped to [0, Nk]) and zero (every row of that batch element sees no key:
 O = 0, L = -inf, zero gradients, and every K/V block of it is a work item
 with no query steps)."""
 import math
@@ -59,7 +59,7 @@ def _check(fa, q, k, v, do, kv_len, causal, what, dropout=None, layout=None):
 @pytest.mark.parametrize("causal", [False, True])
 def test_key_padding(fa, d, causal):
     N = 300
-    kv_len = [N, 1, 129, 0, 127, 1000]
+    kv_len = [N, 1, 129, 0, 127, 1000, -5]  # past Nk and negative: clamped
     q, k, v, do = W.make_tensors(len(kv_len), 2, N, N, d, "bf16", seed=31 + d, device="cuda")
     _check(fa, q, k, v, do, kv_len, causal, f"kv_len d{d} causal={causal}")
 
