@@ -144,7 +144,10 @@ def test_dropout_backward_matches_torch_autograd(causal):
                             for h in range(H)]) for b in range(B)])
     O, L = oracle.attention_forward(Q, K, V, scale, causal, dropout=(p, seed, off))
     dQ, dK, dV, D = oracle.attention_backward(Q, K, V, dO, scale, causal, dropout=(p, seed, off))
-    tO, tq, tk, tv = _torch_dropout_attention(Q, K, V, dO, scale, causal, Z, philox.keep_scale(p))
+    # the factor written out, independent of the oracle: p = 0.3 keeps a
+    # weight iff its byte is below T = round(0.7 · 256) = 179, scaled by 256/179
+    assert philox.dropout_threshold(p) == 179
+    tO, tq, tk, tv = _torch_dropout_attention(Q, K, V, dO, scale, causal, Z, 256 / 179)
     assert np.max(np.abs(O - tO)) <= 1e-12
     for got, want in ((dQ, tq), (dK, tk), (dV, tv)):
         assert np.max(np.abs(got - want)) <= 1e-10
