@@ -325,14 +325,13 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   std::memset(&a, 0, sizeof(a));
   const int bm = bwd_block_rows(d);
   // (the fp32 path stages its operands without TMA)
-  bool m4[6] = {false, false, false, false, false, false};
+  // (dK and dV are written with plain stores: their strides go to the kernel)
+  bool m4[5] = {false, false, false, false, false};
   if (dtype != FA_FP32 &&
       (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, bm, &m4[0]) ||
        !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
        !make_map(&a.tmV, V, dtype, d, Nk, H, B, *lv, 128, &m4[2]) ||
-       !make_map(&a.tmdO, dO, dtype, d, Nq, H, B, *ldo, bm, &m4[4]) ||
-       !make_map(&a.tmdK, dK, dtype, d, Nk, H, B, *ldk, 128, &m4[3]) ||
-       !make_map(&a.tmdV, dV, dtype, d, Nk, H, B, *ldv, 128, &m4[5])))
+       !make_map(&a.tmdO, dO, dtype, d, Nq, H, B, *ldo, bm, &m4[4])))
     return FA_ERR_CUDA;
   BwdParams& p = a.params;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.dO = dO; p.L = L;
@@ -354,7 +353,25 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   p.s_dq = to_strides(ldq);
   p.s_dk = to_strides(ldk);
   p.s_dv = to_strides(ldv);
-  for (int i = 0; i < 6; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dK 3, dO 4, dV 5
+  for (int i = 0; i < 5; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dO 4
+  if (dtype != FA_FP32 && d == 64) {
+    // The d = 64 kernel reduces each step's dQ tile into the fp32 accumulator
+    // (or stores it into its K/V block's partial) through a 2-D map over it:
+    // [rows, 64] fp32, boxes of 32 columns (128 bytes, 128-byte swizzle) by
+    // 128 rows.
+    const uint64_t rows = uint64_t(BH) * p.Nq_pad * (mode == 2 ? uint64_t(p.n_kblocks) : 1u);
+    if (rows > uint64_t(INT32_MAX)) return FA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
+    EncodeTiledFn enc = encode_fn();
+    cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};
+    cuuint64_t strides[1] = {cuuint64_t(d) * sizeof(float)};
+    cuuint32_t box[2] = {32, 128};
+    cuuint32_t estr[2] = {1, 1};
+    if (!enc || enc(&a.tmdQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.dQacc, dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return FA_ERR_CUDA;
+  }
   p.drop = drop;
   p.kv_len = kv_len;
   a.stream = static_cast<cudaStream_t>(stream);

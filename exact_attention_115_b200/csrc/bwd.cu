@@ -198,7 +198,7 @@ template <typename T, int D, bool CAUSAL, bool GEN, bool DROP>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
-                    const __grid_constant__ CUtensorMap tmdK, const __grid_constant__ CUtensorMap tmdV,
+                    const __grid_constant__ CUtensorMap tmdQ,
                     BwdParams p) {
   using Tr = BwdTraits<T, D>;
   constexpr int BM = Tr::BM;
@@ -271,8 +271,7 @@ __global__ void __launch_bounds__(512, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
-    tma_prefetch_desc(&tmdK);
-    tma_prefetch_desc(&tmdV);
+    if constexpr (!Tr::DQ_T) tma_prefetch_desc(&tmdQ);
   }
   tc_fence_before();
   __syncthreads();
@@ -291,7 +290,7 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sQ = smem + Tr::OFF_Q;
   uint8_t* sdO = smem + Tr::OFF_DO;
   uint8_t* sdS = smem + Tr::OFF_DS;
-  float* sdQ = reinterpret_cast<float*>(smem + Tr::OFF_DQ);
+  uint8_t* sdQ = smem + Tr::OFF_DQ;  // d = 64: two [128 rows × 128 B] swizzled halves
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
 
   // Register split (the CTA launches with 128 per thread): the compute and
@@ -761,27 +760,35 @@ __global__ void __launch_bounds__(512, 1)
           // The previous bulk operation must have finished reading the staging buffer.
           if (leader) bulk_wait_read0();
           named_bar(1, 128);
-          // write the row's D values, rotating the 16-byte chunk order by lane
-          // to spread shared-memory banks
+          // The row's 64 values go to two 128-byte-swizzled halves (columns
+          // 0-31, 32-63): 16-byte chunk j of row r at chunk position
+          // j ^ (r % 8), the tensor map's 128-byte swizzle.  Static register
+          // indices, and the 8 rows of a store phase hit 8 different chunks.
 #pragma unroll
-          for (int cc = 0; cc < D / 4; ++cc) {
-            const int c4 = (cc + lane) % (D / 4);
-            float4 x;
-            x.x = __uint_as_float(v[c4 * 4 + 0]);
-            x.y = __uint_as_float(v[c4 * 4 + 1]);
-            x.z = __uint_as_float(v[c4 * 4 + 2]);
-            x.w = __uint_as_float(v[c4 * 4 + 3]);
-            *reinterpret_cast<float4*>(sdQ + r * D + c4 * 4) = x;
+          for (int h = 0; h < 2; ++h) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int c = 32 * h + 4 * j;
+              float4 x;
+              x.x = __uint_as_float(v[c + 0]);
+              x.y = __uint_as_float(v[c + 1]);
+              x.z = __uint_as_float(v[c + 2]);
+              x.w = __uint_as_float(v[c + 3]);
+              *reinterpret_cast<float4*>(sdQ + h * (BM * 128) + r * 128 + ((j ^ (r & 7)) << 4)) = x;
+            }
           }
           fence_async_smem();
           named_bar(1, 128);
           if (leader) {
+            // rows of the accumulator viewed as [rows, 64] fp32 (x = column, y = row)
             if (p.dq_mode == 2) {
-              float* dst = p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D;
-              bulk_store(dst, sdQ, Tr::DQ_STAGE);
+              const int row = (kb * p.B * p.H + bh) * p.Nq_pad + q0;
+              tma_store_2d(&tmdQ, sdQ, 0, row);
+              tma_store_2d(&tmdQ, sdQ + BM * 128, 32, row);
             } else {
-              float* dst = p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D;
-              bulk_reduce_add_f32(dst, sdQ, Tr::DQ_STAGE);
+              const int row = bh * p.Nq_pad + q0;
+              tma_reduce_add_2d(&tmdQ, sdQ, 0, row);
+              tma_reduce_add_2d(&tmdQ, sdQ + BM * 128, 32, row);
             }
             bulk_commit();
           }
@@ -1074,8 +1081,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   }
   // persistent: one CTA per SM (or per work item, if fewer)
   const int grid = std::min(p.n_kblocks * BH, sm_count());
-  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdK,
-                                                        a.tmdV, p);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdQ, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.ev_stop) {

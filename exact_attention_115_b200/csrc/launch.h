@@ -83,14 +83,14 @@ struct BwdParams {
   int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials
   int head_group;     // heads per launch-order group (see head_group_for)
   Strides s_o, s_do, s_dq, s_dk, s_dv;  // plain (non-TMA) accesses; Q, K, V, dO go through tensor maps
-  int map4d;  // bit per tensor map (Q 0, K 1, V 2, dK 3, dO 4, dV 5): 4-D (d, N, H, B), else 3-D (d, N, B·H)
+  int map4d;  // bit per tensor map (Q 0, K 1, V 2, dO 4): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
   const int* kv_len;  // key padding, as in FwdParams
 };
 
 struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmdO;
-  CUtensorMap tmdK, tmdV;  // outputs, written by TMA stores
+  CUtensorMap tmdQ;  // d = 64: the fp32 dQ accumulator as a [rows, 64] tensor (tensor reduce-add)
   BwdParams params;
   cudaStream_t stream;
   cudaEvent_t ev_start, ev_stop;  // optional timing events around the main kernel
