@@ -43,6 +43,11 @@ Readings where the pages are silent (each also listed in the design notes):
   51CTO notes' background list names custom masks as a reason to write
   one's own kernel.  Which masks is not fixed; this one is the padding of
   batched sequences of different lengths.
+* additive bias (``bias``): the 51CTO background list names adding a bias as
+  the first modification one writes one's own kernel for.  Reading: a
+  constant added to the scaled scores, S' = scale·Q Kᵀ + bias (natural-log
+  units, -inf allowed), before the masks and the softmax; L is the
+  logsumexp of S'.  The bias gets no gradient (it is an input constant).
 
 Everything is float64.  Inputs are whatever the caller passes (normally the
 storage-dtype values the GPU sees, upcast exactly).  Rows are processed in
@@ -109,13 +114,15 @@ def tiled_softmax_then_matmul(s_row, V) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Forward: the plain definition, per (batch, head), rows in chunks.
 # --------------------------------------------------------------------------
-def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None, nk_valid=None):
+def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None, nk_valid=None,
+               bias=None):
     """P (softmax rows) and L for the given query rows of one head.
 
     q: [r, d] the query rows, k: [Nk, d].  ``rows`` are the absolute indices
     of those query rows (needed for the causal mask) and ``nq_total`` the
     head's full query length; keys j >= ``nk_valid`` are masked (key
-    padding).  Returns (P [r, Nk], L [r]).
+    padding); ``bias`` [r, Nk] is added to the scaled scores of these rows.
+    Returns (P [r, Nk], L [r]).
     """
     q = _f64(q)
     k = _f64(k)
@@ -126,6 +133,8 @@ def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None, nk_va
     if nq_total is None:
         nq_total = r
     s = scale * (q @ k.T)
+    if bias is not None:
+        s = s + _f64(bias)
     if causal:
         s = np.where(causal_visible(nq_total, nk, rows), s, -np.inf)
     if nk_valid is not None:
@@ -142,7 +151,7 @@ def head_probs(q, k, scale: float, causal: bool, rows=None, nq_total=None, nk_va
 
 
 def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None, keep_fn=None,
-                 kscale: float = 1.0, nk_valid=None):
+                 kscale: float = 1.0, nk_valid=None, bias=None):
     """O [r, d] and L [r] for query rows of one head (see ``head_probs``).
 
     With dropout, ``keep_fn(rows, cols)`` gives the boolean keep mask at
@@ -161,7 +170,8 @@ def head_forward(q, k, v, scale: float, causal: bool, rows=None, nq_total=None, 
     L = np.empty(r)
     for c0 in range(0, r, _ROW_CHUNK):
         c1 = min(r, c0 + _ROW_CHUNK)
-        p, l = head_probs(q[c0:c1], k, scale, causal, rows[c0:c1], nq_total, nk_valid)
+        p, l = head_probs(q[c0:c1], k, scale, causal, rows[c0:c1], nq_total, nk_valid,
+                          None if bias is None else bias[c0:c1])
         if keep_fn is not None:
             p = p * keep_fn(rows[c0:c1], np.arange(k.shape[0])) * kscale
         O[c0:c1] = p @ v
@@ -179,13 +189,17 @@ def _dropout_fn(dropout, bh):
     return (lambda r, c: philox.keep_mask(bh, r, c, p, seed, offset)), philox.keep_scale(p)
 
 
-def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None, kv_len=None):
+def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None, kv_len=None,
+                      bias=None):
     """O [B,H,Nq,d] and L [B,H,Nq] (float64) for [B,H,N,d] inputs.
     ``dropout`` = (p, seed, offset) applies the Philox keep mask of
     ``oracle/philox.py`` to head index b·H + h; ``kv_len`` (B integers)
-    hides keys j >= kv_len[b] of batch element b."""
+    hides keys j >= kv_len[b] of batch element b; ``bias`` (broadcastable to
+    [B, H, Nq, Nk]) is added to the scaled scores."""
     Q, K, V = _f64(Q), _f64(K), _f64(V)
     B, H, Nq, d = Q.shape
+    if bias is not None:
+        bias = np.broadcast_to(_f64(bias), (B, H, Nq, K.shape[2]))
     O = np.empty((B, H, Nq, V.shape[3]))
     L = np.empty((B, H, Nq))
     for b in range(B):
@@ -193,7 +207,8 @@ def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None,
             fn, ks = _dropout_fn(dropout, b * H + h)
             O[b, h], L[b, h] = head_forward(Q[b, h], K[b, h], V[b, h], scale, causal,
                                             keep_fn=fn, kscale=ks,
-                                            nk_valid=None if kv_len is None else int(kv_len[b]))
+                                            nk_valid=None if kv_len is None else int(kv_len[b]),
+                                            bias=None if bias is None else bias[b, h])
     return O, L
 
 
@@ -201,7 +216,7 @@ def attention_forward(Q, K, V, scale: float, causal: bool = False, dropout=None,
 # Backward: the exact gradient of O = softmax(scale Q Kᵀ [masked]) V.
 # --------------------------------------------------------------------------
 def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale: float = 1.0,
-                  nk_valid=None):
+                  nk_valid=None, bias=None):
     """dQ, dK, dV, D for one head (all query rows), float64.
 
     D_i = Σ_c dO_ic O_ic; dP = dO Vᵀ; dS = P ∘ (dP − D); dV = Pᵀ dO;
@@ -218,7 +233,8 @@ def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale:
     rows_all = np.arange(nq)
     for c0 in range(0, nq, _ROW_CHUNK):
         c1 = min(nq, c0 + _ROW_CHUNK)
-        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq, nk_valid)
+        p, _ = head_probs(q[c0:c1], k, scale, causal, rows_all[c0:c1], nq, nk_valid,
+                          None if bias is None else bias[c0:c1])
         z = 1.0 if keep_fn is None else keep_fn(rows_all[c0:c1], np.arange(k.shape[0])) * kscale
         pz = p * z
         o = pz @ v
@@ -233,11 +249,14 @@ def head_backward(q, k, v, do, scale: float, causal: bool, keep_fn=None, kscale:
 
 
 def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=None,
-                       kv_len=None):
+                       kv_len=None, bias=None):
     """dQ, dK, dV ([B,H,N,d]) and D ([B,H,Nq]) in float64 (``dropout`` and
-    ``kv_len`` as in ``attention_forward``)."""
+    ``kv_len`` and ``bias`` as in ``attention_forward``; no gradient for
+    the bias)."""
     Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
     B, H = Q.shape[:2]
+    if bias is not None:
+        bias = np.broadcast_to(_f64(bias), (B, H, Q.shape[2], K.shape[2]))
     dQ = np.empty_like(Q)
     dK = np.empty_like(K)
     dV = np.empty_like(V)
@@ -247,7 +266,8 @@ def attention_backward(Q, K, V, dO, scale: float, causal: bool = False, dropout=
             fn, ks = _dropout_fn(dropout, b * H + h)
             dQ[b, h], dK[b, h], dV[b, h], D[b, h] = head_backward(
                 Q[b, h], K[b, h], V[b, h], dO[b, h], scale, causal, keep_fn=fn, kscale=ks,
-                nk_valid=None if kv_len is None else int(kv_len[b]))
+                nk_valid=None if kv_len is None else int(kv_len[b]),
+                bias=None if bias is None else bias[b, h])
     return dQ, dK, dV, D
 
 

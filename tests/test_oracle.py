@@ -402,3 +402,42 @@ def test_decode_key_padding_matches_sdpa():
     for b, n in enumerate(kv_len):
         ref = np.log(np.exp(s[b, :, :, :n]).sum(-1))
         assert np.max(np.abs(L[b] - ref)) <= 1e-12
+
+
+# --------------------------------------------------------------------------
+# Additive bias: pinned by torch SDPA with the same float mask.
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_bias_matches_torch_autograd(causal):
+    rng = _rng(504)
+    B, H, Nq, Nk, d = 2, 3, 9, 13, 4
+    Q, dO = rng.standard_normal((B, H, Nq, d)), rng.standard_normal((B, H, Nq, d))
+    K, V = rng.standard_normal((B, H, Nk, d)), rng.standard_normal((B, H, Nk, d))
+    bias = rng.standard_normal((1, H, Nq, Nk))  # broadcast over the batch
+    bias[0, 1, 2, :5] = -np.inf                 # some hidden keys
+    O, L = oracle.attention_forward(Q, K, V, 0.6, causal, bias=bias)
+    dQ, dK, dV, _ = oracle.attention_backward(Q, K, V, dO, 0.6, causal, bias=bias)
+    m = np.broadcast_to(bias, (B, H, Nq, Nk)).copy()
+    if causal:
+        vis = np.arange(Nk)[None, :] <= np.arange(Nq)[:, None] + (Nk - Nq)
+        m = np.where(vis, m, -np.inf)
+    q, k, v = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+    o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.tensor(m), scale=0.6)
+    o.backward(torch.tensor(dO))
+    assert np.max(np.abs(O - o.detach().numpy())) <= 1e-12
+    for got, want in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        assert np.max(np.abs(got - want.numpy())) <= 1e-11
+    s = 0.6 * np.einsum("bhqd,bhkd->bhqk", Q, K) + m
+    ref_L = np.log(np.exp(s - s.max(-1, keepdims=True)).sum(-1)) + s.max(-1)
+    assert np.max(np.abs(L - ref_L)) <= 1e-12
+
+
+def test_bias_constant_per_row_changes_nothing_but_L():
+    """softmax is invariant to a per-row constant: O unchanged, L shifted."""
+    rng = _rng(505)
+    Q, K, V = (rng.standard_normal((1, 2, 6, 4)) for _ in range(3))
+    c = rng.standard_normal((1, 2, 6, 1))
+    O0, L0 = oracle.attention_forward(Q, K, V, 0.5, False)
+    O1, L1 = oracle.attention_forward(Q, K, V, 0.5, False, bias=np.broadcast_to(c, (1, 2, 6, 6)))
+    assert np.max(np.abs(O1 - O0)) <= 1e-12
+    assert np.max(np.abs(L1 - L0 - c[..., 0])) <= 1e-12

@@ -5,7 +5,8 @@ undone when the test ends) and checks that a pin of tests/test_oracle.py or
 tests/test_oracle_dropout.py fails on it: a dropped scale, an off-by-one in
 the causal mask, a missing -D term, dV without the transpose, the dropout
 factor forgotten, the keep-mask words and bytes swapped, a Philox round too
-few, and an off-by-one in the key-padding length.
+few, an off-by-one in the key-padding length, and a bias added before the
+scale.
 """
 import numpy as np
 import pytest
@@ -49,7 +50,7 @@ def test_causal_off_by_one_is_caught(monkeypatch):
 
 def _backward_with(mistake):
     """head_backward restated with one planted mistake."""
-    def hb(q, k, v, do, scale, causal, keep_fn=None, kscale=1.0, nk_valid=None):
+    def hb(q, k, v, do, scale, causal, keep_fn=None, kscale=1.0, nk_valid=None, bias=None):
         q, k, v, do = (np.asarray(x, dtype=np.float64) for x in (q, k, v, do))
         p, _ = att.head_probs(q, k, scale, causal, None, None, nk_valid)
         o = p @ v
@@ -110,7 +111,20 @@ def test_missing_philox_round_is_caught(monkeypatch):
 def test_key_padding_off_by_one_is_caught(monkeypatch):
     orig = att.head_probs
 
-    def plus_one(q, k, scale, causal, rows=None, nq_total=None, nk_valid=None):
-        return orig(q, k, scale, causal, rows, nq_total, None if nk_valid is None else nk_valid + 1)
+    def plus_one(q, k, scale, causal, rows=None, nq_total=None, nk_valid=None, bias=None):
+        return orig(q, k, scale, causal, rows, nq_total, None if nk_valid is None else nk_valid + 1,
+                    bias)
     monkeypatch.setattr(att, "head_probs", plus_one)
     _fails(pins.test_key_padding_matches_torch_autograd, True)
+
+
+def test_bias_before_scale_is_caught(monkeypatch):
+    """The bias belongs to the scaled scores; adding it before the scale (so
+    that it gets scaled too) must fail the SDPA pin."""
+    orig = att.head_probs
+
+    def scaled_bias(q, k, scale, causal, rows=None, nq_total=None, nk_valid=None, bias=None):
+        return orig(q, k, scale, causal, rows, nq_total, nk_valid,
+                    None if bias is None else np.asarray(bias) * scale)
+    monkeypatch.setattr(att, "head_probs", scaled_bias)
+    _fails(pins.test_bias_matches_torch_autograd, False)
