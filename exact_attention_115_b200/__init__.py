@@ -34,9 +34,9 @@ SIGNATURES = {
     "fa_bwd_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I, _I]),
     "fa_bwd": (_I, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I, _F, _I,
                     _VP, _SZ, _VP]),
-    "fa_fwd_ex": (_I, [_VP] * 9 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP]),
-    "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _SZ,
-                                               _VP]),
+    "fa_fwd_ex": (_I, [_VP] * 9 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP, _VP]),
+    "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP,
+                                               _VP, _SZ, _VP]),
     "fa_set_bwd_dq_mode": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
@@ -113,6 +113,21 @@ def _kv_len_ptr(kv_len, B, device):
     return kv_len.data_ptr()
 
 
+def _bias_args(bias, q, B, H, Nq, Nk):
+    """(pointer, Layout) of an additive bias broadcastable to [B, H, Nq, Nk]
+    (input dtype, key columns contiguous), or (None, None)."""
+    if bias is None:
+        return None, None
+    if not isinstance(bias, torch.Tensor) or bias.dtype != q.dtype or bias.device != q.device:
+        raise TypeError("bias must be a tensor of the inputs' dtype on their device")
+    if bias.dim() != 4:
+        raise ValueError("bias must be 4-D, broadcastable to [B, H, Nq, Nk]")
+    b = bias.expand(B, H, Nq, Nk)  # broadcast dimensions get stride 0
+    if b.stride(3) != 1:
+        raise ValueError("bias must have contiguous key columns")
+    return b.data_ptr(), Layout(b.stride(0), b.stride(1), b.stride(2))
+
+
 def _layout(t) -> Layout:
     s = t.stride()
     return Layout(s[0], s[1], s[2])
@@ -146,13 +161,15 @@ def _raise(fn, code):
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, kv_len=None):
+            dropout_p: float = 0.0, seed: int = 0, offset: int = 0, kv_len=None, bias=None):
     """O, L = attention(q, k, v).  q, k, v (and out) are [B, H, N, d] with any
     strides whose d dimension is contiguous (a [B, N, H, d] tensor viewed
     with .transpose(1, 2) works as is).  ``dropout_p`` > 0 drops attention
     weights with the keep mask that ``seed`` and ``offset`` select (pass the
     same three to ``backward``).  ``kv_len`` (int32 [B] on the device) hides
-    keys j >= kv_len[b] of batch element b.  Returns (O [B,H,Nq,d] q.dtype,
+    keys j >= kv_len[b] of batch element b; ``bias`` (broadcastable to
+    [B, H, Nq, Nk], q's dtype) is added to the scaled scores.  Returns
+    (O [B,H,Nq,d] q.dtype,
     L [B,H,Nq] fp32 contiguous)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
@@ -169,7 +186,8 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     _check("lse", lse, (B, H, Nq), torch.float32)
     dr = _dropout(dropout_p, seed, offset)
     kvl = _kv_len_ptr(kv_len, B, q.device)
-    if dr is None and kvl is None and all(t.is_contiguous() for t in (q, k, v, out)):
+    bp, bl = _bias_args(bias, q, B, H, Nq, Nk)
+    if dr is None and kvl is None and bp is None and all(t.is_contiguous() for t in (q, k, v, out)):
         rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
                           lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
                           _dtype_code(q), _stream(q.device))
@@ -179,7 +197,8 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
                          ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
                          B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                         None if dr is None else ctypes.byref(dr), kvl, _stream(q.device))
+                         None if dr is None else ctypes.byref(dr), kvl, bp,
+                         None if bl is None else ctypes.byref(bl), _stream(q.device))
     _raise("fa_fwd_ex", rc)
     return out, lse
 
@@ -199,9 +218,10 @@ def set_bwd_dq_mode(mode: int) -> int:
 
 def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = None,
              dq=None, dk=None, dv=None, workspace=None, dropout_p: float = 0.0, seed: int = 0,
-             offset: int = 0, kv_len=None):
+             offset: int = 0, kv_len=None, bias=None):
     """dQ, dK, dV of attention given the forward's O and L and the upstream dO
-    (and the forward's ``dropout_p``, ``seed``, ``offset`` and ``kv_len``)."""
+    (and the forward's ``dropout_p``, ``seed``, ``offset``, ``kv_len`` and
+    ``bias``; the bias gets no gradient)."""
     _check("q", q, strided=True)
     B, H, Nq, d = q.shape
     Nk = k.shape[2]
@@ -223,7 +243,8 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     ts = (q, k, v, o, do, dq, dk, dv)
     dr = _dropout(dropout_p, seed, offset)
     kvl = _kv_len_ptr(kv_len, B, dev)
-    if dr is None and kvl is None and all(t.is_contiguous() for t in ts):
+    bp, bl = _bias_args(bias, q, B, H, Nq, Nk)
+    if dr is None and kvl is None and bp is None and all(t.is_contiguous() for t in ts):
         rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
                           lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                           B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
@@ -236,7 +257,7 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
                          *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d, int(bool(causal)),
                          float(scale), _dtype_code(q), None if dr is None else ctypes.byref(dr),
-                         kvl, workspace.data_ptr(), workspace.numel() * workspace.element_size(),
+                         kvl, bp, None if bl is None else ctypes.byref(bl), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
                          _stream(dev))
     _raise("fa_bwd_ex", rc)
     return dq, dk, dv
@@ -247,27 +268,27 @@ class _Attention(torch.autograd.Function):
     q, k, v, O and L (not P); the backward recomputes P in the kernel."""
 
     @staticmethod
-    def forward(ctx, q, k, v, causal, scale, dropout_p, seed, offset, kv_len):
+    def forward(ctx, q, k, v, causal, scale, dropout_p, seed, offset, kv_len, bias):
         O, L = forward(q, k, v, causal=causal, scale=scale, dropout_p=dropout_p, seed=seed,
-                       offset=offset, kv_len=kv_len)
+                       offset=offset, kv_len=kv_len, bias=bias)
         ctx.save_for_backward(q, k, v, O, L)
-        ctx.args = (causal, scale, dropout_p, seed, offset, kv_len)
+        ctx.args = (causal, scale, dropout_p, seed, offset, kv_len, bias)
         ctx.mark_non_differentiable(L)
         return O, L
 
     @staticmethod
     def backward(ctx, dO, dL):
         q, k, v, O, L = ctx.saved_tensors
-        causal, scale, dropout_p, seed, offset, kv_len = ctx.args
+        causal, scale, dropout_p, seed, offset, kv_len, bias = ctx.args
         if dO.stride(-1) != 1:
             dO = dO.contiguous()
         dq, dk, dv = backward(q, k, v, O, dO, L, causal=causal, scale=scale, dropout_p=dropout_p,
-                              seed=seed, offset=offset, kv_len=kv_len)
-        return dq, dk, dv, None, None, None, None, None, None
+                              seed=seed, offset=offset, kv_len=kv_len, bias=bias)
+        return dq, dk, dv, None, None, None, None, None, None, None
 
 
 def attention(q, k, v, causal: bool = False, scale: float | None = None, dropout_p: float = 0.0,
-              seed: int | None = None, offset: int = 0, kv_len=None):
+              seed: int | None = None, offset: int = 0, kv_len=None, bias=None):
     """Differentiable O = attention(q, k, v) for [B, H, N, d] CUDA tensors
     (any strides with d contiguous), through forward() and backward().  With
     dropout and no ``seed``, one is drawn from torch's default CPU generator
@@ -278,7 +299,7 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, dropout
     if dropout_p > 0 and seed is None:
         seed = int(torch.randint(0, 2**62, (1,)).item())
     O, _ = _Attention.apply(q, k, v, bool(causal), float(scale), float(dropout_p),
-                            0 if seed is None else int(seed), int(offset), kv_len)
+                            0 if seed is None else int(seed), int(offset), kv_len, bias)
     return O
 
 

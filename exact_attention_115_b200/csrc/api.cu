@@ -218,7 +218,7 @@ extern "C" {
 int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              const int* kv_len, void* stream) {
+              const int* kv_len, const void* bias, const fa_layout* lbias, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
@@ -240,11 +240,18 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID;
   if (kv_len && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (bias && (!aligned16(bias) || !valid_layout(lbias, dtype))) return FA_ERR_INVALID;
+  if (bias && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int BH = B * H;
   FwdLaunch a;
   std::memset(&a, 0, sizeof(a));
   a.params.drop = drop;
   a.params.kv_len = kv_len;
+  if (bias) {
+    a.params.bias = bias;
+    a.params.s_bias = Strides{lbias->b, lbias->h, lbias->n};
+    a.params.bias_mul = 1.0f / scale;
+  }
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
@@ -273,7 +280,7 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
            int Nk, int d, int causal, float scale, int dtype, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
   return fa_fwd_ex(Q, K, V, O, L, &lq, &lk, &lk, &lq, B, H, Nq, Nk, d, causal, scale, dtype, nullptr,
-                   nullptr, stream);
+                   nullptr, nullptr, nullptr, stream);
 }
 
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
@@ -292,7 +299,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
               const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
               int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              const int* kv_len, void* workspace, size_t ws_bytes, void* stream) {
+              const int* kv_len, const void* bias, const fa_layout* lbias, void* workspace,
+              size_t ws_bytes, void* stream) {
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
@@ -316,6 +324,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   if (drop.t4 && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   if (kv_len && (reinterpret_cast<uintptr_t>(kv_len) & 3u)) return FA_ERR_INVALID;
   if (kv_len && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
+  if (bias && (!aligned16(bias) || !valid_layout(lbias, dtype))) return FA_ERR_INVALID;
+  if (bias && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int mode = effective_dq_mode(B, H, Nq, Nk, d);
   const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
@@ -374,6 +384,11 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   }
   p.drop = drop;
   p.kv_len = kv_len;
+  if (bias) {
+    p.bias = bias;
+    p.s_bias = Strides{lbias->b, lbias->h, lbias->n};
+    p.bias_l2 = 1.4426950408889634f;
+  }
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;
@@ -385,7 +400,8 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
            int causal, float scale, int dtype, void* workspace, size_t ws_bytes, void* stream) {
   const fa_layout lq = contiguous_layout(H, Nq, d), lk = contiguous_layout(H, Nk, d);
   return fa_bwd_ex(Q, K, V, O, dO, L, dQ, dK, dV, &lq, &lk, &lk, &lq, &lq, &lq, &lk, &lk, B, H, Nq,
-                   Nk, d, causal, scale, dtype, nullptr, nullptr, workspace, ws_bytes, stream);
+                   Nk, d, causal, scale, dtype, nullptr, nullptr, nullptr, nullptr, workspace,
+                   ws_bytes, stream);
 }
 
 size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {

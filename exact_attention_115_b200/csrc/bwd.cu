@@ -194,7 +194,8 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
 // GEN: some tensor has a general layout (4-D tensor maps or plain strided
 // accesses); otherwise every access uses the contiguous [B·H, N, d] form.
 // DROP: the forward dropped weights; the compute warps redraw its keep mask.
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP>
+// BIAS: the forward added a bias to the scaled scores; P is rebuilt with it.
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS>
 __global__ void __launch_bounds__(512, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -596,6 +597,21 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int g16 = 0; g16 < CWC / 16; ++g16) keep16_col(p.drop, bh, key, q0 + 16 * g16, keep + 4 * g16);
         }
+        // Bias: this key's values for the CWC query columns, as packed pairs
+        // (warp lanes hold consecutive keys, so each load is coalesced);
+        // zero past Nq or past Nk.
+        uint32_t bpk[BIAS ? CWC / 2 : 1];
+        if constexpr (BIAS) {
+          const uint16_t* bcol = reinterpret_cast<const uint16_t*>(p.bias) + (bh / p.H) * p.s_bias.b +
+                                 (bh % p.H) * p.s_bias.h + (key < p.Nk ? key : 0);
+#pragma unroll
+          for (int c = 0; c < CWC; c += 2) {
+            const int qa = q0 + c;
+            const uint32_t lo = (key < p.Nk && qa < p.Nq) ? __ldg(bcol + (long long)qa * p.s_bias.n) : 0u;
+            const uint32_t hi = (key < p.Nk && qa + 1 < p.Nq) ? __ldg(bcol + (long long)(qa + 1) * p.s_bias.n) : 0u;
+            bpk[c >> 1] = lo | (hi << 16);
+          }
+        }
         // ---- P = exp2(S·c − L·log2e), causal / ragged masking
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, gs & 1, abort_flag));
         tc_fence_after();
@@ -625,8 +641,12 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int q = c + e + 2 * h2;
-              const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2,
-                                          h2 ? pk2(nl.z, nl.w) : pk2(nl.x, nl.y)));
+              uint64_t nlq = h2 ? pk2(nl.z, nl.w) : pk2(nl.x, nl.y);
+              if constexpr (BIAS) {  // − L·log2e + bias·log2e
+                const float2 b2 = ElemTraits<T>::unpack2(bpk[q >> 1]);
+                nlq = ffma2(pk2(b2.x, b2.y), pk2(p.bias_l2, p.bias_l2), nlq);
+              }
+              const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2, nlq));
               float p0 = ex2(x.x), p1 = ex2(x.y);
               if (need_mask) {
                 if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
@@ -897,7 +917,9 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   const size_t row = size_t(bh) * p.Nq_pad + q;
   if (sl == 0) {
     p.neg_D[row] = q < p.Nq ? -dsum : 0.f;
-    p.neg_Lsc[row] = -lsc;
+    // a row that sees no key (L = -inf) keeps P = 0 whatever its scores and
+    // bias are, as the padding rows do
+    p.neg_Lsc[row] = lsc == -INFINITY ? -INFINITY : -lsc;
   }
   if (p.dq_mode == 1) {
     float4* z = reinterpret_cast<float4*>(p.dQacc + row * D + sl * 8);
@@ -1053,7 +1075,7 @@ static cudaError_t launch_bwd_fp32(const BwdLaunch& a) {
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false>
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false>
 static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   using Tr = BwdTraits<T, D>;
   const BwdParams& p = a.params;
@@ -1062,7 +1084,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   bwd_preprocess_kernel<T, D, GEN><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  auto kern = bwd_main_kernel<T, D, CAUSAL, GEN, DROP>;
+  auto kern = bwd_main_kernel<T, D, CAUSAL, GEN, DROP, BIAS>;
   e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg.inc draws on the registers the CTA was launched with: refuse
@@ -1102,9 +1124,15 @@ cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
                    !contiguous_strides(p.s_dk, p.H, p.Nk, d) ||
                    !contiguous_strides(p.s_dv, p.H, p.Nk, d);
   const bool drop = p.drop.t4 != 0;
-  // dropout runs in the general-layout variant only (one extra build per shape)
+  const bool bias = p.bias != nullptr;
+  // dropout and bias run in general-layout variants only
 #define FA_BWD_CASE(TY, DD)                                                        \
   {                                                                                \
+    if (bias)                                                                      \
+      return causal ? (drop ? launch_bwd_t<TY, DD, true, true, true, true>(a)     \
+                            : launch_bwd_t<TY, DD, true, true, false, true>(a))   \
+                    : (drop ? launch_bwd_t<TY, DD, false, true, true, true>(a)    \
+                            : launch_bwd_t<TY, DD, false, true, false, true>(a)); \
     if (drop)                                                                      \
       return causal ? launch_bwd_t<TY, DD, true, true, true>(a)                    \
                     : launch_bwd_t<TY, DD, false, true, true>(a);                  \

@@ -193,7 +193,8 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 // GEN: some tensor map is 4-D (a layout whose heads and batches do not merge
 // into one index); otherwise every map is the 3-D (d, N, B·H) form.
 // DROP: dropout on P (16-bit types only), masks drawn in the softmax warps.
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP>
+// BIAS: an additive bias on the scaled scores (16-bit types only).
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS>
 __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -469,7 +470,23 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
     float row_sum_p = 0.f;  // Σ of P as rounded for the P·V product: normalises O
     bool ok = true;
 
+    // bias row of this thread's query (batch b = bh / H, head h = bh % H)
+    const uint16_t* brow = nullptr;
+    if constexpr (BIAS && !TF32)
+      if (qi < p.Nq)
+        brow = reinterpret_cast<const uint16_t*>(p.bias) + (bh / p.H) * p.s_bias.b +
+               (bh % p.H) * p.s_bias.h + (long long)qi * p.s_bias.n;
     for (int j = 0; j < n_kv; ++j) {
+      // Bias: this row's values for the tile's columns, loaded before S
+      // arrives so the loads overlap the wait (zero past Nk or past Nq).
+      uint4 bv[(BIAS && !TF32) ? Tr::BN / 8 : 1];
+      if constexpr (BIAS && !TF32) {
+#pragma unroll
+        for (int v = 0; v < Tr::BN / 8; ++v) {
+          const int col = j * Tr::BN + 8 * v;
+          bv[v] = brow ? load8_16bit(brow + col, p.Nk - col) : make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
@@ -477,11 +494,30 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       const bool tr = trace_on && quad == 0 && lane == 0;
       trace_ev(tr, 1000 + 100 * t + j);
 #endif
-      // All four 32-column loads in flight, one wait.
       uint32_t su[4][32];
+      if constexpr (BIAS && !TF32) {
+        // 32 columns at a time, each plus its bias / scale (so the bias
+        // registers free up as the scores arrive)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, su[q]);
-      tmem_ld_wait();
+        for (int q = 0; q < 4; ++q) {
+          tmem_ld32(tS + 32 * q, su[q]);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int c = 32 * q + e;
+            const uint32_t w = (c & 7) < 2 ? bv[c >> 3].x : (c & 7) < 4 ? bv[c >> 3].y
+                             : (c & 7) < 6 ? bv[c >> 3].z : bv[c >> 3].w;
+            const float2 b2 = ElemTraits<T>::unpack2(w);
+            su[q][e] = __float_as_uint(fmaf(b2.x, p.bias_mul, __uint_as_float(su[q][e])));
+            su[q][e + 1] = __float_as_uint(fmaf(b2.y, p.bias_mul, __uint_as_float(su[q][e + 1])));
+          }
+        }
+      } else {
+        // All four 32-column loads in flight, one wait.
+#pragma unroll
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, su[q]);
+        tmem_ld_wait();
+      }
       float* s = reinterpret_cast<float*>(&su[0][0]);
       const int k0 = j * Tr::BN;
       const bool tail = k0 + Tr::BN > nk;
@@ -673,10 +709,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false>
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false>
 static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   using Tr = FwdTraits<T, D>;
-  auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP>;
+  auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP, BIAS>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg redistributes the registers the CTA was launched with; refuse
@@ -701,9 +737,15 @@ int fwd_rows_per_cta(int dtype, int d) { return 128 * fwd_tiles(dtype == FA_FP32
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
   const bool gen = a.params.map4d != 0;  // only 4-D tensor maps differ: every access is TMA
   const bool drop = a.params.drop.t4 != 0;
-  // dropout runs in the general-layout variant only (one extra build per shape)
+  const bool bias = a.params.bias != nullptr;
+  // dropout and bias run in general-layout variants only
 #define FA_FWD_CASE(TY, DD)                                                                      \
   {                                                                                              \
+    if (bias)                                                                                    \
+      return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true>(a)                   \
+                            : launch_fwd_t<TY, DD, true, true, false, true>(a))                 \
+                    : (drop ? launch_fwd_t<TY, DD, false, true, true, true>(a)                  \
+                            : launch_fwd_t<TY, DD, false, true, false, true>(a));               \
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \

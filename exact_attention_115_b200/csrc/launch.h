@@ -47,6 +47,9 @@ struct FwdParams {
   int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
   const int* kv_len;  // key padding: keys of batch element b are [0, kv_len[b]); null = all Nk
+  const void* bias;   // additive bias on the scaled scores, [B', H', Nq, Nk] input dtype; null = none
+  Strides s_bias;     // its element strides (0 broadcasts a batch or head; columns contiguous)
+  float bias_mul;     // 1 / scale: the bias in units of the unscaled scores
 };
 
 struct FwdLaunch {
@@ -86,6 +89,9 @@ struct BwdParams {
   int map4d;  // bit per tensor map (Q 0, K 1, V 2, dO 4): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
   const int* kv_len;  // key padding, as in FwdParams
+  const void* bias;   // additive bias, as in FwdParams
+  Strides s_bias;
+  float bias_l2;      // log2(e): the bias in the backward's log2 units
 };
 
 struct BwdLaunch {

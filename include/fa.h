@@ -100,7 +100,20 @@ typedef struct {
   unsigned int offset;     /* counter word 3: a separate stream per call */
 } fa_dropout;
 
-/* Key padding (`kv_len`, for fa_fwd_ex and fa_bwd_ex): NULL, or a DEVICE
+/* Additive bias (`bias`, `lbias`, for fa_fwd_ex and fa_bwd_ex): NULL, or a
+ * device tensor of the input dtype viewed as [B, H, Nq, Nk] through the
+ * element strides in `lbias` {b, h, n} (row = query; key columns contiguous;
+ * a stride of 0 broadcasts over batches or heads).  It is added to the
+ * scaled scores before the masks and the softmax, S' = scale·Q Kᵀ + bias,
+ * in natural-log units (-inf hides a key), and L is the logsumexp of S'.
+ * The 51CTO notes' background list names adding a bias as the first change
+ * one writes one's own kernel for.  The bias is an input constant: the
+ * backward rebuilds P with it and returns no gradient for it.  The pointer
+ * must be 16-byte aligned and each stride a non-negative multiple of 16
+ * bytes (rows padded to a multiple of 8 keys), else FA_ERR_INVALID; fp32 has
+ * no bias (FA_ERR_UNSUPPORTED).
+ *
+ * Key padding (`kv_len`, for fa_fwd_ex and fa_bwd_ex): NULL, or a DEVICE
  * array of B int32 lengths; batch element b then sees only keys
  * j < kv_len[b] (values are clamped to [0, Nk] on the device).  It is the
  * additive 0 / -inf mask of batched sequences padded to Nk, ANDed with the
@@ -122,7 +135,7 @@ typedef struct {
 int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              const int* kv_len, void* stream);
+              const int* kv_len, const void* bias, const fa_layout* lbias, void* stream);
 
 /* Bytes of device workspace fa_bwd needs for this problem (0 on invalid
  * arguments).  The workspace holds D = rowsum(dO ∘ O) [B,H,Nq] and the fp32
@@ -150,7 +163,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,
               const fa_layout* ldq, const fa_layout* ldk, const fa_layout* ldv, int B, int H,
               int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
-              const int* kv_len, void* workspace, size_t ws_bytes, void* stream);
+              const int* kv_len, const void* bias, const fa_layout* lbias, void* workspace,
+              size_t ws_bytes, void* stream);
 
 /* How fa_bwd reduces the dQ contributions of the different K/V blocks:
  *   0 = automatic (the measured faster strategy for the shape),

@@ -149,16 +149,16 @@ def test_ex_entry_points_validate_layouts(lib):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     assert lib.fa_fwd_ex(P, P, P, P, P, r(bad), r(good), r(good), r(good), *args, fa.FA_BF16,
-                         None, None, None) == fa.FA_ERR_INVALID
+                         None, None, None, None, None) == fa.FA_ERR_INVALID
     assert lib.fa_fwd_ex(P, P, P, P, P, None, r(good), r(good), r(good), *args, fa.FA_BF16,
-                         None, None, None) == fa.FA_ERR_INVALID
+                         None, None, None, None, None) == fa.FA_ERR_INVALID
     # fp32 reads contiguous tensors only
     nc = L(2 * 64 * 64, 64, 2 * 64)
     assert lib.fa_fwd_ex(P, P, P, P, P, r(nc), r(good), r(good), r(good), *args, fa.FA_FP32,
-                         None, None, None) == fa.FA_ERR_UNSUPPORTED
+                         None, None, None, None, None) == fa.FA_ERR_UNSUPPORTED
     lays = [r(good)] * 8
     assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, r(bad), *lays[1:], *args, fa.FA_BF16, None, None,
-                         P, 1 << 30, None) == fa.FA_ERR_INVALID
+                         None, None, P, 1 << 30, None) == fa.FA_ERR_INVALID
 
 
 @pytest.mark.parametrize("p", [-0.1, 1.0, 1.5, float("nan"), 0.999])
@@ -170,10 +170,10 @@ def test_ex_entry_points_reject_bad_dropout(lib, p):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     dr = fa.Dropout(p, 1, 0)
-    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_BF16, r(dr), None,
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_BF16, r(dr), None, None, None,
                          None) == fa.FA_ERR_INVALID
     assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *[r(good)] * 8, *args, fa.FA_BF16, r(dr), None,
-                         P, 1 << 30, None) == fa.FA_ERR_INVALID
+                         None, None, P, 1 << 30, None) == fa.FA_ERR_INVALID
 
 
 def test_fp32_has_no_dropout(lib):
@@ -182,7 +182,7 @@ def test_fp32_has_no_dropout(lib):
     args = (1, 2, 64, 64, 64, 0, 0.125)
     r = ctypes.byref
     dr = fa.Dropout(0.1, 1, 0)
-    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_FP32, r(dr), None,
+    assert lib.fa_fwd_ex(P, P, P, P, P, *[r(good)] * 4, *args, fa.FA_FP32, r(dr), None, None, None,
                          None) == fa.FA_ERR_UNSUPPORTED
 
 
@@ -193,11 +193,28 @@ def test_key_padding_pointer_checks(lib):
     r = ctypes.byref
     lays4, lays8 = [r(good)] * 4, [r(good)] * 8
     # a misaligned length array is invalid; fp32 has no key padding
-    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, P + 2,
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, P + 2, None, None,
                          None) == fa.FA_ERR_INVALID
-    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *lays8, *args, fa.FA_BF16, None, P + 2, P,
-                         1 << 30, None) == fa.FA_ERR_INVALID
-    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_FP32, None, P,
+    assert lib.fa_bwd_ex(P, P, P, P, P, P, P, P, P, *lays8, *args, fa.FA_BF16, None, P + 2, None,
+                         None, P, 1 << 30, None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_FP32, None, P, None, None,
+                         None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_bias_pointer_and_layout_checks(lib):
+    good = fa.Layout(2 * 64 * 64, 64 * 64, 64)
+    P = 4096
+    args = (1, 2, 64, 64, 64, 0, 0.125)
+    r = ctypes.byref
+    lays4 = [r(good)] * 4
+    bl_ok, bl_bad = fa.Layout(0, 64 * 64, 64), fa.Layout(0, 64 * 64, 60)  # 60 keys: not 16-byte rows
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, None, P + 8, r(bl_ok),
+                         None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, None, P, r(bl_bad),
+                         None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_BF16, None, None, P, None,
+                         None) == fa.FA_ERR_INVALID
+    assert lib.fa_fwd_ex(P, P, P, P, P, *lays4, *args, fa.FA_FP32, None, None, P, r(bl_ok),
                          None) == fa.FA_ERR_UNSUPPORTED
 
 
