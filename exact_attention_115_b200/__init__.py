@@ -296,6 +296,9 @@ def attention(q, k, v, causal: bool = False, scale: float | None = None, dropout
     Returns O only (L is kept for the backward)."""
     if scale is None:
         scale = 1.0 / math.sqrt(q.shape[-1])
+    if bias is not None and bias.requires_grad:
+        raise ValueError("the bias is an input constant: its gradient is not computed "
+                         "(pass bias.detach() to use it as one)")
     if dropout_p > 0 and seed is None:
         seed = int(torch.randint(0, 2**62, (1,)).item())
     O, _ = _Attention.apply(q, k, v, bool(causal), float(scale), float(dropout_p),

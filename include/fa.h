@@ -126,8 +126,9 @@ typedef struct {
  *
  * fa_fwd for tensors with arbitrary strides (one fa_layout each for Q, K, V
  * and O; L stays contiguous [B, H, Nq]), optional dropout (NULL or p = 0:
- * none) and optional key padding.  fa_fwd is this call with contiguous
- * layouts, no dropout and no padding.
+ * none), optional key padding and an optional additive bias (both above).
+ * fa_fwd is this call with contiguous layouts, no dropout, no padding and
+ * no bias.
  * Layout errors and a dropout probability outside [0, 1) (or one that keeps
  * nothing after rounding): FA_ERR_INVALID; a non-contiguous fp32 tensor or
  * fp32 with dropout: FA_ERR_UNSUPPORTED (the fp32 path reads contiguous
@@ -153,11 +154,12 @@ int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const voi
 
 /* fa_bwd for tensors with arbitrary strides (layouts of Q, K, V, O, dO, dQ,
  * dK, dV in that order; L stays contiguous), the forward's dropout (the
- * same fa_dropout as the forward call, or NULL) and its key padding.  With dropout the gradient
+ * same fa_dropout as the forward call, or NULL), its key padding and its
+ * bias (P is rebuilt with the bias; no bias gradient is returned).  With dropout the gradient
  * is the exact one for the drawn Z: dV = (P ∘ Z · s)ᵀ dO,
  * dP = (dO Vᵀ) ∘ Z · s, dS = P ∘ (dP − D), s = 256/T.  fa_bwd is this call
- * with contiguous layouts, no dropout and no padding.  Errors as for
- * fa_fwd_ex and fa_bwd. */
+ * with contiguous layouts, no dropout, no padding and no bias.  Errors as
+ * for fa_fwd_ex and fa_bwd. */
 int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
               const float* L, void* dQ, void* dK, void* dV, const fa_layout* lq,
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, const fa_layout* ldo,

@@ -225,3 +225,13 @@ def test_decode_ex_checks_the_length_pointer(lib):
                             None) == fa.FA_ERR_INVALID
     assert lib.fa_decode_ex(P, P, P, P, P, 1, 2, 64, 64, 0.125, fa.FA_FP32, 0, None, P, 1 << 20,
                             None) == fa.FA_ERR_UNSUPPORTED
+
+
+def test_attention_rejects_a_bias_that_wants_a_gradient():
+    """The bias is an input constant; asking autograd for its gradient fails
+    loudly instead of silently returning none (checked before any launch)."""
+    import torch
+    b = torch.zeros(1, 1, 4, 8, requires_grad=True)
+    q = torch.zeros(1, 1, 4, 64)
+    with pytest.raises(ValueError):
+        fa.attention(q, q, q, bias=b)
