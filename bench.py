@@ -8,7 +8,10 @@ B=8, H=16, N=2048, d=128, bf16: fa_fwd (forward kernel), then fa_bwd
 forward and 2.5× that for the backward (causal halves both).  Inputs live in
 HBM before the timed region; each step touches ~0.4 GB, larger than the
 126 MB L2, so no flush is inserted.  The decode workload (B=32, H=32,
-Nk=32768, d=128) is timed separately and reported under "decode".
+Nk=32768, d=128) is timed separately and reported under "decode", and the
+other training workloads (B4 H16 N1024 d64, B1 H32 N16384 d128 causal with
+Q×3, and the causal 2K one in fp16) under "other_workloads", each with its
+fwd, bwd and fwd+bwd TFLOPS against both measured bf16 peaks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -24,7 +27,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -88,61 +90,81 @@ def dist_info():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling during the timed region."""
+    """SM clock, power and throttle reasons sampled DURING the timed region.
 
-    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    A thread polls NVML about every 2 ms (the driver's default 20-step
+    region lasts ~15 ms, far shorter than nvidia-smi's sampling period), and
+    one sample is taken right at the start and one right at the end of the
+    region, so even a short region has a record.  Without NVML the record
+    says so and holds no samples."""
 
-    def __init__(self, gpu_index: int):
-        self.gpu = gpu_index
-        self.proc = None
+    REASONS = {"hw_slowdown": 0x8, "hw_thermal_slowdown": 0x40, "sw_thermal_slowdown": 0x20,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int):
+        import threading
+
+        self.dev = device_index
+        self.samples = []
+        self.smax = None
+        self.handle = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nvml = pynvml
+            props = torch.cuda.get_device_properties(device_index)
+            try:
+                self.handle = pynvml.nvmlDeviceGetHandleByUUID(f"GPU-{props.uuid}")
+            except Exception:  # noqa: BLE001 - fall back to the PCI address
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                self.handle = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001 - NVML missing or the device not found
+            self.handle = None
+
+    def sample(self):
+        if self.handle is None:
+            return
+        n = self.nvml
+        try:
+            self.samples.append((n.nvmlDeviceGetClockInfo(self.handle, n.NVML_CLOCK_SM),
+                                 n.nvmlDeviceGetPowerUsage(self.handle) / 1000.0,
+                                 n.nvmlDeviceGetCurrentClocksEventReasons(self.handle)))
+        except Exception:  # noqa: BLE001
+            pass
+
+    def _run(self):
+        while not self._stop.wait(0.002):
+            self.sample()
 
     def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+        """Call right before the timed region (after any warm-up)."""
+        import threading
 
-    def stop(self, window=None):
-        """Summary of the samples taken inside `window` (host seconds, as from
-        time.time()), or of all of them when no window is given."""
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            out, _ = self.proc.communicate(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-            out, _ = self.proc.communicate()
-        import datetime
+        self.samples = []
+        self.sample()
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
 
-        sm, pw, smax, reasons = [], [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in out.strip().splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 10:
-                continue
-            try:
-                ts = datetime.datetime.strptime(f[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
-                clk, cmax = float(f[2]), float(f[3])
-                watts = float(f[4])
-            except ValueError:
-                continue
-            if window is not None and not (window[0] <= ts <= window[1]):
-                continue
-            sm.append(clk)
-            pw.append(watts)
-            smax = cmax
-            for n, v in zip(names, f[6:10]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "power_w": statistics.median(pw) if pw else None, "reasons": sorted(reasons),
-                "samples": len(sm)}
+    def stop(self):
+        """Call right after the timed region; returns the summary."""
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join()
+        self.sample()
+        if self.handle is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["NVML unavailable"],
+                    "samples": 0}
+        sm = [c for c, _, _ in self.samples]
+        pw = [p for _, p, _ in self.samples]
+        reasons = sorted({name for _, _, r in self.samples
+                          for name, bit in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_min_mhz": min(sm) if sm else None,
+                "sm_max_mhz": self.smax, "power_w": statistics.median(pw) if pw else None,
+                "reasons": reasons, "samples": len(sm), "source": "nvml, ~2 ms"}
 
 
 def time_oracle_sample(w, budget_s=12.0):
@@ -198,6 +220,78 @@ def run_reference(args, w):
     print(json.dumps(line), flush=True)
 
 
+def peak_fracs(achieved, peaks):
+    """achieved TFLOP/s against both measured bf16 peaks."""
+    return {"frac_burst": achieved / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])),
+            "frac_sustained": achieved / float(peaks.get("bf16_tflops_sustained",
+                                                         FALLBACK_PEAKS["bf16_tflops_sustained"]))}
+
+
+def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None):
+    """fwd and bwd of one workload, each launch bracketed by CUDA events on
+    the launching stream (the main backward kernel by the library's own
+    timing events); with ``flush`` (a buffer larger than L2) L2 is cleared
+    before every timed launch.  Returns the workload's sub-object."""
+    q, k, v, do = W.make_inputs(w, device=dev)
+    O, L = fa.forward(q, k, v, causal=w.causal)
+    dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
+    ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d, q.dtype), dtype=torch.uint8,
+                     device=dev)
+
+    def fwd():
+        fa.forward(q, k, v, causal=w.causal, out=O, lse=L)
+
+    def bwd():
+        fa.backward(q, k, v, O, do, L, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+
+    for _ in range(3):
+        fwd()
+        bwd()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(6)] for _ in range(iters)]
+    for e in ev:
+        for x in e:
+            x.record(stream)
+    torch.cuda.synchronize()
+    for e in ev:
+        if flush is not None:
+            flush.zero_()
+        e[0].record(stream)
+        fwd()
+        e[1].record(stream)
+        if flush is not None:
+            flush.zero_()
+        e[2].record(stream)
+        fa.set_bwd_timing_events(e[4], e[5])
+        bwd()
+        e[3].record(stream)
+    torch.cuda.synchronize()
+    fa.set_bwd_timing_events(None, None)
+    st = fa.status()
+    if st != fa.FA_OK:
+        raise RuntimeError(f"{w.name}: kernel status {fa.STATUS_NAMES.get(st, st)}")
+    f_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    b_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    m_ms = statistics.mean(e[4].elapsed_time(e[5]) for e in ev)
+    f_tf = w.fwd_flops / (f_ms * 1e-3) / 1e12
+    b_tf = w.bwd_flops / (b_ms * 1e-3) / 1e12
+    fb_tf = (w.fwd_flops + w.bwd_flops) / ((f_ms + b_ms) * 1e-3) / 1e12
+    main_tf = w.bwd_flops / (m_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"]))
+    if w.dtype == "fp16":  # the same dense tensor rate as bf16 (kind::f16 MMAs)
+        pk = f"{peak_kind} burst bf16 (fp16 runs at the bf16 rate)"
+    else:
+        pk = f"{peak_kind} burst bf16"
+    return {"workload": w.name, "shape": w.describe(), "iters": iters,
+            "l2": "flushed before every timed launch" if flush is not None
+                  else "inputs larger than L2; no flush",
+            "fwd": {"ms": f_ms, "tflops": f_tf, **peak_fracs(f_tf, peaks)},
+            "bwd": {"ms": b_ms, "tflops": b_tf, "main_kernel_ms": m_ms,
+                    "main_kernel_tflops": main_tf, **peak_fracs(b_tf, peaks)},
+            "fwd_bwd": {"ms": f_ms + b_ms, "tflops": fb_tf, **peak_fracs(fb_tf, peaks)},
+            "roofline": {"bound": "tensor", "kernel": "bwd_main_kernel", "achieved": main_tf,
+                         "peak": peak, "unit": UNIT, "frac": main_tf / peak, "peak_kind": pk}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -208,6 +302,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads (B4 H16 N1024 d64, the 16K causal one, fp16)")
     args = ap.parse_args()
     w = W.CAUSAL_2K
     if args.impl == "reference":
@@ -261,12 +357,10 @@ def main():
     torch.cuda.synchronize()
 
     sampler = ClockSampler(local)
-    sampler.start()
-    time.sleep(0.3)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    host_t0 = time.time()
+    sampler.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
     t_start.record(stream)
@@ -279,11 +373,10 @@ def main():
         ev["s1"][i].record(stream)
     t_stop.record(stream)
     torch.cuda.synchronize()
-    host_t1 = time.time()
+    clocks = sampler.stop()
     fa.set_bwd_timing_events(None, None)
     if pg:
         pg.barrier()
-    clocks = sampler.stop(window=(host_t0, host_t1))
     st = fa.status()
     if st != fa.FA_OK:
         raise RuntimeError(f"kernel status {fa.STATUS_NAMES.get(st, st)}, "
@@ -371,13 +464,25 @@ def main():
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": ksteps}
 
+    # The other workloads' fwd, bwd and fwd+bwd, each timed on its own (no
+    # collective: every rank runs its own copy and rank 0 reports its own).
+    del dq, dk, dv, ws, q, k, v, do, O, L
+    torch.cuda.empty_cache()
+    others = None
+    if not args.no_extra:
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        flush = torch.empty(4 * l2, dtype=torch.uint8, device=dev)  # written before each launch
+        iters = max(5, min(K, 20))
+        others = [time_workload(fa, W.MEDIUM, dev, stream, iters, peaks, peak_kind, flush=flush),
+                  time_workload(fa, W.LONG_16K, dev, stream, iters, peaks, peak_kind),
+                  time_workload(fa, W.CAUSAL_2K_FP16, dev, stream, iters, peaks, peak_kind)]
+        del flush
+        torch.cuda.empty_cache()
+
     # Decode (split-KV + combine), timed on its own.
     decode = None
-    del dq, dk, dv, ws
     if not args.no_decode:
         wd = W.DECODE_32K
-        del q, k, v, do, O, L
-        torch.cuda.empty_cache()
         dq_, dk_, dv_, _ = W.make_inputs(wd, device=dev, with_grad=False)
         Od, Ld = fa.decode(dq_, dk_, dv_)
         wsd = torch.empty(fa.decode_workspace_bytes(wd.B, wd.H, wd.Nk, wd.d), dtype=torch.uint8,
@@ -421,13 +526,21 @@ def main():
                    "seq_len": w.Nq, "heads": w.H, "head_dim": w.d, "causal": True,
                    "parallelism": f"replicas{world}",
                    "l2": "inputs ~0.4 GB per step > 126 MB L2; no flush"},
-        "fwd": {"ms": fwd_avg, "tflops": achieved_fwd},
+        "fwd": {"ms": fwd_avg, "tflops": achieved_fwd, **peak_fracs(achieved_fwd, peaks)},
         "bwd": {"ms": bwd_avg, "tflops": w.bwd_flops / (bwd_avg * 1e-3) / 1e12,
-                "main_kernel_ms": bwd_main_avg},
+                "main_kernel_ms": bwd_main_avg,
+                **peak_fracs(w.bwd_flops / (bwd_avg * 1e-3) / 1e12, peaks)},
+        # the 60 % target of the fwd+bwd step is stated against the burst
+        # (isolated-GEMM) peak; the sustained one is the figure under the
+        # power cap that a long run reaches
         "pct_of_peak": value / world / peak_bf16,
+        "step_fracs": {**peak_fracs(value / world, peaks), "target": 0.60,
+                       "target_uses": "frac_burst"},
         "roofline": {"bound": "tensor", "kernel": "bwd_main_kernel", "achieved": achieved_bwd,
                      "peak": peak_bf16, "unit": "TFLOP/s", "frac": achieved_bwd / peak_bf16,
+                     **peak_fracs(achieved_bwd, peaks),
                      "peak_kind": f"{peak_kind} {'sustained' if sustained else 'burst'} bf16",
+                     "fwd_kernel": {"achieved": achieved_fwd, **peak_fracs(achieved_fwd, peaks)},
                      "traffic": kernel_traffic("bwd_main_kernel", (
                          "exact_attention_115_b200/csrc/bwd.cu",
                          "exact_attention_115_b200/csrc/common.cuh")),
@@ -436,6 +549,7 @@ def main():
         "gpu_launches": 4 * K,
         "clocks": clocks,
         "decode": decode,
+        "other_workloads": others,
         "cpu_baseline": cpu,
     }
     print(json.dumps(line), flush=True)

@@ -155,6 +155,13 @@ def _stream(device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
 
+def _on(device):
+    """Context that makes ``device`` current for one library call: the C side
+    launches on the current device and looks up per-device state (tensor-map
+    encoder, scratch addresses) there, so it must be the tensors' device."""
+    return torch.cuda.device(device)
+
+
 def _raise(fn, code):
     if code != FA_OK:
         raise FAError(fn, code)
@@ -188,17 +195,19 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
     kvl = _kv_len_ptr(kv_len, B, q.device)
     bp, bl = _bias_args(bias, q, B, H, Nq, Nk)
     if dr is None and kvl is None and bp is None and all(t.is_contiguous() for t in (q, k, v, out)):
-        rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                          lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
-                          _dtype_code(q), _stream(q.device))
+        with _on(q.device):
+            rc = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                              lse.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                              _dtype_code(q), _stream(q.device))
         _raise("fa_fwd", rc)
         return out, lse
     lq, lk, lv, lo = _layout(q), _layout(k), _layout(v), _layout(out)
-    rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                         ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv), ctypes.byref(lo),
-                         B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                         None if dr is None else ctypes.byref(dr), kvl, bp,
-                         None if bl is None else ctypes.byref(bl), _stream(q.device))
+    with _on(q.device):
+        rc = lib().fa_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                             lse.data_ptr(), ctypes.byref(lq), ctypes.byref(lk), ctypes.byref(lv),
+                             ctypes.byref(lo), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                             _dtype_code(q), None if dr is None else ctypes.byref(dr), kvl, bp,
+                             None if bl is None else ctypes.byref(bl), _stream(q.device))
     _raise("fa_fwd_ex", rc)
     return out, lse
 
@@ -245,20 +254,23 @@ def backward(q, k, v, o, do, lse, causal: bool = False, scale: float | None = No
     kvl = _kv_len_ptr(kv_len, B, dev)
     bp, bl = _bias_args(bias, q, B, H, Nq, Nk)
     if dr is None and kvl is None and bp is None and all(t.is_contiguous() for t in ts):
-        rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                          lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                          B, H, Nq, Nk, d, int(bool(causal)), float(scale), _dtype_code(q),
-                          workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                          _stream(dev))
+        with _on(dev):
+            rc = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                              do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                              dv.data_ptr(), B, H, Nq, Nk, d, int(bool(causal)), float(scale),
+                              _dtype_code(q), workspace.data_ptr(),
+                              workspace.numel() * workspace.element_size(), _stream(dev))
         _raise("fa_bwd", rc)
         return dq, dk, dv
     lays = [_layout(t) for t in ts]
-    rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(),
-                         lse.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(),
-                         *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d, int(bool(causal)),
-                         float(scale), _dtype_code(q), None if dr is None else ctypes.byref(dr),
-                         kvl, bp, None if bl is None else ctypes.byref(bl), workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                         _stream(dev))
+    with _on(dev):
+        rc = lib().fa_bwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                             do.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                             dv.data_ptr(), *[ctypes.byref(l) for l in lays], B, H, Nq, Nk, d,
+                             int(bool(causal)), float(scale), _dtype_code(q),
+                             None if dr is None else ctypes.byref(dr), kvl, bp,
+                             None if bl is None else ctypes.byref(bl), workspace.data_ptr(),
+                             workspace.numel() * workspace.element_size(), _stream(dev))
     _raise("fa_bwd_ex", rc)
     return dq, dk, dv
 
@@ -271,15 +283,18 @@ class _Attention(torch.autograd.Function):
     def forward(ctx, q, k, v, causal, scale, dropout_p, seed, offset, kv_len, bias):
         O, L = forward(q, k, v, causal=causal, scale=scale, dropout_p=dropout_p, seed=seed,
                        offset=offset, kv_len=kv_len, bias=bias)
-        ctx.save_for_backward(q, k, v, O, L)
-        ctx.args = (causal, scale, dropout_p, seed, offset, kv_len, bias)
+        # bias and kv_len are saved too (None when absent), so that an
+        # in-place change between the passes raises instead of silently
+        # rebuilding a different P in the backward
+        ctx.save_for_backward(q, k, v, O, L, kv_len, bias)
+        ctx.args = (causal, scale, dropout_p, seed, offset)
         ctx.mark_non_differentiable(L)
         return O, L
 
     @staticmethod
     def backward(ctx, dO, dL):
-        q, k, v, O, L = ctx.saved_tensors
-        causal, scale, dropout_p, seed, offset, kv_len, bias = ctx.args
+        q, k, v, O, L, kv_len, bias = ctx.saved_tensors
+        causal, scale, dropout_p, seed, offset = ctx.args
         if dO.stride(-1) != 1:
             dO = dO.contiguous()
         dq, dk, dv = backward(q, k, v, O, dO, L, causal=causal, scale=scale, dropout_p=dropout_p,
@@ -331,16 +346,18 @@ def decode(q, k, v, scale: float | None = None, num_splits: int = 0, out=None, l
         workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     kvl = _kv_len_ptr(kv_len, B, q.device)
     if kvl is None:
-        rc = lib().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                             lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
-                             int(num_splits), workspace.data_ptr(),
-                             workspace.numel() * workspace.element_size(), _stream(q.device))
+        with _on(q.device):
+            rc = lib().fa_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                 lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
+                                 int(num_splits), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(), _stream(q.device))
         _raise("fa_decode", rc)
         return out, lse
-    rc = lib().fa_decode_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr(),
-                            B, H, Nk, d, float(scale), _dtype_code(q), int(num_splits), kvl,
-                            workspace.data_ptr(), workspace.numel() * workspace.element_size(),
-                            _stream(q.device))
+    with _on(q.device):
+        rc = lib().fa_decode_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
+                                int(num_splits), kvl, workspace.data_ptr(),
+                                workspace.numel() * workspace.element_size(), _stream(q.device))
     _raise("fa_decode_ex", rc)
     return out, lse
 
@@ -365,9 +382,10 @@ def decode_noalloc(q, k, v, scale: float | None = None, num_splits: int = 0, out
         lse = torch.empty((B, H, 1), dtype=torch.float32, device=q.device)
     _check("out", out, q.shape, q.dtype)
     _check("lse", lse, (B, H, 1), torch.float32)
-    rc = lib().fa_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                                 lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
-                                 int(num_splits), _stream(q.device))
+    with _on(q.device):
+        rc = lib().fa_decode_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                                     lse.data_ptr(), B, H, Nk, d, float(scale), _dtype_code(q),
+                                     int(num_splits), _stream(q.device))
     _raise("fa_decode_noalloc", rc)
     return out, lse
 

@@ -33,8 +33,9 @@
 // MN-major operand of the dQ product:
 //   d = 128: dQᵀ = Kᵀ dSᵀ (M = d = 128), reduced from registers with one
 //            coalesced red.global.add.f32 per warp and query row;
-//   d = 64:  dQ = dS K (M = BM = 128), staged in shared memory and reduced
-//            with one bulk reduce-add (cp.reduce.async.bulk .add.f32).
+//   d = 64:  dQ = dS K (M = BM = 128), staged in shared memory as two
+//            128-byte-swizzled [128 × 32] fp32 halves and reduced with two
+//            TMA tensor reduce-adds (cp.reduce.async.bulk.tensor .add.f32).
 // Roles (512 threads, setmaxnreg split 136 / 136 / 104 registers):
 //   warpgroups 0 and 1: thread = key row; warpgroup c computes P and dS for
 //                query columns [64c, 64c + 64) of each step;
@@ -67,16 +68,6 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
       "l"(src), "r"(bytes), "r"(smem_u32(bar))
       : "memory");
 }
-__device__ __forceinline__ void bulk_reduce_add_f32(float* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst),
-               "r"(smem_u32(src)), "r"(bytes)
-               : "memory");
-}
 __device__ __forceinline__ void red_add_f32(float* dst, float v) {
   asm volatile("red.global.add.f32 [%0], %1;" ::"l"(dst), "f"(v) : "memory");
 }
@@ -95,8 +86,8 @@ struct BwdTraits {
   static constexpr int Q_CHUNK = BM * 128;
   static constexpr int DS_TILE = BN * BM * ES;       // dSᵀ, rows = keys, q contiguous
   // dQ staging (d = 64 only): the whole [BM × 64] fp32 tile (32 KB) goes to
-  // shared memory and out with one bulk reduce-add; d = 128 reduces dQᵀ from
-  // registers and needs no staging.
+  // shared memory as two swizzled halves and out with two tensor reduce-adds;
+  // d = 128 reduces dQᵀ from registers and needs no staging.
   static constexpr int DQ_STAGE = DQ_T ? 0 : BM * D * 4;
   // shared-memory offsets (all 1024-aligned).  K is double buffered (the
   // next work item's K loads while this item runs); Q is double buffered
@@ -131,21 +122,6 @@ struct BwdTraits {
   static constexpr uint32_t IDESC_DQ = make_idesc(F, 128, DQ_T ? BM : D, 1, 1);
 };
 
-#ifdef FA_TRACE
-// One fixed slot per event code (plain stores; no atomics on the critical path).
-__device__ long long g_btrace[32768];
-__device__ __forceinline__ void btrace(bool on, int code) {
-  if (!on || code >= 32768) return;
-  long long t;
-  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
-  g_btrace[code] = t;
-}
-#define BTRACE(code) btrace(trace_on, (code))
-// per CTA: globaltimer and clock64 at set-up and at exit
-__device__ long long g_cta_times[4][1024];
-#else
-#define BTRACE(code) ((void)0)
-#endif
 
 // The kernel is persistent: a CTA takes work items (K/V block, head) in turn
 // and numbers its steps across items (g).  The per-step barriers complete
@@ -235,9 +211,6 @@ __global__ void __launch_bounds__(512, 1)
     j = *reinterpret_cast<volatile int*>(&bars->item_idx[it & 3]);
     return j >= 0;
   };
-#ifdef FA_TRACE
-  const bool trace_cta = blockIdx.x == 0;
-#endif
 
   if (threadIdx.x == 0) {
     for (int b = 0; b < 2; ++b) {
@@ -278,13 +251,6 @@ __global__ void __launch_bounds__(512, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
-#ifdef FA_TRACE
-  btrace(trace_cta && threadIdx.x == 0, 15000);  // set-up done
-  if (threadIdx.x == 0 && blockIdx.x < 1024) {
-    g_cta_times[0][blockIdx.x] = (long long)globaltimer_ns();
-    g_cta_times[1][blockIdx.x] = clock64();
-  }
-#endif
 
   uint8_t* sK0 = smem + Tr::OFF_K;  // two K buffers, KV_TILE apart
   uint8_t* sV = smem + Tr::OFF_V;
@@ -326,17 +292,11 @@ __global__ void __launch_bounds__(512, 1)
           ok = false;
           continue;
         }
-#ifdef FA_TRACE
-        btrace(trace_cta && it < 200, 19600 + it);  // item: K load issued
-#endif
         mbar_arrive_expect_tx(&bars->k_full[b], Tr::KV_TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
           tma_load_bh(sK0 + b * Tr::KV_TILE + c * Tr::KV_CHUNK, &tmK, GEN && ((p.map4d >> 1) & 1),
                       &bars->k_full[b], c * 64, key0, bh, p.H);
-#ifdef FA_TRACE
-        btrace(trace_cta && it < 200, 19400 + it);  // item: V load issued
-#endif
         mbar_arrive_expect_tx(&bars->v_full, Tr::KV_TILE);
 #pragma unroll
         for (int c = 0; c < D / 64; ++c)
@@ -462,9 +422,6 @@ __global__ void __launch_bounds__(512, 1)
         item(j, bh, kb, i0, n_q);
         (void)bh;
         (void)i0;
-#ifdef FA_TRACE
-        const bool trace_on = trace_cta && it == 0;
-#endif
         const int b = it & 1;
         const uint64_t dK_k = kbuf(dK_k0, b), dK_mn = kbuf(dK_mn0, b);
         ok = MBAR_WAIT(&bars->k_full[b], (it >> 1) & 1, abort_flag);
@@ -473,10 +430,6 @@ __global__ void __launch_bounds__(512, 1)
                MBAR_WAIT(&bars->do_full, g & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
-        BTRACE(15001);
-#ifdef FA_TRACE
-        btrace(trace_cta && it < 200, 19000 + it);  // item: K, Q0, dO0 landed
-#endif
         if (n_q > 0) {
           mma_st(colS, dK_k, stg(dQ_k0, g & 1));
           tc_commit(&bars->s_full);
@@ -511,10 +464,8 @@ __global__ void __launch_bounds__(512, 1)
           ok = MBAR_WAIT(&bars->p_ready, gs & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          BTRACE(2000 + i);
           mma_dv(i > 0);
           tc_commit(&bars->do_empty);
-          BTRACE(3000 + i);
           if (more) {
             ok = MBAR_WAIT(&bars->q_full[s ^ 1], ((gs + 1) >> 1) & 1, abort_flag);
             tc_fence_after();
@@ -522,14 +473,9 @@ __global__ void __launch_bounds__(512, 1)
             mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
             tc_commit(&bars->s_full);
           }
-          BTRACE(1000 + i);
           ok = MBAR_WAIT(&bars->ds_ready, gs & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          BTRACE(4000 + i);
-#ifdef FA_TRACE
-          btrace(trace_cta && gs < 2000, 20000 + gs);  // got dS of global step gs
-#endif
           // dQ first, so warpgroup 2 drains it while the tensor core runs dK.
           mma_dq(dK_mn);
           tc_commit(&bars->dq_full);
@@ -537,7 +483,6 @@ __global__ void __launch_bounds__(512, 1)
           mma_dk(stg(dQ_mn0, s), i > 0);
           tc_commit(&bars->q_empty[s]);
           tc_commit(&bars->ds_free);
-          BTRACE(5000 + i);
           if (more) {
             ok = MBAR_WAIT(&bars->dq_empty, gs & 1, abort_flag) &&
                  MBAR_WAIT(&bars->do_full, (gs + 1) & 1, abort_flag);
@@ -546,15 +491,11 @@ __global__ void __launch_bounds__(512, 1)
             mma_st(colDP, dV_k, dO_k);
             tc_commit(&bars->dp_full);
             if (i + 2 == n_q) tc_commit(&bars->v_free);  // the item's last dPᵀ
-            BTRACE(6000 + i);
           }
         }
         if (!ok) break;
         if (n_q == 0) tc_commit(&bars->k_free[b]);
         tc_commit(&bars->dkv_done);  // after the item's last dK (or at once if it has no steps)
-#ifdef FA_TRACE
-        btrace(trace_cta && it < 200, 19200 + it);  // item: last products issued
-#endif
         g += n_q;
       }
     }
@@ -576,9 +517,6 @@ __global__ void __launch_bounds__(512, 1)
     for (int j; ok && __all_sync(0xffffffffu, take_item(it, j)); ++it) {
       int bh, kb, i0, n_q;
       item(j, bh, kb, i0, n_q);
-#ifdef FA_TRACE
-      const bool trace_on = trace_cta && it == 0;
-#endif
       const int key0 = kb * Tr::BN;
       const int key = key0 + kr;
       const bool key_live = key < keys_of(p.kv_len, bh, p.H, p.Nk);
@@ -616,10 +554,6 @@ __global__ void __launch_bounds__(512, 1)
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, gs & 1, abort_flag));
         tc_fence_after();
         if (!ok) break;
-#ifdef FA_TRACE
-        btrace(trace_on && quad == 0 && lane == 0, 7000 + 100 * cw + i);  // got S
-        btrace(trace_cta && warp == 0 && lane == 0 && i == 0 && it < 200, 19800 + it);  // item: first S
-#endif
         const bool need_mask = !key_live || (CAUSAL && (key0 + Tr::BN - 1 > q0 + off));
         uint32_t Pk[CWC / 2];  // P as packed pairs of the input type
         const uint64_t c2 = pk2(sl2, sl2);
@@ -722,9 +656,6 @@ __global__ void __launch_bounds__(512, 1)
         }
         fence_async_smem();
         tc_fence_before();
-#ifdef FA_TRACE
-        btrace(trace_on && quad == 0 && lane == 0, 8000 + 100 * cw + i);  // dS done
-#endif
         mbar_arrive(&bars->ds_ready);
       }
       g += n_q;
@@ -866,17 +797,8 @@ __global__ void __launch_bounds__(512, 1)
     if (leader) bulk_wait0();
   }
 
-#ifdef FA_TRACE
-  btrace(trace_cta && lane == 0, 14100 + warp);  // warp finished
-#endif
   tc_fence_before();
   __syncthreads();
-#ifdef FA_TRACE
-  if (threadIdx.x == 0 && blockIdx.x < 1024) {
-    g_cta_times[2][blockIdx.x] = (long long)globaltimer_ns();
-    g_cta_times[3][blockIdx.x] = clock64();
-  }
-#endif
   if (warp == 12) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -1157,20 +1079,5 @@ cudaError_t launch_bwd(int dtype, int d, bool causal, const BwdLaunch& a) {
 
 FA_ERROR_ACCESSOR(take_error_bwd)
 
-#ifdef FA_TRACE
-}  // namespace fa
-extern "C" int fa_cta_times_read(long long* out) {
-  cudaMemcpyFromSymbol(out, fa::g_cta_times, sizeof(fa::g_cta_times));
-  return 4 * 1024;
-}
-extern "C" int fa_btrace_read(long long* out, int max) {
-  const int n = max < 32768 ? max : 32768;
-  cudaMemcpyFromSymbol(out, fa::g_btrace, sizeof(long long) * n);
-  static long long zeros[32768];
-  cudaMemcpyToSymbol(fa::g_btrace, zeros, sizeof(zeros));
-  return n;
-}
-namespace fa {
-#endif
 
 }  // namespace fa

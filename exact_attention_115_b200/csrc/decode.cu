@@ -225,20 +225,59 @@ size_t decode_scratch_bytes() { return kDecodeScratchBytes; }
 // In host code g_decode_scratch names a host-side stand-in, not device
 // memory, so its device address on the current device is looked up with
 // cudaGetSymbolAddress, once per device (by the first no-alloc call made
-// with that device current), and cached.
+// with that device current), and cached.  The cache is keyed by the unique
+// ID of the device's context as well: a cudaDeviceReset (or any other
+// teardown of the primary context) reloads the module, possibly at another
+// address, and the next call then looks the address up again instead of
+// handing the kernels a stale one.
+namespace {
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique ID of the current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+}  // namespace
+
 cudaError_t decode_scratch_ptr(void** out) {
   static std::mutex mu;
   static void* cached[64] = {};
+  static unsigned long long cached_ctx[64] = {};
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  // make the device's primary context current (a no-op when it already is),
+  // so that its ID can be read
+  e = cudaSetDevice(dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(mu);
-  if (cached[dev] == nullptr) {
+  if (cached[dev] == nullptr || ctx == 0 || cached_ctx[dev] != ctx) {
     void* ptr = nullptr;
     e = cudaGetSymbolAddress(&ptr, g_decode_scratch);
     if (e != cudaSuccess) return e;
     cached[dev] = ptr;
+    cached_ctx[dev] = ctx;
   }
   *out = cached[dev];
   return cudaSuccess;

@@ -80,20 +80,6 @@ struct FwdTraits {
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
 
-#ifdef FA_TRACE
-// One fixed slot per event code (no atomics: a plain store does not stall).
-__device__ long long g_trace[16384][2];
-__device__ int g_trace_n;
-__device__ __forceinline__ void trace_ev(bool on, int code) {
-  if (!on) return;
-  long long t;
-  asm volatile("mov.u64 %0, %%clock64;" : "=l"(t));
-  if (code < 16384) { g_trace[code][0] = code; g_trace[code][1] = t; }
-}
-#define TRACE(code) trace_ev(trace_on, (code))
-#else
-#define TRACE(code) ((void)0)
-#endif
 
 struct FwdBarriers {
   uint64_t q_full[2];
@@ -215,9 +201,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
   grouped_order(blockIdx.x, p.B * p.H, n_qb, p.head_group, bh, blk);
   const int qb = CAUSAL ? n_qb - 1 - blk : blk;  // causal: the last query blocks see the most keys
   const int q_row0 = qb * 128 * Tr::TILES;
-#ifdef FA_TRACE
-  const bool trace_on = blockIdx.x == 0;
-#endif
   const int off = p.Nk - p.Nq;  // bottom-right causal alignment (full Nk)
   const int nk = keys_of(p.kv_len, bh, p.H, p.Nk);  // keys this batch element sees
 
@@ -264,14 +247,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
   if (warp > Tr::PRODUCER_WARP) {
     // idle warps of the producer/MMA warpgroup
     regs_dec<Tr::REGS_OTHER>();
-#ifdef FA_TRACE
-    if (warp == Tr::PRODUCER_WARP + 1 && lane == 0 && trace_on && Tr::NS < 8) {
-      for (int g = 0; g < 4 * n_kv; ++g) {
-        if (!MBAR_WAIT(&bars->kv_full[7], g & 1, abort_flag)) break;
-        trace_ev(true, 7000 + g);
-      }
-    }
-#endif
   } else if (warp == Tr::PRODUCER_WARP) {
     // ------------------------------------------------------------ producer
     regs_dec<Tr::REGS_OTHER>();
@@ -371,11 +346,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
           ok = kv_wait(iv) && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          TRACE(3000 + j);
           issue_pv(0, sv, j > 0);
           tc_commit(&bars->o_full[0]);
           tc_commit(&bars->kv_empty[sv]);
-          TRACE(4000 + j);
           if (j + 1 < n_kv) {
             ok = kv_wait(ik);
             tc_fence_after();
@@ -383,7 +356,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
             issue_qk(0, sk);
             tc_commit(&bars->s_full[0]);
             tc_commit(&bars->kv_empty[sk]);
-            TRACE(5000 + j);
           }
         }
       } else {
@@ -391,31 +363,19 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       tc_fence_after();
       if (ok) issue_qk(0, 0);
       tc_commit(&bars->s_full[0]);
-#ifdef FA_TRACE
-      if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
       ok = ok && MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
       tc_fence_after();
       if (ok) issue_qk(1, 0);
       tc_commit(&bars->s_full[1]);
-#ifdef FA_TRACE
-      if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
       tc_commit(&bars->kv_empty[0]);
       for (int j = 0; j < n_kv && ok; ++j) {
         const int iv = 2 * j + 1, ik = 2 * j + 2;
         const int sv = iv % Tr::NS, sk = ik % Tr::NS;
         ok = kv_wait(iv);
-        TRACE(6000 + j);
         ok = ok && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
-        TRACE(3000 + j);
         issue_pv(0, sv, j > 0);
-        TRACE(4000 + j);
-#ifdef FA_TRACE
-        if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
         tc_commit(&bars->o_full[0]);
         const bool more = j + 1 < n_kv;
         if (more) {
@@ -424,30 +384,17 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
           if (!ok) break;
           issue_qk(0, sk);
           tc_commit(&bars->s_full[0]);
-          TRACE(5000 + j);
-#ifdef FA_TRACE
-          if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
         }
         ok = MBAR_WAIT(&bars->p_full[1], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
-        TRACE(3100 + j);
         issue_pv(1, sv, j > 0);
-        TRACE(4100 + j);
-#ifdef FA_TRACE
-        if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
         tc_commit(&bars->o_full[1]);
         tc_commit(&bars->kv_empty[sv]);
         if (more) {
           issue_qk(1, sk);
           tc_commit(&bars->s_full[1]);
           tc_commit(&bars->kv_empty[sk]);
-          TRACE(5100 + j);
-#ifdef FA_TRACE
-          if (trace_on) tc_commit(&bars->kv_full[7]);
-#endif
         }
       }
       }
@@ -490,10 +437,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
       tc_fence_after();
       if (!ok) break;
-#ifdef FA_TRACE
-      const bool tr = trace_on && quad == 0 && lane == 0;
-      trace_ev(tr, 1000 + 100 * t + j);
-#endif
       uint32_t su[4][32];
       if constexpr (BIAS && !TF32) {
         // 32 columns at a time, each plus its bias / scale (so the bias
@@ -625,9 +568,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       }
       tmem_st_wait();
       tc_fence_before();
-#ifdef FA_TRACE
-      trace_ev(tr, 2000 + 100 * t + j);
-#endif
       mbar_arrive(&bars->p_full[t]);
     }
 
@@ -767,17 +707,5 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
 
 FA_ERROR_ACCESSOR(take_error_fwd)
 
-#ifdef FA_TRACE
-}  // namespace fa
-extern "C" int fa_trace_read(long long* out, int max) {
-  const int n = max < 16384 ? max : 16384;
-  cudaMemcpyFromSymbol(out, fa::g_trace, sizeof(long long) * 2 * n);
-  cudaMemset(out, 0, 0);
-  static long long zeros[16384][2];
-  cudaMemcpyToSymbol(fa::g_trace, zeros, sizeof(zeros));
-  return n;
-}
-namespace fa {
-#endif
 
 }  // namespace fa

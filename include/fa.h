@@ -225,7 +225,9 @@ int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L,
  *
  * The first call on each device looks up the array's device address (with
  * that device current) and caches it; make that first call before any
- * stream capture.  All calls share the one array and it keeps the last
+ * stream capture.  The cache remembers the device's context too: after a
+ * cudaDeviceReset the next call looks the address up again (in the new
+ * context) rather than reusing the old one.  All calls share the one array and it keeps the last
  * call's contents (nothing in it needs to start at zero); calls whose
  * kernels overlap on the GPU, on different streams or host threads, race on
  * it and must be serialised by the caller. */

@@ -59,7 +59,11 @@ from __future__ import annotations
 
 import numpy as np
 
-_ROW_CHUNK = 2048
+# Rows of S held at a time.  Rows are independent, so the chunk size changes
+# no result; a small one keeps each temporary (128 × Nk floats) in the
+# allocator's heap instead of a fresh mapping per chunk, whose page faults
+# otherwise dominate the run time at long sequence lengths.
+_ROW_CHUNK = 128
 
 
 def _f64(x) -> np.ndarray:

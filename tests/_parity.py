@@ -9,6 +9,10 @@ up to half a unit in the last place of that dtype (0.0156 for bf16 values in
 therefore 1e-2 plus half an ulp of the output dtype at the reference value;
 the mean-abs bound and the L bound are applied as stated.  ``check_fwd``
 also returns the plain max-abs error so callers can report it."""
+import ctypes
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import torch
 
@@ -61,3 +65,41 @@ def check_grad(G, G_ref, name, what="", scale_ref=None):
     bound = max(G_REL * ref_max, G_ABS_FLOOR)
     assert e <= bound, f"{what}: {name} max-abs {e:.3e} > {bound:.3e} (max|ref| {ref_max:.3e})"
     return e / max(ref_max, 1e-30)
+
+
+def _keep_freed_memory_in_heap():
+    """The oracle's temporaries at long sequence lengths are tens of MB each;
+    glibc maps and unmaps every such block, and the page faults then dominate
+    the oracle's run time.  Raising the trim and mmap thresholds keeps freed
+    blocks in the heap for reuse.  This affects only the test process."""
+    try:
+        libc = ctypes.CDLL("libc.so.6")
+        libc.mallopt(-1, 1 << 30)   # M_TRIM_THRESHOLD
+        libc.mallopt(-3, 32 << 20)  # M_MMAP_THRESHOLD (its largest allowed value)
+    except (OSError, AttributeError):
+        pass
+
+
+_keep_freed_memory_in_heap()
+
+
+def host_cores() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def oracle_map(fn, items):
+    """[fn(x) for x in items] on all host cores, in threads (numpy releases
+    the GIL in its matrix products and element-wise loops, so the calls run
+    in parallel), the cores' BLAS threads shared out between the calls."""
+    from threadpoolctl import threadpool_limits
+
+    workers = min(host_cores(), max(1, len(items)))
+    with threadpool_limits(max(1, host_cores() // workers)):
+        with ThreadPoolExecutor(workers) as ex:
+            return list(ex.map(fn, items))
+
+
+def nan_like(t):
+    """A NaN-filled buffer shaped like ``t``: passed as an output, it shows any
+    element a kernel failed to write (the check then finds a non-finite value)."""
+    return torch.full_like(t, float("nan"))

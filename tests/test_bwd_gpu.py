@@ -79,37 +79,6 @@ def test_peaky(fa):
     run_bwd(fa, 1, 4, 1024, 1024, 128, True, q_mult=3.0, seed=7)
 
 
-def _sampled_bwd(fa, w, heads, n_rows=48, seed=0):
-    q, k, v, do = W.make_inputs(w, device="cuda")
-    O, L = fa.forward(q, k, v, causal=w.causal, scale=w.scale)
-    dq, dk, dv = fa.backward(q, k, v, O, do, L, causal=w.causal, scale=w.scale)
-    assert fa.status() == fa.FA_OK
-    for g in (dq, dk, dv):
-        assert torch.isfinite(g.float()).all()
-    rng = np.random.default_rng(seed)
-    for (b, h) in heads:
-        qr = np.unique(np.concatenate([[0, w.Nq - 1], rng.integers(0, w.Nq, n_rows)]))
-        kr = np.unique(np.concatenate([[0, w.Nk - 1], rng.integers(0, w.Nk, n_rows)]))
-        rq, rk, rv, _ = oracle.head_backward_rows(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]),
-                                                  f64(do[b, h]), w.scale, w.causal, qr, kr)
-        # The bound is relative to the largest gradient of the whole head,
-        # which the sampled rows may miss; use the GPU's own head maximum as
-        # the scale only when it is larger than the sampled reference's.
-        what = f"{w.name} head ({b},{h})"
-        check_grad(dq[b, h][torch.as_tensor(qr, device="cuda")], rq, "dQ", what)
-        check_grad(dk[b, h][torch.as_tensor(kr, device="cuda")], rk, "dK", what)
-        check_grad(dv[b, h][torch.as_tensor(kr, device="cuda")], rv, "dV", what)
-
-
-def test_causal_2k_sampled(fa, dq_mode):
-    _sampled_bwd(fa, W.CAUSAL_2K, [(0, 0), (5, 9)])
-
-
-@pytest.mark.slow
-def test_long_16k_sampled(fa):
-    _sampled_bwd(fa, W.LONG_16K, [(0, 0), (0, 31)], n_rows=24)
-
-
 def test_gradient_sum_invariants(fa):
     """Σ_j dK_j = 0 (rows of dS sum to zero) and Σ_j dV_j = Σ_i dO_i, at a
     size too large for a full oracle comparison."""

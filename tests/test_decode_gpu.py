@@ -45,43 +45,3 @@ def test_decode_matches_forward_kernel(fa):
     O2, L2 = fa.forward(q, k, v)
     assert (O1.float() - O2.float()).abs().max().item() <= 1e-2
     assert (L1 - L2).abs().max().item() <= 1e-3
-
-
-def test_decode_full_size_sampled(fa):
-    w = W.DECODE_32K
-    q, k, v, _ = W.make_inputs(w, device="cuda", with_grad=False)
-    O, L = fa.decode(q, k, v, scale=w.scale)
-    assert fa.status() == fa.FA_OK
-    assert torch.isfinite(O.float()).all() and torch.isfinite(L).all()
-    rng = np.random.default_rng(0)
-    pairs = [(0, 0), (31, 31)] + [tuple(x) for x in rng.integers(0, 32, (6, 2))]
-    for b, h in pairs:
-        O_ref, L_ref = oracle.head_forward(f64(q[b, h]), f64(k[b, h]), f64(v[b, h]), w.scale, False)
-        check_fwd(O[b, h], L[b, h], O_ref, L_ref, f"decode head ({b},{h})")
-    del q, k, v
-    torch.cuda.empty_cache()
-
-
-@pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("splits", [0, 1, 5, 64])
-def test_decode_key_padding(fa, d, splits):
-    """Per-sequence lengths of a KV cache padded to Nk (fa_decode_ex): parts
-    past a length are empty; a zero length gives O = 0, L = -inf."""
-    Nk = 3000
-    kv_len = [Nk, 1, 0, 1537, 64, 5000]
-    B = len(kv_len)
-    q, k, v, _ = W.make_tensors(B, 2, 1, Nk, d, "bf16", seed=70 + d, device="cuda", with_grad=False)
-    scale = 1 / math.sqrt(d)
-    kvl = torch.tensor(kv_len, dtype=torch.int32, device="cuda")
-    O, L = fa.decode(q, k, v, scale=scale, num_splits=splits, kv_len=kvl)
-    assert fa.status() == fa.FA_OK
-    eff = [min(n, Nk) for n in kv_len]
-    O_ref, L_ref = oracle.attention_decode(f64(q), f64(k), f64(v), scale, kv_len=eff)
-    live = [b for b in range(B) if eff[b] > 0]
-    check_fwd(O[live], L[live], O_ref[live], L_ref[live], f"decode kv_len d{d} splits{splits}")
-    assert torch.all(O[2] == 0) and torch.all(torch.isneginf(L[2]))
-    # full lengths equal the unpadded call bit for bit
-    full = torch.full((B,), Nk, dtype=torch.int32, device="cuda")
-    O1, L1 = fa.decode(q, k, v, scale=scale, num_splits=splits, kv_len=full)
-    O0, L0 = fa.decode(q, k, v, scale=scale, num_splits=splits)
-    assert torch.equal(O1, O0) and torch.equal(L1, L0)

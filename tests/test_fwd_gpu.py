@@ -97,32 +97,3 @@ def test_keys_sorted_ascending_force_rescales(fa):
     O, L = fa.forward(q, k, v, causal=False, scale=1.0)
     O_ref, L_ref = oracle.attention_forward(f64(q), f64(k), f64(v), 1.0, False)
     check_fwd(O, L, O_ref, L_ref, "ascending scores")
-
-
-def _sampled(fa, w, heads, rows_per_head=96, seed=0):
-    q, k, v, _ = W.make_inputs(w, device="cuda", with_grad=False)
-    O, L = fa.forward(q, k, v, causal=w.causal, scale=w.scale)
-    assert fa.status() == fa.FA_OK
-    rng = np.random.default_rng(seed)
-    for (b, h) in heads:
-        rows = np.unique(np.concatenate([[0, 1, 127, 128, w.Nq - 1],
-                                         rng.integers(0, w.Nq, rows_per_head)]))
-        qh = f64(q[b, h])
-        O_ref, L_ref = oracle.head_forward(qh[rows], f64(k[b, h]), f64(v[b, h]), w.scale,
-                                           w.causal, rows=rows, nq_total=w.Nq)
-        check_fwd(O[b, h][torch.as_tensor(rows, device="cuda")],
-                  L[b, h][torch.as_tensor(rows, device="cuda")], O_ref, L_ref,
-                  f"{w.name} head ({b},{h})")
-    # properties at every output: finite, |O| bounded by max|V| of the head
-    assert torch.isfinite(O.float()).all() and torch.isfinite(L).all()
-    assert (O.float().abs().amax(dim=(2, 3)) <= v.float().abs().amax(dim=(2, 3)) * 1.01 + 1e-3).all()
-
-
-def test_causal_2k_sampled(fa):
-    w = W.CAUSAL_2K
-    _sampled(fa, w, [(0, 0), (3, 7), (7, 15)])
-
-
-def test_long_16k_sampled(fa):
-    w = W.LONG_16K
-    _sampled(fa, w, [(0, 0), (0, 13), (0, 31)], rows_per_head=64)

@@ -6,9 +6,9 @@ scratch array instead of a caller-provided workspace.
 
 Checked through the C ABI against the existing entry point, fa_decode, on
 two calls in a row (the second call reuses the scratch the first one left),
-with the tolerances used throughout (O 1e-2 plus half an ulp of the output
-dtype, L 1e-3), plus the rejection of sizes beyond the built-in scratch.
-This file is named to be collected last."""
+and against the fp64 oracle, with the tolerances used throughout (O 1e-2
+plus half an ulp of the output dtype, L 1e-3), plus the rejection of sizes
+beyond the built-in scratch.  This file is named to be collected last."""
 import ctypes
 import math
 
@@ -16,6 +16,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import workloads as W
 from tests._parity import check_fwd, f64
 
@@ -45,7 +46,9 @@ def test_noalloc_matches_decode_on_two_calls(num_splits):
         assert fa.status() == fa.FA_OK
         O_ref, L_ref = fa.decode(q, k, v, num_splits=num_splits)
         assert fa.status() == fa.FA_OK
-        check_fwd(O, L, f64(O_ref), f64(L_ref), f"no-alloc decode call {call}")
+        check_fwd(O, L, f64(O_ref), f64(L_ref), f"no-alloc decode call {call} vs fa_decode")
+        O_o, L_o = oracle.attention_decode(f64(q), f64(k), f64(v), 1.0 / math.sqrt(d))
+        check_fwd(O, L, O_o, L_o, f"no-alloc decode call {call} vs the oracle")
 
 
 def test_noalloc_full_size_workload_matches_decode():
@@ -56,6 +59,11 @@ def test_noalloc_full_size_workload_matches_decode():
     assert fa.status() == fa.FA_OK
     O_ref, L_ref = fa.decode(q, k, v)
     check_fwd(O, L, f64(O_ref), f64(L_ref), "no-alloc decode, B32 H32 Nk32768")
+    # batch element 0 (32 heads) against the oracle as well
+    hq, hk, hv = f64(q[0]), f64(k[0]), f64(v[0])
+    for h in range(w.H):
+        O_o, L_o = oracle.head_forward(hq[h], hk[h], hv[h], w.scale, False)
+        check_fwd(O[0, h], L[0, h], O_o, L_o, f"no-alloc decode head (0,{h}) vs the oracle")
     del q, k, v
     torch.cuda.empty_cache()
 

@@ -56,6 +56,8 @@ TINY_BF16 = Workload("tiny_bf16", 1, 1, 128, 128, 64, False, "bf16")
 MEDIUM = Workload("b4h16n1024d64", 4, 16, 1024, 1024, 64, False, "bf16")
 CAUSAL_2K = Workload("b8h16n2048d128_causal", 8, 16, 2048, 2048, 128, True, "bf16")
 LONG_16K = Workload("b1h32n16384d128_causal_q3", 1, 32, 16384, 16384, 128, True, "bf16", q_mult=3.0)
+# the causal 2K workload in fp16 (timed like bf16; a parity case as well)
+CAUSAL_2K_FP16 = Workload("b8h16n2048d128_causal_fp16", 8, 16, 2048, 2048, 128, True, "fp16")
 DECODE_32K = Workload("decode_b32h32nk32768d128", 32, 32, 1, 32768, 128, False, "bf16", decode=True)
 
 ALL = [TINY_FP32, TINY_BF16, MEDIUM, CAUSAL_2K, LONG_16K, DECODE_32K]
