@@ -355,7 +355,13 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp == 12) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<Tr::REGS_OTHER>();
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptor
+    // arithmetic); the elected lane issues the MMAs and commits.
+    {
+      const bool leader = elect_one();
+      auto commit = [&](uint64_t* bar) {
+        if (leader) tc_commit(bar);
+      };
       const uint32_t aK0 = smem_u32(sK0), aV = smem_u32(sV), aQ = smem_u32(sQ), adO = smem_u32(sdO);
       const uint32_t adS = smem_u32(sdS);
       const uint32_t colS = tmem + Tr::COL_S, colDP = tmem + Tr::COL_DP;
@@ -378,7 +384,7 @@ __global__ void __launch_bounds__(512, 1)
         for (int ks = 0; ks < D / 16; ++ks) {
           const uint64_t oa = uint64_t((ks >> 2) * (Tr::KV_CHUNK / 16) + (ks & 3) * 2);
           const uint64_t ob = uint64_t((ks >> 2) * (Tr::Q_CHUNK / 16) + (ks & 3) * 2);
-          mma_ss<false>(dcol, dx + oa, dy + ob, Tr::IDESC_ST, ks > 0);
+          if (leader) mma_ss<false>(dcol, dx + oa, dy + ob, Tr::IDESC_ST, ks > 0);
         }
       };
       // dV [128 × D] += Pᵀ[128 × BM] (TMEM) · dO[BM × D] (MN-major).  Pᵀ
@@ -389,7 +395,7 @@ __global__ void __launch_bounds__(512, 1)
         constexpr int kPerWg = CWC / 16;
 #pragma unroll
         for (int ks = 0; ks < BM / 16; ++ks)
-          mma_ts<false>(colDV, colS + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
+          if (leader) mma_ts<false>(colDV, colS + (ks / kPerWg) * CWC + (ks % kPerWg) * 8,
                         dO_mn + uint64_t(ks * 128), Tr::IDESC_GRAD, (acc || ks > 0) ? 1u : 0u);
       };
       // dK [128 × D] += dSᵀ [128 keys × BM] (shared memory, K-major: key rows of
@@ -398,7 +404,7 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int ks = 0; ks < BM / 16; ++ks) {
           const uint64_t oa = uint64_t((ks >> 2) * (Tr::BN * 128 / 16) + (ks & 3) * 2);
-          mma_ss<false>(colDK, dS_k + oa, dy + uint64_t(ks * 128), Tr::IDESC_GRAD,
+          if (leader) mma_ss<false>(colDK, dS_k + oa, dy + uint64_t(ks * 128), Tr::IDESC_GRAD,
                         (acc || ks > 0) ? 1u : 0u);
         }
       };
@@ -408,49 +414,51 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / 16; ++ks) {
           const uint64_t o = uint64_t(ks * 128);
-          if constexpr (Tr::DQ_T)
-            mma_ss<false>(colDP, dkmn + o, dS_mn + o, Tr::IDESC_DQ, ks > 0);
-          else
-            mma_ss<false>(colDP, dS_mn + o, dkmn + o, Tr::IDESC_DQ, ks > 0);
+          if (leader) {
+            if constexpr (Tr::DQ_T)
+              mma_ss<false>(colDP, dkmn + o, dS_mn + o, Tr::IDESC_DQ, ks > 0);
+            else
+              mma_ss<false>(colDP, dS_mn + o, dkmn + o, Tr::IDESC_DQ, ks > 0);
+          }
         }
       };
 
       bool ok = true;
       int g = 0, it = 0;
-      for (int j; ok && take_item(it, j); ++it) {
+      for (int j; ok && __all_sync(0xffffffffu, take_item(it, j)); ++it) {
         int bh, kb, i0, n_q;
         item(j, bh, kb, i0, n_q);
         (void)bh;
         (void)i0;
         const int b = it & 1;
         const uint64_t dK_k = kbuf(dK_k0, b), dK_mn = kbuf(dK_mn0, b);
-        ok = MBAR_WAIT(&bars->k_full[b], (it >> 1) & 1, abort_flag);
+        ok = MBAR_WAIT_WARP(&bars->k_full[b], (it >> 1) & 1, abort_flag);
         if (ok && n_q > 0)
-          ok = MBAR_WAIT(&bars->q_full[g & 1], (g >> 1) & 1, abort_flag) &&
-               MBAR_WAIT(&bars->do_full, g & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->q_full[g & 1], (g >> 1) & 1, abort_flag) &&
+               MBAR_WAIT_WARP(&bars->do_full, g & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         if (n_q > 0) {
           mma_st(colS, dK_k, stg(dQ_k0, g & 1));
-          tc_commit(&bars->s_full);
+          commit(&bars->s_full);
           // dPᵀ(0) needs V, and the previous item's last dQ out of the dPᵀ columns
-          ok = MBAR_WAIT(&bars->v_full, it & 1, abort_flag);
-          if (ok && g > 0) ok = MBAR_WAIT(&bars->dq_empty, (g - 1) & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->v_full, it & 1, abort_flag);
+          if (ok && g > 0) ok = MBAR_WAIT_WARP(&bars->dq_empty, (g - 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
           mma_st(colDP, dV_k, dO_k);
-          tc_commit(&bars->dp_full);
-          if (n_q == 1) tc_commit(&bars->v_free);  // the item's last dPᵀ
+          commit(&bars->dp_full);
+          if (n_q == 1) commit(&bars->v_free);  // the item's last dPᵀ
         } else {
-          ok = MBAR_WAIT(&bars->v_full, it & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->v_full, it & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          tc_commit(&bars->v_free);
+          commit(&bars->v_free);
         }
         // dV and dK restart from zero: the previous item's epilogue must
         // have read them.
         if (it > 0) {
-          ok = MBAR_WAIT(&bars->dkv_free, (it - 1) & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->dkv_free, (it - 1) & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
         }
@@ -461,41 +469,41 @@ __global__ void __launch_bounds__(512, 1)
         for (int i = 0; i < n_q; ++i) {
           const int gs = g + i, s = gs & 1;
           const bool more = i + 1 < n_q;
-          ok = MBAR_WAIT(&bars->p_ready, gs & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->p_ready, gs & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
           mma_dv(i > 0);
-          tc_commit(&bars->do_empty);
+          commit(&bars->do_empty);
           if (more) {
-            ok = MBAR_WAIT(&bars->q_full[s ^ 1], ((gs + 1) >> 1) & 1, abort_flag);
+            ok = MBAR_WAIT_WARP(&bars->q_full[s ^ 1], ((gs + 1) >> 1) & 1, abort_flag);
             tc_fence_after();
             if (!ok) break;
             mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
-            tc_commit(&bars->s_full);
+            commit(&bars->s_full);
           }
-          ok = MBAR_WAIT(&bars->ds_ready, gs & 1, abort_flag);
+          ok = MBAR_WAIT_WARP(&bars->ds_ready, gs & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
           // dQ first, so warpgroup 2 drains it while the tensor core runs dK.
           mma_dq(dK_mn);
-          tc_commit(&bars->dq_full);
-          if (!more) tc_commit(&bars->k_free[b]);  // the item's last product reading K
+          commit(&bars->dq_full);
+          if (!more) commit(&bars->k_free[b]);  // the item's last product reading K
           mma_dk(stg(dQ_mn0, s), i > 0);
-          tc_commit(&bars->q_empty[s]);
-          tc_commit(&bars->ds_free);
+          commit(&bars->q_empty[s]);
+          commit(&bars->ds_free);
           if (more) {
-            ok = MBAR_WAIT(&bars->dq_empty, gs & 1, abort_flag) &&
-                 MBAR_WAIT(&bars->do_full, (gs + 1) & 1, abort_flag);
+            ok = MBAR_WAIT_WARP(&bars->dq_empty, gs & 1, abort_flag) &&
+                 MBAR_WAIT_WARP(&bars->do_full, (gs + 1) & 1, abort_flag);
             tc_fence_after();
             if (!ok) break;
             mma_st(colDP, dV_k, dO_k);
-            tc_commit(&bars->dp_full);
-            if (i + 2 == n_q) tc_commit(&bars->v_free);  // the item's last dPᵀ
+            commit(&bars->dp_full);
+            if (i + 2 == n_q) commit(&bars->v_free);  // the item's last dPᵀ
           }
         }
         if (!ok) break;
-        if (n_q == 0) tc_commit(&bars->k_free[b]);
-        tc_commit(&bars->dkv_done);  // after the item's last dK (or at once if it has no steps)
+        if (n_q == 0) commit(&bars->k_free[b]);
+        commit(&bars->dkv_done);  // after the item's last dK (or at once if it has no steps)
         g += n_q;
       }
     }

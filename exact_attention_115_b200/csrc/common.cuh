@@ -150,6 +150,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // mbar_wait tagged with the call's source line (plus a per-file base set by
 // FA_SITE_BASE) so a timeout can be traced to its wait.
 #define MBAR_WAIT(bar, parity, abort_flag) mbar_wait(bar, parity, abort_flag, FA_SITE_BASE + __LINE__)
+// The same, by every lane of a converged warp, with a warp-uniform result.
+#define MBAR_WAIT_WARP(bar, parity, abort_flag) \
+  __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag, FA_SITE_BASE + __LINE__))
 
 // ------------------------------------------------------------------ TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -278,6 +281,18 @@ __device__ __forceinline__ int keys_of(const int* kv_len, int bh, int H, int Nk)
 }
 
 // ------------------------------------------------------------------ tcgen05
+// True in exactly one lane of the calling warp (elect.sync over all 32 lanes,
+// which must all execute it).  The MMA-issuing warps run their loops with the
+// whole warp, so descriptor arithmetic stays warp-uniform, and only the
+// elected lane issues each tcgen05.mma / tcgen05.commit.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
   asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                    smem_u32(dst_smem)),

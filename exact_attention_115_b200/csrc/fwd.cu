@@ -296,7 +296,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
   } else if (warp == Tr::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
     regs_dec<Tr::REGS_OTHER>();
-    if (lane == 0) {
+    // The whole warp runs the loop (warp-uniform waits and descriptor
+    // arithmetic); the elected lane issues the MMAs and commits.
+    {
+      const bool leader = elect_one();
       const uint32_t tS[2] = {tmem, tmem + 128};
       const uint32_t tO[2] = {tmem + 128 * Tr::TILES, tmem + 128 * Tr::TILES + D};
       const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
@@ -313,7 +316,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
         for (int ks = 0; ks < D / Tr::KSTEP; ++ks) {
           constexpr int kChunk16 = Tr::CHUNK / 16;
           const uint64_t o = uint64_t((ks >> 2) * kChunk16 + (ks & 3) * 2);
-          mma_ss<TF32>(tS[t], da + o, db + o, Tr::IDESC_QK, ks > 0);
+          if (leader) mma_ss<TF32>(tS[t], da + o, db + o, Tr::IDESC_QK, ks > 0);
         }
       };
       auto issue_pv = [&](int t, int slot, bool acc) {
@@ -325,76 +328,79 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
         for (int ks = 0; ks < Tr::BN / Tr::KSTEP; ++ks) {
           const uint64_t o = TF32 ? uint64_t((ks >> 2) * (D * 8) + (ks & 3) * 2)
                                   : uint64_t(ks * Tr::KSTEP * 8);
-          mma_ts<TF32>(tO[t], tS[t] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
+          if (leader) mma_ts<TF32>(tO[t], tS[t] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
         }
       };
+      auto commit = [&](uint64_t* bar) {
+        if (leader) tc_commit(bar);
+      };
       auto kv_wait = [&](int i) {
-        return MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
+        return MBAR_WAIT_WARP(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       };
 
       if constexpr (Tr::TILES == 1) {
         // One tile: S(j), then (once the softmax has written P(j)) P(j)·V(j)
         // and S(j+1) into the same columns, in issue order after P·V read P.
-        bool ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+        bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
         tc_fence_after();
         if (ok) issue_qk(0, 0);
-        tc_commit(&bars->s_full[0]);
-        tc_commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
+        commit(&bars->s_full[0]);
+        commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
         for (int j = 0; j < n_kv && ok; ++j) {
           const int iv = 2 * j + 1, ik = 2 * j + 2;
           const int sv = iv % Tr::NS, sk = ik % Tr::NS;
-          ok = kv_wait(iv) && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
+          ok = kv_wait(iv) && MBAR_WAIT_WARP(&bars->p_full[0], j & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
           issue_pv(0, sv, j > 0);
-          tc_commit(&bars->o_full[0]);
-          tc_commit(&bars->kv_empty[sv]);
+          commit(&bars->o_full[0]);
+          commit(&bars->kv_empty[sv]);
           if (j + 1 < n_kv) {
             ok = kv_wait(ik);
             tc_fence_after();
             if (!ok) break;
             issue_qk(0, sk);
-            tc_commit(&bars->s_full[0]);
-            tc_commit(&bars->kv_empty[sk]);
+            commit(&bars->s_full[0]);
+            commit(&bars->kv_empty[sk]);
           }
         }
       } else {
-      bool ok = MBAR_WAIT(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+      bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
       tc_fence_after();
       if (ok) issue_qk(0, 0);
-      tc_commit(&bars->s_full[0]);
-      ok = ok && MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
+      commit(&bars->s_full[0]);
+      ok = ok && MBAR_WAIT_WARP(&bars->q_full[1], 0, abort_flag);
       tc_fence_after();
       if (ok) issue_qk(1, 0);
-      tc_commit(&bars->s_full[1]);
-      tc_commit(&bars->kv_empty[0]);
+      commit(&bars->s_full[1]);
+      commit(&bars->kv_empty[0]);
       for (int j = 0; j < n_kv && ok; ++j) {
         const int iv = 2 * j + 1, ik = 2 * j + 2;
         const int sv = iv % Tr::NS, sk = ik % Tr::NS;
         ok = kv_wait(iv);
-        ok = ok && MBAR_WAIT(&bars->p_full[0], j & 1, abort_flag);
+        ok = ok && MBAR_WAIT_WARP(&bars->p_full[0], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         issue_pv(0, sv, j > 0);
-        tc_commit(&bars->o_full[0]);
+        commit(&bars->o_full[0]);
         const bool more = j + 1 < n_kv;
         if (more) {
           ok = kv_wait(ik);
           tc_fence_after();
           if (!ok) break;
           issue_qk(0, sk);
-          tc_commit(&bars->s_full[0]);
+          commit(&bars->s_full[0]);
         }
-        ok = MBAR_WAIT(&bars->p_full[1], j & 1, abort_flag);
+        ok = MBAR_WAIT_WARP(&bars->p_full[1], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         issue_pv(1, sv, j > 0);
-        tc_commit(&bars->o_full[1]);
-        tc_commit(&bars->kv_empty[sv]);
+        commit(&bars->o_full[1]);
+        commit(&bars->kv_empty[sv]);
         if (more) {
           issue_qk(1, sk);
-          tc_commit(&bars->s_full[1]);
-          tc_commit(&bars->kv_empty[sk]);
+          commit(&bars->s_full[1]);
+          commit(&bars->kv_empty[sk]);
         }
       }
       }
