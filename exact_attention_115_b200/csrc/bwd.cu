@@ -79,7 +79,13 @@ struct BwdTraits {
   static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
   static constexpr int BM = 128;                     // query rows per step
   static constexpr int CWC = BM / 2;                 // query columns per compute warpgroup
-  static constexpr bool DQ_T = D == 128;             // dQᵀ = Kᵀ dSᵀ (else dQ = dS K)
+  // d = 128: dQᵀ = Kᵀ dSᵀ with d on the TMEM lanes, so that a warp adds one
+  // 128-byte line of the accumulator per query row.  (dQ = dS K with rows on
+  // the lanes and four-wide reductions of each thread's row measured 30 %
+  // slower: the L2 takes reductions per request, and 16-byte requests
+  // scattered over 32 rows are 8 times as many as 128-byte lines.)
+  static constexpr bool DQ_T = D == 128;
+  static constexpr bool DQ_STAGED = D == 64;           // dQ staged in smem, TMA tensor reduce-add
   static constexpr int KV_TILE = BN * D * ES;        // bytes of the K (or V) tile
   static constexpr int KV_CHUNK = BN * 128;          // one 128-byte column block of it
   static constexpr int Q_TILE = BM * D * ES;         // bytes of a Q (or dO) tile
@@ -88,7 +94,7 @@ struct BwdTraits {
   // dQ staging (d = 64 only): the whole [BM × 64] fp32 tile (32 KB) goes to
   // shared memory as two swizzled halves and out with two tensor reduce-adds;
   // d = 128 reduces dQᵀ from registers and needs no staging.
-  static constexpr int DQ_STAGE = DQ_T ? 0 : BM * D * 4;
+  static constexpr int DQ_STAGE = DQ_STAGED ? BM * D * 4 : 0;
   // shared-memory offsets (all 1024-aligned).  K is double buffered (the
   // next work item's K loads while this item runs); Q is double buffered
   // (the next step's Sᵀ needs it while this step's dK still reads the
@@ -245,7 +251,7 @@ __global__ void __launch_bounds__(512, 1)
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
-    if constexpr (!Tr::DQ_T) tma_prefetch_desc(&tmdQ);
+    if constexpr (Tr::DQ_STAGED) tma_prefetch_desc(&tmdQ);
   }
   tc_fence_before();
   __syncthreads();
@@ -626,14 +632,20 @@ __global__ void __launch_bounds__(512, 1)
         const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
         for (int c = 0; c < CWC; c += 32) {
-          // one 32-column TMEM load per chunk (measured faster here than
+          // −D of the chunk's 32 query columns first, so that the
+          // shared-memory loads run during the TMEM load (which, like every
+          // tcgen05 wait, orders memory, so the compiler cannot hoist them);
+          // then one 32-column TMEM load per chunk (measured faster here than
           // loading all CWC columns before the arithmetic)
+          float4 ndc[8];
+#pragma unroll
+          for (int e4 = 0; e4 < 8; ++e4) ndc[e4] = sD4[(c >> 2) + e4];
           tmem_ld32(tDP + cw * CWC + c, *reinterpret_cast<uint32_t(*)[32]>(u + c));
           tmem_ld_wait();
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 32; e += 4) {
-            const float4 nd = sD4[(c + e) >> 2];
+            const float4 nd = ndc[e >> 2];
 #pragma unroll
             for (int h2 = 0; h2 < 2; ++h2) {
               const int q = c + e + 2 * h2;
