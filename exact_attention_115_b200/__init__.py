@@ -24,8 +24,10 @@ FA_FP32, FA_BF16, FA_FP16 = 0, 1, 2
 FA_DECODE_NOALLOC_SCRATCH_BYTES = 8 << 20  # include/fa.h
 FA_OK, FA_ERR_INVALID, FA_ERR_UNSUPPORTED, FA_ERR_WORKSPACE, FA_ERR_CUDA, FA_ERR_TIMEOUT = (
     0, -1, -2, -3, -4, -5)
+FA_ERR_BOUNDS = -6  # debug builds only
 STATUS_NAMES = {0: "FA_OK", -1: "FA_ERR_INVALID", -2: "FA_ERR_UNSUPPORTED",
-                -3: "FA_ERR_WORKSPACE", -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT"}
+                -3: "FA_ERR_WORKSPACE", -4: "FA_ERR_CUDA", -5: "FA_ERR_TIMEOUT",
+                -6: "FA_ERR_BOUNDS"}
 
 # Every symbol include/fa.h declares: name -> (restype, argtypes)
 _VP, _I, _F, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t

@@ -509,6 +509,7 @@ int fa_status(void* stream) {
   if (take_error_decode(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
   if (site != 0) g_last_site = site;
   if (word & 2) return FA_ERR_CUDA;  // a kernel found its shared memory misaligned (kErrLayout)
+  if (word & 4) return FA_ERR_BOUNDS;  // a debug build's index check failed (kErrBounds)
   if (word != 0) return FA_ERR_TIMEOUT;
   return FA_OK;
 }
@@ -532,6 +533,10 @@ int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
              : FA_ERR_CUDA;
 }
 
+#ifdef FA_DEBUG
+const char* fa_version(void) { return "fa-b200 0.1 (sm_100a, debug index checks)"; }
+#else
 const char* fa_version(void) { return "fa-b200 0.1 (sm_100a)"; }
+#endif
 
 }  // extern "C"

@@ -49,7 +49,25 @@ constexpr unsigned long long kWaitLimitNs = 2000000000ull;  // 2 s
 enum : int {
   kErrTimeout = 1,  // a bounded wait expired
   kErrLayout = 2,   // a kernel found its dynamic shared memory misaligned and did nothing
+  kErrBounds = 4,   // debug builds: an index check failed (the access was skipped)
 };
+
+// Index checks of the debug build (FA_DEBUG): FA_INBOUNDS(cond) is true when
+// cond holds; otherwise it records kErrBounds and the check's site (file
+// base + line) in the device error word and is false, and the caller skips
+// the access.  Release builds compile it to `true`.
+__device__ __forceinline__ bool fa_inbounds(bool ok, int site) {
+  if (!ok) {
+    atomicOr(&g_fa_error, kErrBounds);
+    atomicCAS(&g_fa_site, 0, site);
+  }
+  return ok;
+}
+#ifdef FA_DEBUG
+#define FA_INBOUNDS(cond) fa_inbounds(bool(cond), FA_SITE_BASE + __LINE__)
+#else
+#define FA_INBOUNDS(cond) true
+#endif
 
 constexpr float kLn2 = 0.6931471805599453f;
 

@@ -72,7 +72,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
   // this part's keys, cut at the batch element's key-padding length (a part
   // past it is empty: L_part = -inf, weight 0 in the combine)
   const int k_begin = part * p.keys_per_split;
-  const int k_end = min(keys_of(p.kv_len, bh, p.H, p.Nk), k_begin + p.keys_per_split);
+  int k_end = min(keys_of(p.kv_len, bh, p.H, p.Nk), k_begin + p.keys_per_split);
+  if (!FA_INBOUNDS(part < p.splits && bh < p.BH && (k_end <= k_begin || k_begin < p.Nk))) k_end = k_begin;
 
   // q slice, pre-multiplied by scale·log2(e) so scores come out in log2 units.
   float q[8];
@@ -160,6 +161,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
       }
     }
     const size_t idx = size_t(bh) * p.splits + part;
+    if (!FA_INBOUNDS(part < p.splits && bh < p.BH)) continue;
     p.Opart[idx * D + c] = lt > 0.f ? o / lt : 0.f;
     if (c == 0) p.Lpart[idx] = lt > 0.f ? (M + lg2(lt)) * kLn2 : -INFINITY;
   }
@@ -169,6 +171,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 template <typename T, int D>
 __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
   const int bh = blockIdx.x, c = threadIdx.x;
+  if (!FA_INBOUNDS(bh < p.BH && c < D)) return;
   const float* Lp = p.Lpart + size_t(bh) * p.splits;
   const float* Op = p.Opart + size_t(bh) * p.splits * D;
   float M = -INFINITY;

@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
         if (lane == 0) mbar_arrive(bar);
       } else if (lane == 0) {
         const CUtensorMap* map = which == 0 ? &tmQ : which == 1 ? &tmK : &tmV;
+        // (a tile may start past the end only by the CTA's second Q tile:
+        // TMA fills its rows with zeros)
+        if (!FA_INBOUNDS(bh < p.B * p.H && row >= 0 && row < (which == 0 ? p.Nq + 128 : p.Nk))) return;
         mbar_arrive_expect_tx(bar, Tr::TILE);
 #pragma unroll
         for (int c = 0; c < Tr::DC; ++c)
@@ -437,7 +440,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 #pragma unroll
         for (int v = 0; v < Tr::BN / 8; ++v) {
           const int col = j * Tr::BN + 8 * v;
-          bv[v] = brow ? load8_16bit(brow + col, p.Nk - col) : make_uint4(0u, 0u, 0u, 0u);
+          bv[v] = brow && FA_INBOUNDS(col < p.Nk || p.Nk - col <= 0)
+                      ? load8_16bit(brow + col, p.Nk - col)
+                      : make_uint4(0u, 0u, 0u, 0u);
         }
       }
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
@@ -626,7 +631,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
         }
         fence_async_smem();
       }
-      if (live)
+      if (live && FA_INBOUNDS(bh < p.B * p.H && qi < p.Nq))
         p.L[size_t(bh) * p.Nq + qi] =
             row_sum > 0.f ? (m_ref + lg2(row_sum)) * kLn2 : -INFINITY;
     }
@@ -634,7 +639,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
       // The tile's 128 rows are staged: one thread stores its D/64 column
       // blocks (rows past Nq are clipped by the tensor map) and waits until
       // TMA has read them before the CTA may exit.
-      if (named_bar_and(1 + t, 128, ok) && r == 0) {
+      if (named_bar_and(1 + t, 128, ok) && r == 0 &&
+          FA_INBOUNDS(bh < p.B * p.H && tile_first_row < p.Nq + 128)) {
 #pragma unroll
         for (int blk = 0; blk < Tr::DC; ++blk)
           tma_store_bh(&tmO, GEN && ((p.map4d >> 3) & 1), smem + t * Tr::TILE + blk * Tr::CHUNK, blk * Tr::AW,

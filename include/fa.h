@@ -58,7 +58,9 @@ typedef enum {
                               backward with B*H > 65535 */
   FA_ERR_WORKSPACE = -3,   /* workspace pointer null or smaller than the query says */
   FA_ERR_CUDA = -4,        /* a CUDA runtime error at launch or in fa_status */
-  FA_ERR_TIMEOUT = -5      /* a kernel's bounded wait expired (reported by fa_status) */
+  FA_ERR_TIMEOUT = -5,     /* a kernel's bounded wait expired (reported by fa_status) */
+  FA_ERR_BOUNDS = -6       /* debug builds only: a kernel index check failed (reported by
+                              fa_status; the access was skipped) */
 } fa_status_t;
 
 /* Forward.  Writes O [B,H,Nq,d] (dtype) and L [B,H,Nq] (float32, natural
@@ -237,13 +239,19 @@ int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, floa
 /* Synchronises `stream`, then returns and clears the device error word:
  * FA_OK, FA_ERR_TIMEOUT if a kernel's bounded wait expired, FA_ERR_CUDA if
  * the stream reports a CUDA error or a kernel found its shared memory
- * misaligned (it then did nothing). */
+ * misaligned (it then did nothing), and, in a library built with FA_DEBUG,
+ * FA_ERR_BOUNDS if a kernel found an index outside its buffer (the access
+ * was skipped; fa_last_timeout_site names the check).  The debug build
+ * (libfa_b200_debug.so, same ABI) checks every plain global access and TMA
+ * coordinate of the kernels against the buffer it addresses, in place of a
+ * memory checker. */
 int fa_status(void* stream);
 
-/* Diagnostic: identifies the first kernel wait that timed out among those
- * fa_status has reported (10000 + line in the forward kernel file, 20000 +
- * line in the backward file, 30000 + line in the decode file); 0 if none
- * has.  No counterpart on the pages. */
+/* Diagnostic: identifies the first kernel wait that timed out (or, in a
+ * debug build, the first failed index check) among those fa_status has
+ * reported (10000 + line in the forward kernel file, 20000 + line in the
+ * backward file, 30000 + line in the decode file); 0 if none has.  No
+ * counterpart on the pages. */
 int fa_last_timeout_site(void);
 
 /* Measurement hook (no counterpart on the pages, which only say to profile
