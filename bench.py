@@ -51,20 +51,21 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_traffic(kernel: str, sources):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel's source changed since that capture (hash mismatch)."""
+def kernel_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary
+    (profiles/dram_traffic.json), or None when one of the kernel's sources
+    listed there changed since that capture (sha256 mismatch)."""
     import hashlib
 
     try:
         with open(os.path.join(ROOT, "profiles", "dram_traffic.json")) as f:
             rec = json.load(f)[kernel]
+        m = hashlib.sha256()
+        for p in rec["sources"]:
+            with open(os.path.join(ROOT, p), "rb") as f:
+                m.update(f.read())
     except (OSError, KeyError, ValueError):
         return None
-    m = hashlib.sha256()
-    for p in sources:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            m.update(f.read())
     return rec["bytes_per_launch"] if m.hexdigest() == rec["source_sha256"] else None
 
 
@@ -292,6 +293,39 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None):
                          "peak": peak, "unit": UNIT, "frac": main_tf / peak, "peak_kind": pk}}
 
 
+# Decode shape for kernel captures: the decode workload with B = 4 instead of
+# 32 (2.1 GB of K/V, far larger than L2, within a capture's memory budget);
+# its bytes per key row are those of the full workload.
+DECODE_PROFILE = W.Workload("decode_b4h32nk32768d128", 4, 32, 1, 32768, 128, False, "bf16",
+                            decode=True)
+
+
+def profile_case(name: str):
+    """Three launches of one kernel's case: the causal B8 H16 N2048 d128
+    forward or backward, or the reduced decode shape.  A capture skips the
+    first two launches of the kernel (``-s 2 -c 1``)."""
+    import exact_attention_115_b200 as fa
+
+    dev = torch.device("cuda", 0)
+    w = DECODE_PROFILE if name == "decode" else W.CAUSAL_2K
+    q, k, v, do = W.make_inputs(w, device=dev, with_grad=name == "bwd")
+    if name == "decode":
+        for _ in range(3):
+            fa.decode(q, k, v)
+    else:
+        O, L = fa.forward(q, k, v, causal=w.causal)
+        for _ in range(3 if name == "bwd" else 2):
+            if name == "bwd":
+                fa.backward(q, k, v, O, do, L, causal=w.causal)
+            else:
+                fa.forward(q, k, v, causal=w.causal, out=O, lse=L)
+    torch.cuda.synchronize(dev)
+    st = fa.status()
+    print(f"profile case {name}: {w.describe()} status {fa.STATUS_NAMES.get(st, st)}")
+    if st != fa.FA_OK:
+        raise SystemExit(1)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -304,7 +338,13 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads (B4 H16 N1024 d64, the 16K causal one, fp16)")
+    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode"],
+                    help="run one kernel's small profiling case three times and exit "
+                         "(the command an ncu capture wraps; nothing is timed)")
     args = ap.parse_args()
+    if args.profile_case:
+        profile_case(args.profile_case)
+        return
     w = W.CAUSAL_2K
     if args.impl == "reference":
         run_reference(args, w)
@@ -505,7 +545,9 @@ def main():
                   "unit": "GB/s", "l2": "17.2 GB of K/V per call, far larger than L2",
                   "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                "frac": gbs / hbm, "peak_kind": peak_kind,
-                               "traffic": None}}
+                               "traffic": kernel_traffic("decode_split_kernel"),
+                               "traffic_unit": "bytes per launch of decode_split_kernel "
+                                               "(ncu dram read+write, 8x a B=4 capture)"}}
         assert fa.status() == fa.FA_OK
 
     cpu = None
@@ -540,10 +582,9 @@ def main():
                      "peak": peak_bf16, "unit": "TFLOP/s", "frac": achieved_bwd / peak_bf16,
                      **peak_fracs(achieved_bwd, peaks),
                      "peak_kind": f"{peak_kind} {'sustained' if sustained else 'burst'} bf16",
-                     "fwd_kernel": {"achieved": achieved_fwd, **peak_fracs(achieved_fwd, peaks)},
-                     "traffic": kernel_traffic("bwd_main_kernel", (
-                         "exact_attention_115_b200/csrc/bwd.cu",
-                         "exact_attention_115_b200/csrc/common.cuh")),
+                     "fwd_kernel": {"achieved": achieved_fwd, **peak_fracs(achieved_fwd, peaks),
+                                    "traffic": kernel_traffic("fwd_kernel")},
+                     "traffic": kernel_traffic("bwd_main_kernel"),
                      "traffic_unit": "bytes per launch (ncu dram read+write)"},
         "e2e": e2e,
         "gpu_launches": 4 * K,

@@ -9,7 +9,9 @@
 //     query blocks, so dK and dV stay on chip and are written once.
 //   section "Warp Level 并行": dV = Pᵀ dO, dP = dO Vᵀ, dS = P ∘ (dP − D),
 //     dQ = dS K, dK = dSᵀ Q (with the scale on dQ and dK and
-//     D = rowsum(dO ∘ O), the exact softmax gradient).
+//     D = rowsum(dO ∘ O), the exact softmax gradient).  Here dS is kept
+//     unscaled in the products and the scale is applied once to the fp32
+//     results (dK in its epilogue, dQ in the finalise kernel).
 //   section "Sequence Parallel": dQ receives a contribution from every K/V
 //     block, so it is reduced across CTAs, either by atomic adds into one
 //     buffer or by one buffer per K/V block and a separate reduction kernel.
@@ -531,7 +533,6 @@ __global__ void __launch_bounds__(512, 1)
     const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const float sl2 = p.scale_log2;
-    const float scale = p.scale;
     const uint32_t tS = tmem + lane_off + Tr::COL_S;
     const uint32_t tDP = tmem + lane_off + Tr::COL_DP;
     bool ok = true;
@@ -629,15 +630,16 @@ __global__ void __launch_bounds__(512, 1)
         tc_fence_before();
         mbar_arrive(&bars->p_ready);
 
-        // ---- dS = P ∘ (dP − D) · scale, to shared memory (row = key, BM
-        // query values contiguous, 128-byte swizzled, 64 values per column
-        // block): the A operand of dK += dSᵀ Q and an operand of dQ.
+        // ---- dS = P ∘ (dP − D), to shared memory (row = key, BM query
+        // values contiguous, 128-byte swizzled, 64 values per column block):
+        // the A operand of dK += dSᵀ Q and an operand of dQ.  The softmax
+        // scale is left out here (one multiply per element fewer on the
+        // busiest warps) and applied to the fp32 dK and dQ sums.
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->dp_full, gs & 1, abort_flag));
         if (ok && gs >= 1)
           ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->ds_free, (gs - 1) & 1, abort_flag));
         tc_fence_after();
         if (!ok) break;
-        const uint64_t sc2 = pk2(scale, scale);
 #pragma unroll
         for (int c = 0; c < CWC; c += 32) {
           // −D of the chunk's 32 query columns first, so that the
@@ -670,7 +672,7 @@ __global__ void __launch_bounds__(512, 1)
                           h2 ? pk2(nd.z, nd.w) : pk2(nd.x, nd.y));
               }
               const float2 pq = ElemTraits<T>::unpack2(Pk[q >> 1]);
-              const float2 ds = upk2(fmul2(t, fmul2(pk2(pq.x, pq.y), sc2)));
+              const float2 ds = upk2(fmul2(t, pk2(pq.x, pq.y)));
               w[(e >> 1) + h2] = ElemTraits<T>::pack2(ds.x, ds.y);
             }
           }
@@ -810,9 +812,12 @@ __global__ void __launch_bounds__(512, 1)
               tc_fence_before();
               mbar_arrive(&bars->dkv_free);
             }
-            if (DROP && which == 0) {  // dV: the kept weights' 256/T factor
+            // dK: the softmax scale left out of dS; dV: the kept weights'
+            // 256/T factor under dropout
+            if (which == 1 || DROP) {
+              const float mul = which == 1 ? p.scale : p.drop.scale;
 #pragma unroll
-              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * p.drop.scale);
+              for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * mul);
             }
             if (live && FA_INBOUNDS(bh < p.B * p.H && krow < p.Nk)) {
 #pragma unroll
@@ -888,7 +893,8 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   }
 }
 
-// dQ = Σ (dQ accumulator or per-K/V-block partials), cast to the dtype.
+// dQ = scale · Σ (dQ accumulator or per-K/V-block partials), cast to the
+// dtype (the main kernel's dS leaves the softmax scale out).
 template <typename T, int D, bool CAUSAL, bool GEN>
 __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
@@ -917,6 +923,8 @@ __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
     acc[0] = x.x; acc[1] = x.y; acc[2] = x.z; acc[3] = x.w;
     acc[4] = y.x; acc[5] = y.y; acc[6] = y.z; acc[7] = y.w;
   }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) acc[k] *= p.scale;
   uint4 o;
   o.x = ElemTraits<T>::pack2(acc[0], acc[1]);
   o.y = ElemTraits<T>::pack2(acc[2], acc[3]);
