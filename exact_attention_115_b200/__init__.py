@@ -40,6 +40,7 @@ SIGNATURES = {
     "fa_bwd_ex": (_I, [_VP] * 9 + [_VP] * 8 + [_I, _I, _I, _I, _I, _I, _F, _I, _VP, _VP, _VP, _VP,
                                                _VP, _SZ, _VP]),
     "fa_set_bwd_dq_mode": (_I, [_I]),
+    "fa_set_bwd_dq_groups": (_I, [_I]),
     "fa_decode_workspace_bytes": (_SZ, [_I, _I, _I, _I, _I]),
     "fa_decode": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _VP]),
     "fa_decode_ex": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP, _VP, _SZ, _VP]),
@@ -220,10 +221,20 @@ def bwd_workspace_bytes(B, H, Nq, Nk, d, dtype=torch.bfloat16) -> int:
 
 
 def set_bwd_dq_mode(mode: int) -> int:
-    """0 auto, 1 reduce-add into one fp32 buffer, 2 per-K/V-block partials."""
+    """0 auto, 1 reduce-add into one fp32 buffer, 2 per-K/V-block partials,
+    3 reduce-add into G buffers (K/V block kb into buffer kb mod G; see
+    set_bwd_dq_groups).  Returns the previous mode."""
     rc = lib().fa_set_bwd_dq_mode(int(mode))
     if rc < 0:
         raise FAError("fa_set_bwd_dq_mode", rc)
+    return rc
+
+
+def set_bwd_dq_groups(groups: int) -> int:
+    """G, the buffer count of dQ mode 3 (1..16).  Returns the previous G."""
+    rc = lib().fa_set_bwd_dq_groups(int(groups))
+    if rc < 0:
+        raise FAError("fa_set_bwd_dq_groups", rc)
     return rc
 
 

@@ -16,7 +16,8 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
-std::atomic<int> g_dq_mode{0};  // 0 auto, 1 reduce-add, 2 partial buffers
+std::atomic<int> g_dq_mode{0};    // 0 auto, 1 reduce-add, 2 partial buffers, 3 grouped
+std::atomic<int> g_dq_groups{4};  // accumulators of mode 3
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_bwd_set_timing_events
 std::atomic<int> g_last_site{0};  // fa_last_timeout_site
 
@@ -119,7 +120,7 @@ struct BwdWorkspace {
   size_t d_off, l_off, dq_off, ctr_off, total;
 };
 
-BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
+BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode, int groups) {
   const size_t BH = size_t(B) * H;
   const size_t rows = size_t(bwd_pad_rows(Nq));
   const size_t nkv = (size_t(Nk) + 127) / 128;
@@ -127,7 +128,8 @@ BwdWorkspace bwd_layout(int B, int H, int Nq, int Nk, int d, int mode) {
   w.d_off = 0;
   w.l_off = round_up(BH * rows * sizeof(float), 256);
   w.dq_off = w.l_off + round_up(BH * rows * sizeof(float), 256);
-  const size_t dq = BH * rows * size_t(d) * sizeof(float) * (mode == 2 ? nkv : 1);
+  const size_t slabs = mode == 2 ? nkv : mode == 3 ? size_t(groups) : 1;
+  const size_t dq = BH * rows * size_t(d) * sizeof(float) * slabs;
   w.ctr_off = w.dq_off + round_up(dq, 256);  // work-item counter of the main kernel
   w.total = w.ctr_off + 256;
   return w;
@@ -285,13 +287,18 @@ int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B
 
 size_t fa_bwd_workspace_bytes(int B, int H, int Nq, int Nk, int d, int dtype) {
   if (check_common(B, H, Nq, Nk, d, 1.0f, dtype) != FA_OK) return 0;
-  return bwd_layout(B, H, Nq, Nk, d, effective_dq_mode(B, H, Nq, Nk, d)).total;
+  return bwd_layout(B, H, Nq, Nk, d, effective_dq_mode(B, H, Nq, Nk, d), g_dq_groups.load()).total;
 }
 
 int fa_set_bwd_dq_mode(int mode) {
-  if (mode < 0 || mode > 2) return FA_ERR_INVALID;
+  if (mode < 0 || mode > 3) return FA_ERR_INVALID;
   const int prev = g_dq_mode.exchange(mode);
   return prev;
+}
+
+int fa_set_bwd_dq_groups(int groups) {
+  if (groups < 1 || groups > 16) return FA_ERR_INVALID;
+  return g_dq_groups.exchange(groups);
 }
 
 int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -327,7 +334,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   if (bias && (!aligned16(bias) || !valid_layout(lbias, dtype))) return FA_ERR_INVALID;
   if (bias && dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
   const int mode = effective_dq_mode(B, H, Nq, Nk, d);
-  const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode);
+  const int groups = g_dq_groups.load();
+  const BwdWorkspace w = bwd_layout(B, H, Nq, Nk, d, mode, groups);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || ws_bytes < w.total)
     return FA_ERR_WORKSPACE;
   const int BH = B * H;
@@ -356,6 +364,7 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   p.scale_log2 = scale * 1.4426950408889634f;
   p.n_kblocks = (Nk + 127) / 128;
   p.dq_mode = mode;
+  p.dq_groups = groups;
   p.head_group = head_group_for(size_t(p.Nq_pad) * (size_t(d) * (2 * elem_size(dtype) + 4) + 8), BH);
   auto to_strides = [](const fa_layout* l) { return Strides{l->b, l->h, l->n}; };
   p.s_o = to_strides(lo);
@@ -366,10 +375,11 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   for (int i = 0; i < 5; ++i) p.map4d |= int(m4[i]) << i;  // Q 0, K 1, V 2, dO 4
   if (dtype != FA_FP32 && d == 64) {
     // The d = 64 kernel reduces each step's dQ tile into the fp32 accumulator
-    // (or stores it into its K/V block's partial) through a 2-D map over it:
-    // [rows, 64] fp32, boxes of 32 columns (128 bytes, 128-byte swizzle) by
-    // 128 rows.
-    const uint64_t rows = uint64_t(BH) * p.Nq_pad * (mode == 2 ? uint64_t(p.n_kblocks) : 1u);
+    // (or stores it into its K/V block's partial) through a 2-D map over the
+    // whole buffer: [rows, 64] fp32, boxes of 32 columns (128 bytes,
+    // 128-byte swizzle) by 128 rows.
+    const uint64_t slabs = mode == 2 ? uint64_t(p.n_kblocks) : mode == 3 ? uint64_t(groups) : 1u;
+    const uint64_t rows = uint64_t(BH) * p.Nq_pad * slabs;
     if (rows > uint64_t(INT32_MAX)) return FA_ERR_UNSUPPORTED;  // TMA row coordinates are int32
     EncodeTiledFn enc = encode_fn();
     cuuint64_t dims[2] = {cuuint64_t(d), cuuint64_t(rows)};

@@ -15,7 +15,11 @@
 //   section "Sequence Parallel": dQ receives a contribution from every K/V
 //     block, so it is reduced across CTAs, either by atomic adds into one
 //     buffer or by one buffer per K/V block and a separate reduction kernel.
-//     Both are implemented (dq_mode 1 and 2); mode 1 is the default.
+//     Both are implemented (dq_mode 1 and 2); mode 1 is the default.  The
+//     section's compromise, partial buffers shared by groups of K/V blocks
+//     with atomic adds inside a group, is mode 3: G fp32 accumulators, K/V
+//     block kb reduce-adding into accumulator kb mod G (so K/V blocks of one
+//     head that run at the same time add into different buffers).
 //
 // Kernels: bwd_preprocess (−D = −rowsum(dO ∘ O) and −L·log2e into padded
 // buffers, dQ accumulator cleared), bwd_main (below), bwd_dq_finalise
@@ -173,6 +177,16 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
   i0 = first / BM;
   const int nt = (Nq + BM - 1) / BM;
   n = max(0, nt - i0);
+}
+
+// The fp32 dQ buffer is S slabs of [B·H, Nq_pad, d]: one accumulator
+// (mode 1), one partial per K/V block (mode 2), or dq_groups accumulators
+// (mode 3).  K/V block kb writes slab dq_slab(p, kb).
+__device__ __forceinline__ int dq_slabs(const BwdParams& p) {
+  return p.dq_mode == 2 ? p.n_kblocks : p.dq_mode == 3 ? p.dq_groups : 1;
+}
+__device__ __forceinline__ int dq_slab(const BwdParams& p, int kb) {
+  return p.dq_mode == 2 ? kb : p.dq_mode == 3 ? kb % p.dq_groups : 0;
 }
 
 // GEN: some tensor has a general layout (4-D tensor maps or plain strided
@@ -721,10 +735,9 @@ __global__ void __launch_bounds__(512, 1)
           tmem_ld_wait();
           tc_fence_before();
           mbar_arrive(&bars->dq_empty);  // the dPᵀ columns may take the next dPᵀ
-          float* dst = p.dq_mode == 2
-                           ? p.dQacc + ((size_t(kb) * p.B * p.H + bh) * p.Nq_pad + q0) * D + r
-                           : p.dQacc + (size_t(bh) * p.Nq_pad + q0) * D + r;
-          if (!FA_INBOUNDS(bh < p.B * p.H && q0 + BM <= p.Nq_pad && (p.dq_mode != 2 || kb < p.n_kblocks))) {
+          const int slab = dq_slab(p, kb);
+          float* dst = p.dQacc + ((size_t(slab) * p.B * p.H + bh) * p.Nq_pad + q0) * D + r;
+          if (!FA_INBOUNDS(bh < p.B * p.H && q0 + BM <= p.Nq_pad && slab < dq_slabs(p))) {
           } else if (p.dq_mode == 2) {
 #pragma unroll
             for (int q = 0; q < BM; ++q) dst[q * D] = __uint_as_float(v[q]);
@@ -769,15 +782,14 @@ __global__ void __launch_bounds__(512, 1)
           }
           fence_async_smem();
           named_bar(1, 128);
-          if (leader &&
-              FA_INBOUNDS(bh < p.B * p.H && q0 + BM <= p.Nq_pad && (p.dq_mode != 2 || kb < p.n_kblocks))) {
-            // rows of the accumulator viewed as [rows, 64] fp32 (x = column, y = row)
+          const int slab = dq_slab(p, kb);
+          if (leader && FA_INBOUNDS(bh < p.B * p.H && q0 + BM <= p.Nq_pad && slab < dq_slabs(p))) {
+            // rows of the buffer viewed as [rows, 64] fp32 (x = column, y = row)
+            const int row = (slab * p.B * p.H + bh) * p.Nq_pad + q0;
             if (p.dq_mode == 2) {
-              const int row = (kb * p.B * p.H + bh) * p.Nq_pad + q0;
               tma_store_2d(&tmdQ, sdQ, 0, row);
               tma_store_2d(&tmdQ, sdQ + BM * 128, 32, row);
             } else {
-              const int row = bh * p.Nq_pad + q0;
               tma_reduce_add_2d(&tmdQ, sdQ, 0, row);
               tma_reduce_add_2d(&tmdQ, sdQ + BM * 128, 32, row);
             }
@@ -886,10 +898,14 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
     // bias are, as the padding rows do
     p.neg_Lsc[row] = lsc == -INFINITY ? -INFINITY : -lsc;
   }
-  if (p.dq_mode == 1) {
-    float4* z = reinterpret_cast<float4*>(p.dQacc + row * D + sl * 8);
-    z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-    z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.dq_mode != 2) {  // the accumulator(s) of modes 1 and 3 start from zero
+    const int n = p.dq_mode == 3 ? p.dq_groups : 1;
+    const size_t slab = size_t(p.B) * p.H * p.Nq_pad * D;
+    for (int s = 0; s < n; ++s) {
+      float4* z = reinterpret_cast<float4*>(p.dQacc + s * slab + row * D + sl * 8);
+      z[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+      z[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
 }
 
@@ -905,13 +921,16 @@ __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   if (q >= p.Nq || !FA_INBOUNDS(bh < p.B * p.H)) return;
   float acc[8];
   const size_t row = size_t(bh) * p.Nq_pad + q;
-  if (p.dq_mode == 2) {
+  if (p.dq_mode >= 2) {
+    // the partials of K/V blocks 0 .. last (mode 2), or the accumulators
+    // they added into (mode 3: block kb into kb mod G)
 #pragma unroll
     for (int k = 0; k < 8; ++k) acc[k] = 0.f;
     int last = p.n_kblocks - 1;
     if (CAUSAL) last = min(last, (q + p.Nk - p.Nq) / 128);
+    if (p.dq_mode == 3) last = min(last, p.dq_groups - 1);
     const size_t stride = size_t(p.B) * p.H * p.Nq_pad * D;
-    for (int j = 0; j <= last && FA_INBOUNDS(j < p.n_kblocks); ++j) {
+    for (int j = 0; j <= last && FA_INBOUNDS(j < dq_slabs(p)); ++j) {
       const float4* src = reinterpret_cast<const float4*>(p.dQacc + j * stride + row * D + sl * 8);
       const float4 x = src[0], y = src[1];
       acc[0] += x.x; acc[1] += x.y; acc[2] += x.z; acc[3] += x.w;

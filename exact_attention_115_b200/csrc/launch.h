@@ -77,13 +77,15 @@ struct BwdParams {
   void* dV;
   float* neg_D;    // [B*H, Nq_pad] -rowsum(dO * O), padded rows zero
   float* neg_Lsc;  // [B*H, Nq_pad] -L * log2(e), padded rows -inf
-  float* dQacc;   // [B*H, Nq_pad, d] fp32 (mode 1) or [nkv, B*H, Nq_pad, d] (mode 2)
+  float* dQacc;   // fp32 [S, B*H, Nq_pad, d]: S = 1 (mode 1), nkv (mode 2), dq_groups (mode 3)
   int* item_ctr;  // work items handed out beyond the first wave (zeroed by the preprocess)
   int B, H, Nq, Nk, Nq_pad;
   float scale;        // softmax scale
   float scale_log2;   // scale * log2(e)
   int n_kblocks;      // ceil(Nk / 128)
-  int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials
+  int dq_mode;        // 1 = reduce-add into one buffer, 2 = per-K/V-block partials,
+                      // 3 = reduce-add into dq_groups buffers (K/V block kb into kb mod dq_groups)
+  int dq_groups;      // buffers of mode 3 (1..16)
   int head_group;     // heads per launch-order group (see head_group_for)
   Strides s_o, s_do, s_dq, s_dk, s_dv;  // plain (non-TMA) accesses; Q, K, V, dO go through tensor maps
   int map4d;  // bit per tensor map (Q 0, K 1, V 2, dO 4): 4-D (d, N, H, B), else 3-D (d, N, B·H)

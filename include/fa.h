@@ -172,11 +172,21 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
 
 /* How fa_bwd reduces the dQ contributions of the different K/V blocks:
  *   0 = automatic (the measured faster strategy for the shape),
- *   1 = fp32 bulk reductions (red.add) into one accumulator,
- *   2 = one fp32 partial buffer per K/V block, then a reduction kernel.
- * The 51CTO notes, section "Sequence Parallel", describe both.  Returns the
- * previous mode, or FA_ERR_INVALID for an unknown mode.  Process-wide. */
+ *   1 = fp32 reductions (red.add) into one accumulator,
+ *   2 = one fp32 partial buffer per K/V block, then a reduction kernel,
+ *   3 = fp32 reductions into G accumulators, K/V block kb adding into
+ *       accumulator kb mod G (G from fa_set_bwd_dq_groups), then the same
+ *       reduction kernel over the G buffers.
+ * The 51CTO notes, section "Sequence Parallel", describe 1 and 2, and mode 3
+ * is their compromise (partial buffers shared by groups of K/V blocks, with
+ * atomic adds inside a group).  The workspace grows with the buffers: ×1, ×
+ * the K/V block count, ×G.  Returns the previous mode, or FA_ERR_INVALID for
+ * an unknown mode.  Process-wide; fa_bwd_workspace_bytes follows it. */
 int fa_set_bwd_dq_mode(int mode);
+
+/* G, the accumulator count of dQ mode 3 (1 to 16; 4 initially).  Returns
+ * the previous G, or FA_ERR_INVALID outside 1..16.  Process-wide. */
+int fa_set_bwd_dq_groups(int groups);
 
 /* Bytes of workspace fa_decode needs for `num_splits` parts (0 = the count
  * fa_decode would choose itself). */

@@ -80,15 +80,25 @@ def test_bwd_workspace_query(lib):
 
 def test_bwd_dq_modes_change_workspace(lib):
     prev = lib.fa_set_bwd_dq_mode(2)
+    prev_g = lib.fa_set_bwd_dq_groups(3)
     try:
         n2 = lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16)
         lib.fa_set_bwd_dq_mode(1)
         n1 = lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16)
-        assert n2 > n1 * 4  # 8 K/V blocks of partial buffers vs one accumulator
-        assert lib.fa_set_bwd_dq_mode(3) == fa.FA_ERR_INVALID
+        assert lib.fa_set_bwd_dq_mode(3) == 1
+        n3 = lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16)
+        acc = 1024 * 64 * 4  # one fp32 dQ buffer
+        assert n2 - n1 == 7 * acc  # 8 K/V blocks of partial buffers vs one accumulator
+        assert n3 - n1 == 2 * acc  # 3 accumulators vs one
+        assert lib.fa_set_bwd_dq_groups(5) == 3
+        assert lib.fa_bwd_workspace_bytes(1, 1, 1024, 1024, 64, fa.FA_BF16) - n1 == 4 * acc
+        for bad in (0, 17, -1):
+            assert lib.fa_set_bwd_dq_groups(bad) == fa.FA_ERR_INVALID
+        assert lib.fa_set_bwd_dq_mode(4) == fa.FA_ERR_INVALID
         assert lib.fa_set_bwd_dq_mode(-1) == fa.FA_ERR_INVALID
     finally:
         lib.fa_set_bwd_dq_mode(prev)
+        lib.fa_set_bwd_dq_groups(prev_g)
 
 
 def bwd(lib, ws=FAKE, ws_bytes=1 << 40, **kw):

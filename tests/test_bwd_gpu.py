@@ -20,11 +20,15 @@ def fa():
     return fa
 
 
-@pytest.fixture(params=[1, 2], ids=["dq_reduce_add", "dq_partials"])
+@pytest.fixture(params=[1, 2, 3], ids=["dq_reduce_add", "dq_partials", "dq_grouped3"])
 def dq_mode(request, fa):
+    """Every dQ strategy; the grouped one with G = 3 buffers, so that K/V
+    block counts not divisible by G leave groups of unequal sizes."""
     prev = fa.set_bwd_dq_mode(request.param)
+    prev_g = fa.set_bwd_dq_groups(3)
     yield request.param
     fa.set_bwd_dq_mode(prev)
+    fa.set_bwd_dq_groups(prev_g)
 
 
 def run_bwd(fa, B, H, Nq, Nk, d, causal, dtype="bf16", seed=0, q_mult=1.0):

@@ -81,15 +81,17 @@ def test_causal_2k_forward_every_element(fa, causal_2k):
     check_fwd(O, L, O_ref, L_ref, f"{w.name}, all 128 heads")
 
 
-@pytest.mark.parametrize("mode", [1, 2], ids=["dq_reduce_add", "dq_partials"])
+@pytest.mark.parametrize("mode", [1, 2, 3], ids=["dq_reduce_add", "dq_partials", "dq_grouped4"])
 def test_causal_2k_backward_every_element(fa, causal_2k, mode):
     w, (q, k, v, do), (_, _, dq_ref, dk_ref, dv_ref) = causal_2k
     prev = fa.set_bwd_dq_mode(mode)
+    prev_g = fa.set_bwd_dq_groups(4)
     try:
         O, L = _forward_canary(fa, q, k, v, w)
         dq, dk, dv = _backward_canary(fa, q, k, v, O, do, L, w)
     finally:
         fa.set_bwd_dq_mode(prev)
+        fa.set_bwd_dq_groups(prev_g)
     what = f"{w.name}, all 128 heads, dq mode {mode}"
     for g, r, n in ((dq, dq_ref, "dQ"), (dk, dk_ref, "dK"), (dv, dv_ref, "dV")):
         check_grad(g, r, n, what)
@@ -117,6 +119,19 @@ def test_long_16k_every_element(fa):
                      list(LONG_BWD_HEADS))
     for h, (dq_ref, dk_ref, dv_ref, _) in zip(LONG_BWD_HEADS, bwd):
         what = f"{w.name}, head {h}, every row"
+        check_grad(dq[0, h], dq_ref, "dQ", what)
+        check_grad(dk[0, h], dk_ref, "dK", what)
+        check_grad(dv[0, h], dv_ref, "dV", what)
+
+    # the grouped dQ strategy (8 accumulators) on the same inputs
+    prev, prev_g = fa.set_bwd_dq_mode(3), fa.set_bwd_dq_groups(8)
+    try:
+        dq, dk, dv = _backward_canary(fa, q, k, v, O, do, L, w)
+    finally:
+        fa.set_bwd_dq_mode(prev)
+        fa.set_bwd_dq_groups(prev_g)
+    for h, (dq_ref, dk_ref, dv_ref, _) in zip(LONG_BWD_HEADS, bwd):
+        what = f"{w.name}, head {h}, every row, dq mode 3 (G = 8)"
         check_grad(dq[0, h], dq_ref, "dQ", what)
         check_grad(dk[0, h], dk_ref, "dK", what)
         check_grad(dv[0, h], dv_ref, "dV", what)
