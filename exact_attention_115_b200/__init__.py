@@ -47,6 +47,7 @@ SIGNATURES = {
     "fa_status": (_I, [_VP]),
     "fa_bwd_set_timing_events": (_I, [_VP, _VP]),
     "fa_last_timeout_site": (_I, []),
+    "fa_last_cuda_error": (_I, []),
     "fa_decode_noalloc": (_I, [_VP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "fa_selftest_wait_timeout": (_I, [ctypes.c_uint, _VP]),
     "fa_version": (ctypes.c_char_p, []),
@@ -167,7 +168,13 @@ def _on(device):
 
 def _raise(fn, code):
     if code != FA_OK:
-        raise FAError(fn, code)
+        err = FAError(fn, code)
+        if code == FA_ERR_CUDA:  # name the CUDA error behind it
+            cu = int(lib().fa_last_cuda_error())
+            err.cuda_error = cu
+            err.args = (f"{err.args[0]} (CUDA error {cu}"
+                        + (f", tensor-map encoding CUresult {cu - 100000})" if cu >= 100000 else ")"),)
+        raise err
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,

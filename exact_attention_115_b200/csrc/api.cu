@@ -20,6 +20,25 @@ std::atomic<int> g_dq_mode{0};    // 0 auto, 1 reduce-add, 2 partial buffers, 3 
 std::atomic<int> g_dq_groups{4};  // accumulators of mode 3
 cudaEvent_t g_ev_start = nullptr, g_ev_stop = nullptr;  // fa_bwd_set_timing_events
 std::atomic<int> g_last_site{0};  // fa_last_timeout_site
+std::atomic<int> g_last_cuda{0};  // fa_last_cuda_error
+
+// FA_ERR_CUDA, remembering the code behind it (a cudaError_t, or 100000 +
+// the CUresult of a failed tensor-map encoding) for fa_last_cuda_error.
+int cuda_fail(int code) {
+  g_last_cuda = code;
+  return FA_ERR_CUDA;
+}
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : cuda_fail(int(e)); }
+
+// Tensor-map encoding is a driver call, which needs a current context on the
+// calling thread; a thread that has made no runtime call yet (an autograd
+// worker, a fresh host thread) has none.  cudaSetDevice makes the current
+// device's primary context current on this thread.
+cudaError_t ensure_context() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  return e != cudaSuccess ? e : cudaSetDevice(dev);
+}
 
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                    const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -59,7 +78,10 @@ CUtensorMapDataType tma_type(int dtype) {
 bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int H, int B,
               const fa_layout& l, int box_rows, bool* is4d) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    g_last_cuda = int(cudaErrorSymbolNotFound);
+    return false;
+  }
   const int es = elem_size(dtype);
   const bool merge = l.b == (long long)H * l.h;
   *is4d = !merge;
@@ -70,6 +92,7 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int H, i
   CUresult r = enc(m, tma_type(dtype), merge ? 3 : 4, const_cast<void*>(ptr), dims, strides, box,
                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) g_last_cuda = 100000 + int(r);
   return r == CUDA_SUCCESS;
 }
 
@@ -254,6 +277,8 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
     a.params.s_bias = Strides{lbias->b, lbias->h, lbias->n};
     a.params.bias_mul = 1.0f / scale;
   }
+  st = from_cuda(ensure_context());
+  if (st != FA_OK) return st;
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
@@ -271,11 +296,12 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   a.params.Nq = Nq;
   a.params.Nk = Nk;
   a.params.scale_log2 = scale * 1.4426950408889634f;
-  const int rows = fwd_rows_per_cta(dtype, d);
+  a.params.tiles = fwd_tiles_for(dtype, d, Nq, Nk, causal != 0, !drop.t4 && !bias);
+  const int rows = 128 * a.params.tiles;
   a.params.n_qblocks = (Nq + rows - 1) / rows;
   a.params.head_group = head_group_for(size_t(Nk) * d * 2 * elem_size(dtype), BH);
   a.stream = static_cast<cudaStream_t>(stream);
-  return launch_fwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return from_cuda(launch_fwd(dtype, d, causal != 0, a));
 }
 
 int fa_fwd(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nq,
@@ -344,6 +370,8 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   const int bm = bwd_block_rows(d);
   // (the fp32 path stages its operands without TMA)
   // (dK and dV are written with plain stores: their strides go to the kernel)
+  st = from_cuda(ensure_context());
+  if (st != FA_OK) return st;
   bool m4[5] = {false, false, false, false, false};
   if (dtype != FA_FP32 &&
       (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, bm, &m4[0]) ||
@@ -386,11 +414,11 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
     cuuint64_t strides[1] = {cuuint64_t(d) * sizeof(float)};
     cuuint32_t box[2] = {32, 128};
     cuuint32_t estr[2] = {1, 1};
-    if (!enc || enc(&a.tmdQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.dQacc, dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-      return FA_ERR_CUDA;
+    if (!enc) return cuda_fail(int(cudaErrorSymbolNotFound));
+    const CUresult r = enc(&a.tmdQ, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.dQacc, dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(100000 + int(r));
   }
   p.drop = drop;
   p.kv_len = kv_len;
@@ -402,7 +430,7 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;
   a.ev_stop = g_ev_stop;
-  return launch_bwd(dtype, d, causal != 0, a) == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  return from_cuda(launch_bwd(dtype, d, causal != 0, a));
 }
 
 int fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
@@ -456,9 +484,7 @@ int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L,
   p.scale_log2 = scale * 1.4426950408889634f;
   p.H = H;
   p.kv_len = kv_len;
-  return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FA_OK
-             : FA_ERR_CUDA;
+  return from_cuda(launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)));
 }
 
 int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H, int Nk,
@@ -492,7 +518,8 @@ int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, floa
   s = (Nk + kps - 1) / kps;
   if (need_for(s) > cap) return FA_ERR_WORKSPACE;  // beyond the built-in scratch
   void* scratch = nullptr;
-  if (decode_scratch_ptr(&scratch) != cudaSuccess) return FA_ERR_CUDA;
+  st = from_cuda(decode_scratch_ptr(&scratch));
+  if (st != FA_OK) return st;
   DecodeParams p;
   p.Q = Q; p.K = K; p.V = V; p.O = O; p.L = L;
   p.Opart = static_cast<float*>(scratch);
@@ -505,18 +532,16 @@ int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, floa
   p.scale_log2 = scale * 1.4426950408889634f;
   p.H = H;
   p.kv_len = nullptr;
-  return launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FA_OK
-             : FA_ERR_CUDA;
+  return from_cuda(launch_decode(dtype, d, p, static_cast<cudaStream_t>(stream)));
 }
 
 int fa_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return FA_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(int(e));
   int word = 0, site = 0;
-  if (take_error_fwd(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
-  if (take_error_bwd(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
-  if (take_error_decode(&word, &site) != cudaSuccess) return FA_ERR_CUDA;
+  if ((e = take_error_fwd(&word, &site)) != cudaSuccess) return cuda_fail(int(e));
+  if ((e = take_error_bwd(&word, &site)) != cudaSuccess) return cuda_fail(int(e));
+  if ((e = take_error_decode(&word, &site)) != cudaSuccess) return cuda_fail(int(e));
   if (site != 0) g_last_site = site;
   if (word & 2) return FA_ERR_CUDA;  // a kernel found its shared memory misaligned (kErrLayout)
   if (word & 4) return FA_ERR_BOUNDS;  // a debug build's index check failed (kErrBounds)
@@ -536,11 +561,11 @@ int fa_bwd_set_timing_events(void* start, void* stop) {
 
 int fa_last_timeout_site(void) { return g_last_site.load(); }
 
+int fa_last_cuda_error(void) { return g_last_cuda.load(); }
+
 int fa_selftest_wait_timeout(unsigned int limit_us, void* stream) {
   if (limit_us < 1 || limit_us > 1000000) return FA_ERR_INVALID;
-  return launch_selftest_wait(1000ull * limit_us, static_cast<cudaStream_t>(stream)) == cudaSuccess
-             ? FA_OK
-             : FA_ERR_CUDA;
+  return from_cuda(launch_selftest_wait(1000ull * limit_us, static_cast<cudaStream_t>(stream)));
 }
 
 #ifdef FA_DEBUG

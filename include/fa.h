@@ -264,6 +264,11 @@ int fa_status(void* stream);
  * counterpart on the pages. */
 int fa_last_timeout_site(void);
 
+/* Diagnostic: the CUDA error behind the most recent FA_ERR_CUDA of any call
+ * (a cudaError_t value, or 100000 + the CUresult of a failed tensor-map
+ * encoding); 0 if no call has returned FA_ERR_CUDA.  Process-wide. */
+int fa_last_cuda_error(void);
+
 /* Measurement hook (no counterpart on the pages, which only say to profile
  * kernels with Nsight Compute, 51CTO notes, section "FlashAttention V2相比V1有
  * 哪些改进").  When both are non-NULL, every later fa_bwd call records the

@@ -245,3 +245,15 @@ def test_attention_rejects_a_bias_that_wants_a_gradient():
     q = torch.zeros(1, 1, 4, 64)
     with pytest.raises(ValueError):
         fa.attention(q, q, q, bias=b)
+
+
+def test_cuda_failure_is_recorded(lib):
+    """Without a GPU, fa_status's stream synchronisation fails: FA_ERR_CUDA,
+    and fa_last_cuda_error names the runtime error behind it."""
+    import torch
+
+    if torch.cuda.is_available():
+        pytest.skip("needs a machine without a usable GPU")
+    assert lib.fa_status(None) == fa.FA_ERR_CUDA
+    code = lib.fa_last_cuda_error()
+    assert 0 < code < 100000
