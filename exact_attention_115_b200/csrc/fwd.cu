@@ -12,10 +12,10 @@
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
-// (fwd_tiles: one for 16-bit d = 128, two otherwise).  With two tiles it
-// ping-pongs them so the tensor core works on one tile while the softmax
-// warps work on the other; with one tile two CTAs share an SM and interleave
-// the same way.  Roles per CTA (128 threads per tile + 128):
+// (fwd_tiles_for: two, except one for 16-bit d = 128 when a query tile sees
+// fewer than 12 K/V tiles on average).  With two tiles it ping-pongs them so
+// the tensor core works on one tile while the softmax warps work on the
+// other; with one tile two CTAs share an SM and interleave the same way.  Roles per CTA (128 threads per tile + 128):
 //   warpgroup t (warps 4t..4t+3)  softmax + correction + epilogue of Q tile t
 //                                 (thread = row), 200 registers
 //   last warpgroup: warp 4·TILES issues the tcgen05 MMAs (one thread) and
@@ -28,6 +28,8 @@
 // O is written through the tile's Q buffer (free once the tile's products
 // are done) with TMA tensor stores.
 #define FA_SITE_BASE 10000
+#include <algorithm>
+
 #include "common.cuh"
 #include "dropout.cuh"
 #include "launch.h"
@@ -41,9 +43,11 @@ namespace {
 #endif
 constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entries stay <= 2^8
 
+// Q tiles per CTA of the dropout, bias and fp32 variants (the plain 16-bit
+// d = 128 kernels come with either count; see fwd_tiles_for).
 constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 1 : 2; }
 
-template <typename T, int D>
+template <typename T, int D, int NT = fwd_tiles(ElemTraits<T>::tf32, D)>
 struct FwdTraits {
   static constexpr int ES = sizeof(T);
   static constexpr int BN = 128;                 // keys of a K/V tile
@@ -57,9 +61,12 @@ struct FwdTraits {
   // while the other's products run, and one's set-up and epilogue overlap the
   // other's main loop, at the price of loading each K/V tile twice per SM.
   // With two tiles the CTA ping-pongs its own tiles over one K/V stream.
-  // Measured: one tile is faster for 16-bit d = 128 at causal N = 2048 (+4 %)
-  // and two tiles for d = 64 (+5 %); fp32 keeps two.
-  static constexpr int TILES = fwd_tiles(ElemTraits<T>::tf32, D);
+  // Measured (d = 128, bf16): one tile is faster when a query tile sees few
+  // K/V tiles (causal N = 1024: 113 vs 121 us; causal N = 2048: 174 vs
+  // 176 us), two when it sees many (causal N = 4096, 8192, 16384 and
+  // non-causal N = 2048, 8192: 6-10 % faster), as the CTA's set-up and
+  // epilogue are then spread over more tiles.  d = 64: two tiles (+5 %).
+  static constexpr int TILES = NT;
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
   static constexpr int SMEM_BUDGET = TILES == 1 ? 110 * 1024 : 200 * 1024;  // tiles, per CTA
   static constexpr int NS_RAW = (SMEM_BUDGET - TILES * TILE) / TILE;
@@ -180,12 +187,12 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 // into one index); otherwise every map is the 3-D (d, N, B·H) form.
 // DROP: dropout on P (16-bit types only), masks drawn in the softmax warps.
 // BIAS: an additive bias on the scaled scores (16-bit types only).
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS>
-__global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTAS_PER_SM)
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS, int NT>
+__global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, NT>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                FwdParams p) {
-  using Tr = FwdTraits<T, D>;
+  using Tr = FwdTraits<T, D, NT>;
   constexpr bool TF32 = ElemTraits<T>::tf32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -661,10 +668,12 @@ __global__ void __launch_bounds__(FwdTraits<T, D>::THREADS, FwdTraits<T, D>::CTA
 
 }  // namespace
 
-template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false>
+template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false,
+          int NT = fwd_tiles(ElemTraits<T>::tf32, D)>
 static cudaError_t launch_fwd_t(const FwdLaunch& a) {
-  using Tr = FwdTraits<T, D>;
-  auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP, BIAS>;
+  using Tr = FwdTraits<T, D, NT>;
+  if (a.params.tiles != NT) return cudaErrorInvalidValue;  // the grid was sized for another count
+  auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP, BIAS, NT>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // setmaxnreg redistributes the registers the CTA was launched with; refuse
@@ -684,7 +693,16 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
 
 int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
 
-int fwd_rows_per_cta(int dtype, int d) { return 128 * fwd_tiles(dtype == FA_FP32, d); }
+int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool plain) {
+  const int dflt = fwd_tiles(dtype == FA_FP32, d);
+  if (dtype == FA_FP32 || d != 128 || !plain) return dflt;
+  // K/V tiles a 128-row query tile sees, on average (bottom-right causal:
+  // query tile i sees about i + 1 + (Nk − Nq) / 128 of them)
+  const double kv_tiles = (Nk + 127) / 128;
+  const double q_tiles = (Nq + 127) / 128;
+  const double avg = causal ? std::min(kv_tiles, (q_tiles + 1) / 2 + double(Nk - Nq) / 128) : kv_tiles;
+  return avg >= 12.0 ? 2 : 1;
+}
 
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
   const bool gen = a.params.map4d != 0;  // only 4-D tensor maps differ: every access is TMA
@@ -701,6 +719,11 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \
+    if (DD == 128 && a.params.tiles == 2)                                                        \
+      return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 2>(a)                \
+                           : launch_fwd_t<TY, DD, true, false, false, false, 2>(a))              \
+                    : (gen ? launch_fwd_t<TY, DD, false, true, false, false, 2>(a)               \
+                           : launch_fwd_t<TY, DD, false, false, false, false, 2>(a));            \
     return causal ? (gen ? launch_fwd_t<TY, DD, true, true>(a) : launch_fwd_t<TY, DD, true, false>(a)) \
                   : (gen ? launch_fwd_t<TY, DD, false, true>(a) : launch_fwd_t<TY, DD, false, false>(a)); \
   }

@@ -42,7 +42,8 @@ struct FwdParams {
   float* L;
   int B, H, Nq, Nk;
   float scale_log2;  // scale * log2(e)
-  int n_qblocks;     // ceil(Nq / fwd_rows_per_cta): one CTA per block of query rows
+  int tiles;         // 128-row Q tiles per CTA (fwd_tiles_for)
+  int n_qblocks;     // ceil(Nq / (128 · tiles)): one CTA per block of query rows
   int head_group;    // heads per launch-order group (see head_group_for)
   int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
   DropoutParams drop;
@@ -61,8 +62,9 @@ struct FwdLaunch {
 
 // Elements in one 128-byte swizzled row for the dtype (the TMA box width).
 int fwd_tile_elems(int dtype);
-// Query rows per forward CTA.
-int fwd_rows_per_cta(int dtype, int d);
+// 128-row Q tiles per forward CTA for a call (1 or 2); `plain` = no dropout
+// and no bias.
+int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool plain);
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a);
 
 struct BwdParams {

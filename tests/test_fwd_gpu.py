@@ -55,6 +55,32 @@ def test_rectangular(fa, Nq, Nk, causal):
     run_full(fa, 1, 2, Nq, Nk, 128, causal, seed=Nq + Nk)
 
 
+@pytest.mark.parametrize("Nq,Nk,causal,dtype", [
+    (1600, 1600, False, "bf16"),   # 13 K/V tiles per query tile, 12.5 Q tiles: a half-empty last CTA
+    (3000, 3000, True, "bf16"),    # causal, 12.5 K/V tiles on average, ragged ends
+    (1000, 2000, True, "fp16"),    # bottom-right causal with Nk − Nq = 1000
+    (129, 1700, False, "bf16"),    # two Q tiles, the second with one row
+])
+def test_two_tile_d128_kernel(fa, Nq, Nk, causal, dtype):
+    """Shapes whose query tiles see 12 or more K/V tiles on average run the
+    16-bit d = 128 forward with two Q tiles per CTA."""
+    run_full(fa, 1, 2, Nq, Nk, 128, causal, dtype, seed=Nq + 3 * Nk)
+
+
+def test_two_tile_d128_kernel_strided_with_padding(fa):
+    """The two-tile d = 128 forward on a [B, N, H, d] layout with key padding."""
+    B, H, N, d = 2, 2, 1700, 128
+    q, k, v, _ = W.make_tensors(B, H, N, N, d, "bf16", seed=8, device="cuda", with_grad=False)
+    bshd = lambda t: t.transpose(1, 2).contiguous().transpose(1, 2)  # noqa: E731
+    kv_len = torch.tensor([1700, 900], dtype=torch.int32, device="cuda")
+    scale = 1 / math.sqrt(d)
+    O, L = fa.forward(bshd(q), bshd(k), bshd(v), causal=False, scale=scale, kv_len=kv_len)
+    assert fa.status() == fa.FA_OK
+    O_ref, L_ref = oracle.attention_forward(f64(q), f64(k), f64(v), scale, False,
+                                            kv_len=kv_len.cpu().numpy())
+    check_fwd(O, L, O_ref, L_ref, "two-tile d128, [B, N, H, d], kv_len")
+
+
 @pytest.mark.parametrize("dtype", ["fp16", "bf16"])
 def test_fp16_and_bf16(fa, dtype):
     run_full(fa, 2, 4, 384, 384, 128, True, dtype)
