@@ -182,7 +182,7 @@ __device__ __forceinline__ void q_tile_range(int kb, int Nq, int Nk, int& i0, in
 // The fp32 dQ buffer is S slabs of [B·H, Nq_pad, d]: one accumulator
 // (mode 1), one partial per K/V block (mode 2), or dq_groups accumulators
 // (mode 3).  K/V block kb writes slab dq_slab(p, kb).
-__device__ __forceinline__ int dq_slabs(const BwdParams& p) {
+[[maybe_unused]] __device__ __forceinline__ int dq_slabs(const BwdParams& p) {
   return p.dq_mode == 2 ? p.n_kblocks : p.dq_mode == 3 ? p.dq_groups : 1;
 }
 __device__ __forceinline__ int dq_slab(const BwdParams& p, int kb) {
@@ -863,13 +863,15 @@ __global__ void __launch_bounds__(512, 1)
 // −D = −rowsum(dO ∘ O) and −L·log2e into padded buffers (−inf on padding
 // rows, so their P is 0), stored negated so the main kernel adds them; in
 // mode 1 the fp32 dQ accumulator is cleared.
-// A group of D/8 lanes handles one row (8 elements per lane).
+// A group of D/8 lanes handles one row (8 elements per lane).  Heads go in
+// the reverse of the main kernel's order (blocks run y-major), so the first
+// heads the main kernel takes are the last ones written here, still in L2.
 template <typename T, int D, bool GEN>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;  // rows per block
   const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
-  const int bh = blockIdx.y;
+  const int bh = int(gridDim.y) - 1 - int(blockIdx.y);
   const int q = blockIdx.x * RPB + g;
   if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.item_ctr = 0;
   if (q >= p.Nq_pad || !FA_INBOUNDS(bh < p.B * p.H)) return;
@@ -911,12 +913,14 @@ __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
 
 // dQ = scale · Σ (dQ accumulator or per-K/V-block partials), cast to the
 // dtype (the main kernel's dS leaves the softmax scale out).
+// Heads in the reverse of the main kernel's order too: its last heads'
+// accumulators are the ones still in L2.
 template <typename T, int D, bool CAUSAL, bool GEN>
 __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;
   const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
-  const int bh = blockIdx.y;
+  const int bh = int(gridDim.y) - 1 - int(blockIdx.y);
   const int q = blockIdx.x * RPB + g;
   if (q >= p.Nq || !FA_INBOUNDS(bh < p.B * p.H)) return;
   float acc[8];
