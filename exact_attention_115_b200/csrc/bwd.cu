@@ -84,7 +84,12 @@ struct BwdTraits {
   static constexpr int ES = 2;
   static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
   static constexpr int BM = 128;                     // query rows per step
-  static constexpr int CWC = BM / 2;                 // query columns per compute warpgroup
+  // Compute warpgroups.  Four (32 query columns each, 768 threads, 72
+  // registers per compute thread) measured 2 % slower at causal N = 2048
+  // d = 128 and no faster at d = 64: the P phase is not shortened by more
+  // warps per sub-partition.
+  static constexpr int NCW = 2;
+  static constexpr int CWC = BM / NCW;               // query columns per compute warpgroup
   // d = 128: dQᵀ = Kᵀ dSᵀ with d on the TMEM lanes, so that a warp adds one
   // 128-byte line of the accumulator per query row.  (dQ = dS K with rows on
   // the lanes and four-wide reductions of each thread's row measured 30 %
@@ -121,13 +126,21 @@ struct BwdTraits {
   static constexpr int COL_DK = COL_DV + D;
   static_assert(COL_DK + D <= 512, "TMEM budget");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared-memory budget");
-  static constexpr int THREADS = 512;
-  // setmaxnreg split; 256·REGS_COMPUTE + 128·(REGS_DQ + REGS_OTHER) must not
-  // exceed the 512 × 128 registers the CTA is launched with.
+  // Warps: the compute warpgroups, then the dQ warpgroup, then MMA issue,
+  // Q / dO producer, scheduler + K / V loads and one idle warp.
+  static constexpr int THREADS = 128 * (NCW + 2);
+  static constexpr int WARP_DQ0 = 4 * NCW;
+  static constexpr int WARP_MMA = WARP_DQ0 + 4;
+  static constexpr int WARP_PROD = WARP_MMA + 1;
+  static constexpr int WARP_SCHED = WARP_MMA + 2;
+  // setmaxnreg split; 128·(NCW·REGS_COMPUTE + REGS_DQ + REGS_OTHER) must not
+  // exceed the registers the CTA is launched with (THREADS × LAUNCH_REGS).
+  static constexpr int LAUNCH_REGS = (65536 / THREADS) / 8 * 8;
   static constexpr int REGS_COMPUTE = 136;
   static constexpr int REGS_DQ = 136;
   static constexpr int REGS_OTHER = 104;
-  static_assert(256 * REGS_COMPUTE + 128 * (REGS_DQ + REGS_OTHER) <= THREADS * 128, "register split");
+  static_assert(128 * (NCW * REGS_COMPUTE + REGS_DQ + REGS_OTHER) <= THREADS * LAUNCH_REGS,
+                "register split");
   static constexpr uint32_t F = ElemTraits<T>::fmt;
   static constexpr uint32_t IDESC_ST = make_idesc(F, 128, BM, 0, 0);   // Sᵀ, dPᵀ
   static constexpr uint32_t IDESC_GRAD = make_idesc(F, 128, D, 0, 1);  // dV (A in TMEM), dK (A = dSᵀ K-major)
@@ -194,7 +207,7 @@ __device__ __forceinline__ int dq_slab(const BwdParams& p, int kb) {
 // DROP: the forward dropped weights; the compute warps redraw its keep mask.
 // BIAS: the forward added a bias to the scaled scores; P is rebuilt with it.
 template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS>
-__global__ void __launch_bounds__(512, 1)
+__global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmdQ,
@@ -247,8 +260,8 @@ __global__ void __launch_bounds__(512, 1)
     mbar_init(&bars->do_empty, 1);
     mbar_init(&bars->s_full, 1);
     mbar_init(&bars->dp_full, 1);
-    mbar_init(&bars->p_ready, 256);
-    mbar_init(&bars->ds_ready, 256);
+    mbar_init(&bars->p_ready, 128 * Tr::NCW);
+    mbar_init(&bars->ds_ready, 128 * Tr::NCW);
     mbar_init(&bars->dq_full, 1);
     mbar_init(&bars->dq_empty, 128);
     mbar_init(&bars->ds_free, 1);
@@ -258,11 +271,11 @@ __global__ void __launch_bounds__(512, 1)
     bars->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 12) {
+  if (warp == Tr::WARP_MMA) {
     tmem_alloc(&bars->tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 13 && lane == 0) {
+  if (warp == Tr::WARP_PROD && lane == 0) {
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
@@ -282,12 +295,13 @@ __global__ void __launch_bounds__(512, 1)
   uint8_t* sdQ = smem + Tr::OFF_DQ;  // d = 64: two [128 rows × 128 B] swizzled halves
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
 
-  // Register split (the CTA launches with 128 per thread): the compute and
-  // dQ warpgroups hold a step's TMEM columns in registers, warps 12-15
-  // (MMA issue, loads, scheduling) need few.  Each role sets its own count.
-  if (warp >= 14) {
-    regs_dec<Tr::REGS_OTHER>();
-    if (warp == 14 && lane == 0) {
+  // Register split (the CTA launches with LAUNCH_REGS per thread): the
+  // compute and dQ warpgroups hold a step's TMEM columns in registers, the
+  // last warpgroup (MMA issue, loads, scheduling) needs few.  Each role sets
+  // its own count.
+  if (warp >= Tr::WARP_SCHED) {
+    regs_set<Tr::REGS_OTHER, Tr::LAUNCH_REGS>();
+    if (warp == Tr::WARP_SCHED && lane == 0) {
       // ---------------------------------------------------- scheduler + K/V loads
       // Work items are handed out dynamically in the grouped order: the first
       // wave by CTA index, the rest from a global counter, each taken when
@@ -334,9 +348,9 @@ __global__ void __launch_bounds__(512, 1)
         MBAR_WAIT(&bars->k_full[k & 1], (k >> 1) & 1, abort_flag);
       if (it > 0) MBAR_WAIT(&bars->v_full, (it - 1) & 1, abort_flag);
     }
-  } else if (warp == 13) {
+  } else if (warp == Tr::WARP_PROD) {
     // ------------------------------------------------------------ Q / dO producer
-    regs_dec<Tr::REGS_OTHER>();
+    regs_set<Tr::REGS_OTHER, Tr::LAUNCH_REGS>();
     if (lane == 0) {
       bool ok = true;
       int g = 0, it = 0;
@@ -382,9 +396,9 @@ __global__ void __launch_bounds__(512, 1)
         MBAR_WAIT(&bars->q_full[gs & 1], (gs >> 1) & 1, abort_flag);
       if (g > 0) MBAR_WAIT(&bars->do_full, (g - 1) & 1, abort_flag);
     }
-  } else if (warp == 12) {
+  } else if (warp == Tr::WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    regs_dec<Tr::REGS_OTHER>();
+    regs_set<Tr::REGS_OTHER, Tr::LAUNCH_REGS>();
     // The whole warp runs the loop (warp-uniform waits and descriptor
     // arithmetic); the elected lane issues the MMAs and commits.
     {
@@ -537,11 +551,11 @@ __global__ void __launch_bounds__(512, 1)
         g += n_q;
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < Tr::WARP_DQ0) {
     // ------------------------------------------------------------ P / dS (thread = key)
-    // Two warpgroups; warpgroup cw handles query columns [cw·CWC, (cw+1)·CWC)
+    // NCW warpgroups; warpgroup cw handles query columns [cw·CWC, (cw+1)·CWC)
     // of each step for all 128 key rows.
-    regs_inc<Tr::REGS_COMPUTE>();
+    regs_set<Tr::REGS_COMPUTE, Tr::LAUNCH_REGS>();
     const int cw = warp >> 2;
     const int quad = warp & 3;
     const int kr = quad * 32 + lane;  // key row in the tile = TMEM lane
@@ -705,13 +719,13 @@ __global__ void __launch_bounds__(512, 1)
       g += n_q;
     }
   } else {
-    // ------------------------------------------------------------ dQ (warpgroup 2)
-    regs_inc<Tr::REGS_DQ>();
+    // ------------------------------------------------------------ dQ (the warpgroup after the compute ones)
+    regs_set<Tr::REGS_DQ, Tr::LAUNCH_REGS>();
     const int quad = warp & 3;
     const int r = quad * 32 + lane;  // TMEM lane: d index (dQᵀ) or query row (dQ)
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
     const uint32_t tQ = tmem + lane_off + Tr::COL_DP;  // dQ of the step sits in the dPᵀ columns
-    const bool leader = (warp == 8 && lane == 0);
+    const bool leader = (warp == Tr::WARP_DQ0 && lane == 0);
     bool ok = true;
     int g = 0, it = 0;
     for (int j; ok && named_bar_and(1, 128, take_item(it, j)); ++it) {
@@ -854,7 +868,7 @@ __global__ void __launch_bounds__(512, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 12) {
+  if (warp == Tr::WARP_MMA) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
@@ -1085,7 +1099,8 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
     cudaFuncAttributes attr;
     e = cudaFuncGetAttributes(&attr, reinterpret_cast<const void*>(kern));
     if (e != cudaSuccess) return e;
-    regs_ok = attr.numRegs * Tr::THREADS >= 256 * Tr::REGS_COMPUTE + 128 * (Tr::REGS_DQ + Tr::REGS_OTHER);
+    regs_ok = attr.numRegs * Tr::THREADS >=
+              128 * (Tr::NCW * Tr::REGS_COMPUTE + Tr::REGS_DQ + Tr::REGS_OTHER);
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
   if (a.ev_start) {

@@ -466,6 +466,12 @@ template <int N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// N registers per thread for the warpgroup, from the launch count L.
+template <int N, int L>
+__device__ __forceinline__ void regs_set() {
+  if constexpr (N > L) regs_inc<N>();
+  else if constexpr (N < L) regs_dec<N>();
+}
 
 // ------------------------------------------------------------------ math
 __device__ __forceinline__ float ex2(float x) {
