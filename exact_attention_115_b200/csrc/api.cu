@@ -426,6 +426,30 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
     p.bias = bias;
     p.s_bias = Strides{lbias->b, lbias->h, lbias->n};
     p.bias_l2 = 1.4426950408889634f;
+    // The backward stages each step's [128 queries × 128 keys] bias tile with
+    // one TMA load: a 4-D map (key, query, head, batch) whose query, head or
+    // batch extent is 1 where the bias broadcasts (stride 0); a bias shared
+    // by all query rows loads one row per step, which every query reads.
+    // Past Nq and Nk the tile is zero-filled.
+    p.bias_H = lbias->h ? H : 1;
+    p.bias_B = lbias->b ? B : 1;
+    p.bias_rows = lbias->n ? 128 : 1;
+    const cuuint64_t es = cuuint64_t(elem_size(dtype));
+    // the stride given for an extent-1 dimension (never stepped over)
+    const cuuint64_t unit = (cuuint64_t(Nk) * es + 15) / 16 * 16;
+    cuuint64_t dims[4] = {cuuint64_t(Nk), lbias->n ? cuuint64_t(Nq) : 1, cuuint64_t(p.bias_H),
+                          cuuint64_t(p.bias_B)};
+    cuuint64_t strides[3] = {lbias->n ? cuuint64_t(lbias->n) * es : unit,
+                             lbias->h ? cuuint64_t(lbias->h) * es : unit,
+                             lbias->b ? cuuint64_t(lbias->b) * es : unit};
+    cuuint32_t box[4] = {128, cuuint32_t(p.bias_rows), 1, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cuda_fail(int(cudaErrorSymbolNotFound));
+    const CUresult r = enc(&a.tmBias, tma_type(dtype), 4, const_cast<void*>(bias), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cuda_fail(100000 + int(r));
   }
   a.stream = static_cast<cudaStream_t>(stream);
   a.ev_start = g_ev_start;

@@ -79,7 +79,7 @@ __device__ __forceinline__ void red_add_f32(float* dst, float v) {
 }
 constexpr float kLog2e = 1.4426950408889634f;
 
-template <typename T, int D>
+template <typename T, int D, bool BIAS = false>
 struct BwdTraits {
   static constexpr int ES = 2;
   static constexpr int BN = 128;                     // keys per CTA (TMEM lanes)
@@ -110,6 +110,12 @@ struct BwdTraits {
   // next work item's K loads while this item runs); Q is double buffered
   // (the next step's Sᵀ needs it while this step's dK still reads the
   // current one); V and dO are single buffered.
+  // The bias variants stage each step's [BM queries × BN keys] bias tile in
+  // shared memory (one TMA load).  At d = 128 its 32 KB take the second K
+  // buffer (K is then single buffered); at d = 64 there is room after the rest.
+  static constexpr int BIAS_TILE = BIAS ? BM * BN * ES : 0;
+  static constexpr bool K_SINGLE = BIAS && D == 128;
+  static constexpr int KBUF = K_SINGLE ? 1 : 2;      // K buffers
   static constexpr int OFF_K = 0;                    // 2 buffers
   static constexpr int OFF_V = OFF_K + 2 * KV_TILE;
   static constexpr int OFF_Q = OFF_V + KV_TILE;      // 2 stages
@@ -118,7 +124,9 @@ struct BwdTraits {
   static constexpr int OFF_DQ = OFF_DS + DS_TILE;
   static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;   // L·log2e and D per Q stage
   static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BM * 4;
-  static constexpr int SMEM_BYTES = OFF_BAR + 512;  // the base is checked to be 1024-aligned
+  static constexpr int OFF_BIAS = K_SINGLE ? OFF_K + KV_TILE : (OFF_BAR + 512 + 1023) / 1024 * 1024;
+  // the base is checked to be 1024-aligned
+  static constexpr int SMEM_BYTES = (BIAS && !K_SINGLE) ? OFF_BIAS + BIAS_TILE : OFF_BAR + 512;
   // TMEM columns: Sᵀ | dPᵀ (dQ of the step lands here after dK read dSᵀ) | dV | dK
   static constexpr int COL_S = 0;
   static constexpr int COL_DP = BM;
@@ -175,6 +183,8 @@ struct BwdBarriers {
   uint64_t ds_free;
   uint64_t dkv_done;      // the item's last dK / dV products are complete
   uint64_t dkv_free;      // the epilogue has read the item's dK / dV from TMEM
+  uint64_t bias_full;     // BIAS: the step's bias tile has landed (once per step)
+  uint64_t bias_empty;    // BIAS: the compute warpgroups have copied it out
   uint64_t item_full[4];  // the scheduler published work item `it` in slot it % 4
   int item_idx[4];        // its index in the grouped order, or -1 after the last
   uint32_t tmem_base;
@@ -207,12 +217,12 @@ __device__ __forceinline__ int dq_slab(const BwdParams& p, int kb) {
 // DROP: the forward dropped weights; the compute warps redraw its keep mask.
 // BIAS: the forward added a bias to the scaled scores; P is rebuilt with it.
 template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS>
-__global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
+__global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                     const __grid_constant__ CUtensorMap tmdQ,
-                    BwdParams p) {
-  using Tr = BwdTraits<T, D>;
+                    const __grid_constant__ CUtensorMap tmBias, BwdParams p) {
+  using Tr = BwdTraits<T, D, BIAS>;
   constexpr int BM = Tr::BM;
   constexpr int CWC = Tr::CWC;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -267,6 +277,8 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
     mbar_init(&bars->ds_free, 1);
     mbar_init(&bars->dkv_done, 1);
     mbar_init(&bars->dkv_free, 128);
+    mbar_init(&bars->bias_full, 1);
+    mbar_init(&bars->bias_empty, 128 * Tr::NCW);
     for (int k = 0; k < 4; ++k) mbar_init(&bars->item_full[k], 1);
     bars->abort_flag = 0;
     fence_mbar_init();
@@ -281,6 +293,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
     tma_prefetch_desc(&tmV);
     tma_prefetch_desc(&tmdO);
     if constexpr (Tr::DQ_STAGED) tma_prefetch_desc(&tmdQ);
+    if constexpr (BIAS) tma_prefetch_desc(&tmBias);
   }
   tc_fence_before();
   __syncthreads();
@@ -294,6 +307,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
   uint8_t* sdS = smem + Tr::OFF_DS;
   uint8_t* sdQ = smem + Tr::OFF_DQ;  // d = 64: two [128 rows × 128 B] swizzled halves
   float* sLD = reinterpret_cast<float*>(smem + Tr::OFF_LD);  // [stage][2][BM]
+  uint8_t* sBias = smem + Tr::OFF_BIAS;  // BIAS: [BM queries][BN keys] of the input type
 
   // Register split (the CTA launches with LAUNCH_REGS per thread): the
   // compute and dQ warpgroups hold a step's TMEM columns in registers, the
@@ -308,7 +322,9 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
       // the previous item has issued its last dPᵀ (about one step before it
       // ends), so no CTA holds a claim on work it cannot start soon.  The
       // item's K goes to buffer it % 2 (the previous item still reads the
-      // other), its V to the one V buffer, which that last dPᵀ released.
+      // other; the bias variants at d = 128 have one K buffer, which the
+      // previous item's last dQ product released), its V to the one V buffer,
+      // which that last dPᵀ released.
       bool ok = true;
       int it = 0;
       for (;; ++it) {
@@ -323,8 +339,8 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
         if (last) break;
         int bh, kb, i0, n_q;
         item(j, bh, kb, i0, n_q);
-        const int key0 = kb * Tr::BN, b = it & 1;
-        if (it >= 2 && !MBAR_WAIT(&bars->k_free[b], ((it >> 1) - 1) & 1, abort_flag)) {
+        const int key0 = kb * Tr::BN, b = it % Tr::KBUF;
+        if (it >= Tr::KBUF && !MBAR_WAIT(&bars->k_free[b], ((it / Tr::KBUF) - 1) & 1, abort_flag)) {
           ok = false;
           continue;
         }
@@ -344,8 +360,8 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
                       p.H);
       }
       // Drain every issued load before the CTA may exit (it items loaded).
-      for (int k = max(0, it - 2); k < it; ++k)
-        MBAR_WAIT(&bars->k_full[k & 1], (k >> 1) & 1, abort_flag);
+      for (int k = max(0, it - Tr::KBUF); k < it; ++k)
+        MBAR_WAIT(&bars->k_full[k % Tr::KBUF], (k / Tr::KBUF) & 1, abort_flag);
       if (it > 0) MBAR_WAIT(&bars->v_full, (it - 1) & 1, abort_flag);
     }
   } else if (warp == Tr::WARP_PROD) {
@@ -360,6 +376,21 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
         for (int i = 0; i < n_q && ok; ++i) {
           const int gs = g + i, s = gs & 1;
           const int q0 = (i0 + i) * BM;
+          if constexpr (BIAS) {
+            // the step's [BM queries × BN keys] bias tile (zero past Nq and
+            // Nk), once the compute warpgroups have copied out step gs-1's
+            if (gs >= 1 && !MBAR_WAIT(&bars->bias_empty, (gs - 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            if (!FA_INBOUNDS(kb * Tr::BN < p.Nk && q0 < p.Nq && bh < p.B * p.H)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&bars->bias_full, p.bias_rows * Tr::BN * Tr::ES);
+            tma_load_4d(sBias, &tmBias, &bars->bias_full, kb * Tr::BN, p.bias_rows > 1 ? q0 : 0,
+                        (bh % p.H) % p.bias_H, (bh / p.H) % p.bias_B);
+          }
           // Q (with −L·log2e and −D) into stage s, once step gs-2 has released it
           if (gs >= 2 && !MBAR_WAIT(&bars->q_empty[s], ((gs >> 1) - 1) & 1, abort_flag)) {
             ok = false;
@@ -395,6 +426,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
       for (int gs = max(0, g - 2); gs < g; ++gs)
         MBAR_WAIT(&bars->q_full[gs & 1], (gs >> 1) & 1, abort_flag);
       if (g > 0) MBAR_WAIT(&bars->do_full, (g - 1) & 1, abort_flag);
+      if (BIAS && g > 0) MBAR_WAIT(&bars->bias_full, (g - 1) & 1, abort_flag);
     }
   } else if (warp == Tr::WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
@@ -474,9 +506,13 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
         item(j, bh, kb, i0, n_q);
         (void)bh;
         (void)i0;
-        const int b = it & 1;
+        int b = it % Tr::KBUF;
+        // With one K buffer the index is the constant 0, and the compiler then
+        // keeps every product's descriptors live across items (spilling);
+        // hidden from it, they are formed per item as with two buffers.
+        if constexpr (Tr::KBUF == 1) asm volatile("" : "+r"(b));
         const uint64_t dK_k = kbuf(dK_k0, b), dK_mn = kbuf(dK_mn0, b);
-        ok = MBAR_WAIT_WARP(&bars->k_full[b], (it >> 1) & 1, abort_flag);
+        ok = MBAR_WAIT_WARP(&bars->k_full[b], (it / Tr::KBUF) & 1, abort_flag);
         if (ok && n_q > 0)
           ok = MBAR_WAIT_WARP(&bars->q_full[g & 1], (g >> 1) & 1, abort_flag) &&
                MBAR_WAIT_WARP(&bars->do_full, g & 1, abort_flag);
@@ -587,19 +623,26 @@ __global__ void __launch_bounds__(BwdTraits<T, D>::THREADS, 1)
           for (int g16 = 0; g16 < CWC / 16; ++g16) keep16_col(p.drop, bh, key, q0 + 16 * g16, keep + 4 * g16);
         }
         // Bias: this key's values for the CWC query columns, as packed pairs
-        // (warp lanes hold consecutive keys, so each load is coalesced);
-        // zero past Nq or past Nk.
+        // (zero past Nq or past Nk: the tile's load fills them with zeros).
         uint32_t bpk[BIAS ? CWC / 2 : 1];
         if constexpr (BIAS) {
-          const uint16_t* bcol = reinterpret_cast<const uint16_t*>(p.bias) + (bh / p.H) * p.s_bias.b +
-                                 (bh % p.H) * p.s_bias.h + (key < p.Nk ? key : 0);
+          // out of the step's staged tile (row = query, BN keys contiguous;
+          // a warp's lanes read 64 consecutive bytes of a row), then the tile
+          // is released so the producer can load the next step's
+          ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->bias_full, gs & 1, abort_flag));
+          if (!ok) break;
+          const uint16_t* bt = reinterpret_cast<const uint16_t*>(sBias) + kr;
+          if (p.bias_rows > 1) {
+            bt += cw * CWC * Tr::BN;
 #pragma unroll
-          for (int c = 0; c < CWC; c += 2) {
-            const int qa = q0 + c;
-            const uint32_t lo = (key < p.Nk && qa < p.Nq) ? __ldg(bcol + (long long)qa * p.s_bias.n) : 0u;
-            const uint32_t hi = (key < p.Nk && qa + 1 < p.Nq) ? __ldg(bcol + (long long)(qa + 1) * p.s_bias.n) : 0u;
-            bpk[c >> 1] = lo | (hi << 16);
+            for (int c = 0; c < CWC; c += 2)
+              bpk[c >> 1] = uint32_t(bt[c * Tr::BN]) | (uint32_t(bt[(c + 1) * Tr::BN]) << 16);
+          } else {  // one row shared by all queries
+            const uint32_t v = bt[0];
+#pragma unroll
+            for (int c = 0; c < CWC; c += 2) bpk[c >> 1] = v | (v << 16);
           }
+          mbar_arrive(&bars->bias_empty);
         }
         // ---- P = exp2(S·c − L·log2e), causal / ragged masking
         ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full, gs & 1, abort_flag));
@@ -1082,7 +1125,7 @@ static cudaError_t launch_bwd_fp32(const BwdLaunch& a) {
 
 template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false>
 static cudaError_t launch_bwd_t(const BwdLaunch& a) {
-  using Tr = BwdTraits<T, D>;
+  using Tr = BwdTraits<T, D, BIAS>;
   const BwdParams& p = a.params;
   constexpr int RPB = 256 / (D / 8);
   const int BH = p.B * p.H;
@@ -1109,7 +1152,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   }
   // persistent: one CTA per SM (or per work item, if fewer)
   const int grid = std::min(p.n_kblocks * BH, sm_count());
-  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdQ, p);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmdO, a.tmdQ, a.tmBias, p);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   if (a.ev_stop) {

@@ -96,11 +96,14 @@ struct BwdParams {
   const void* bias;   // additive bias, as in FwdParams
   Strides s_bias;
   float bias_l2;      // log2(e): the bias in the backward's log2 units
+  int bias_H, bias_B; // the bias tensor map's head and batch extents (1 where it broadcasts)
+  int bias_rows;      // query rows of the staged bias tile: 128, or 1 for a bias shared by all rows
 };
 
 struct BwdLaunch {
   CUtensorMap tmQ, tmK, tmV, tmdO;
   CUtensorMap tmdQ;  // d = 64: the fp32 dQ accumulator as a [rows, 64] tensor (tensor reduce-add)
+  CUtensorMap tmBias;  // bias: (key, query, head, batch), boxes of 128 keys × 128 queries
   BwdParams params;
   cudaStream_t stream;
   cudaEvent_t ev_start, ev_stop;  // optional timing events around the main kernel

@@ -65,11 +65,14 @@ def _check_rows(O, L, O_ref, L_ref, what):
 
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-@pytest.mark.parametrize("bshape", ["full", "batch_bcast", "head_bcast"])
+@pytest.mark.parametrize("bshape", ["full", "batch_bcast", "head_bcast", "query_bcast", "keys_only"])
 def test_bias(fa, d, causal, bshape):
+    """Broadcast forms: over batches, heads, query rows ([B, H, 1, Nk]: one
+    row per step staged for every query in the backward), or all three."""
     B, H, N = 2, 3, 300
     q, k, v, do = W.make_tensors(B, H, N, N, d, "bf16", seed=81 + d, device="cuda")
-    shape = {"full": (B, H, N), "batch_bcast": (1, H, N), "head_bcast": (B, 1, N)}[bshape]
+    shape = {"full": (B, H, N), "batch_bcast": (1, H, N), "head_bcast": (B, 1, N),
+             "query_bcast": (B, H, 1), "keys_only": (1, 1, 1)}[bshape]
     bias = _bias(shape + (N,), N, torch.bfloat16, seed=7, ninf=0.05)
     _run(fa, q, k, v, do, bias, causal, f"bias {bshape} d{d} causal={causal}")
 
