@@ -96,6 +96,34 @@ bool make_map(CUtensorMap* m, const void* ptr, int dtype, int d, int N, int H, i
   return r == CUDA_SUCCESS;
 }
 
+// Tensor map of an additive bias for staging [rows × keys] tiles: 4-D (key,
+// query, head, batch), whose query, head or batch extent is 1 where the bias
+// broadcasts (stride 0, which a tensor map cannot hold; the stride given for
+// such a dimension is never stepped over).  A bias shared by all query rows
+// gives 1-row boxes.  Reads past Nq and Nk are zero-filled.  Sets the
+// extents the kernels index with.
+CUresult encode_bias_map(CUtensorMap* m, const void* bias, const fa_layout& lb, int dtype, int B,
+                         int H, int Nq, int Nk, int box_keys, bool swizzle128, int* bias_H,
+                         int* bias_B, int* bias_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return CUDA_ERROR_NOT_FOUND;
+  *bias_H = lb.h ? H : 1;
+  *bias_B = lb.b ? B : 1;
+  *bias_rows = lb.n ? 128 : 1;
+  const cuuint64_t es = cuuint64_t(elem_size(dtype));
+  const cuuint64_t unit = (cuuint64_t(Nk) * es + 15) / 16 * 16;
+  cuuint64_t dims[4] = {cuuint64_t(Nk), lb.n ? cuuint64_t(Nq) : 1, cuuint64_t(*bias_H),
+                        cuuint64_t(*bias_B)};
+  cuuint64_t strides[3] = {lb.n ? cuuint64_t(lb.n) * es : unit, lb.h ? cuuint64_t(lb.h) * es : unit,
+                           lb.b ? cuuint64_t(lb.b) * es : unit};
+  cuuint32_t box[4] = {cuuint32_t(box_keys), cuuint32_t(*bias_rows), 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(m, tma_type(dtype), 4, const_cast<void*>(bias), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE,
+             swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 fa_layout contiguous_layout(int H, int N, int d) {
   return fa_layout{(long long)H * N * d, (long long)N * d, (long long)d};
 }
@@ -272,13 +300,18 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   std::memset(&a, 0, sizeof(a));
   a.params.drop = drop;
   a.params.kv_len = kv_len;
+  st = from_cuda(ensure_context());
+  if (st != FA_OK) return st;
   if (bias) {
     a.params.bias = bias;
     a.params.s_bias = Strides{lbias->b, lbias->h, lbias->n};
     a.params.bias_mul = 1.0f / scale;
+    // the forward stages [128 rows × 128 keys] tiles as two 128-byte-swizzled
+    // halves of 64 keys
+    const CUresult r = encode_bias_map(&a.tmBias, bias, *lbias, dtype, B, H, Nq, Nk, 64, true,
+                                       &a.params.bias_H, &a.params.bias_B, &a.params.bias_rows);
+    if (r != CUDA_SUCCESS) return cuda_fail(100000 + int(r));
   }
-  st = from_cuda(ensure_context());
-  if (st != FA_OK) return st;
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
       !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
@@ -296,7 +329,7 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   a.params.Nq = Nq;
   a.params.Nk = Nk;
   a.params.scale_log2 = scale * 1.4426950408889634f;
-  a.params.tiles = fwd_tiles_for(dtype, d, Nq, Nk, causal != 0, !drop.t4 && !bias);
+  a.params.tiles = fwd_tiles_for(dtype, d, Nq, Nk, causal != 0, drop.t4 != 0, bias != nullptr);
   const int rows = 128 * a.params.tiles;
   a.params.n_qblocks = (Nq + rows - 1) / rows;
   a.params.head_group = head_group_for(size_t(Nk) * d * 2 * elem_size(dtype), BH);
@@ -427,28 +460,9 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
     p.s_bias = Strides{lbias->b, lbias->h, lbias->n};
     p.bias_l2 = 1.4426950408889634f;
     // The backward stages each step's [128 queries × 128 keys] bias tile with
-    // one TMA load: a 4-D map (key, query, head, batch) whose query, head or
-    // batch extent is 1 where the bias broadcasts (stride 0); a bias shared
-    // by all query rows loads one row per step, which every query reads.
-    // Past Nq and Nk the tile is zero-filled.
-    p.bias_H = lbias->h ? H : 1;
-    p.bias_B = lbias->b ? B : 1;
-    p.bias_rows = lbias->n ? 128 : 1;
-    const cuuint64_t es = cuuint64_t(elem_size(dtype));
-    // the stride given for an extent-1 dimension (never stepped over)
-    const cuuint64_t unit = (cuuint64_t(Nk) * es + 15) / 16 * 16;
-    cuuint64_t dims[4] = {cuuint64_t(Nk), lbias->n ? cuuint64_t(Nq) : 1, cuuint64_t(p.bias_H),
-                          cuuint64_t(p.bias_B)};
-    cuuint64_t strides[3] = {lbias->n ? cuuint64_t(lbias->n) * es : unit,
-                             lbias->h ? cuuint64_t(lbias->h) * es : unit,
-                             lbias->b ? cuuint64_t(lbias->b) * es : unit};
-    cuuint32_t box[4] = {128, cuuint32_t(p.bias_rows), 1, 1};
-    cuuint32_t estr[4] = {1, 1, 1, 1};
-    EncodeTiledFn enc = encode_fn();
-    if (!enc) return cuda_fail(int(cudaErrorSymbolNotFound));
-    const CUresult r = enc(&a.tmBias, tma_type(dtype), 4, const_cast<void*>(bias), dims, strides, box,
-                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    // one TMA load (no swizzle: a warp reads 64 consecutive bytes of a row).
+    const CUresult r = encode_bias_map(&a.tmBias, bias, *lbias, dtype, B, H, Nq, Nk, 128, false,
+                                       &p.bias_H, &p.bias_B, &p.bias_rows);
     if (r != CUDA_SUCCESS) return cuda_fail(100000 + int(r));
   }
   a.stream = static_cast<cudaStream_t>(stream);

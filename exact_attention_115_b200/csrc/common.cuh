@@ -280,18 +280,6 @@ __device__ __forceinline__ void tma_store_bh(const CUtensorMap* map, bool map4d,
     tma_store_3d(map, src, x, y, bh);
 }
 
-// Eight consecutive 16-bit values from global memory, of which the first n
-// (0..8) are read and the rest are zero; one 16-byte load when n = 8 (the
-// address is then 16-byte aligned).
-__device__ __forceinline__ uint4 load8_16bit(const uint16_t* ptr, int n) {
-  if (n >= 8) return __ldg(reinterpret_cast<const uint4*>(ptr));
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-  for (int e = 0; e < 8; ++e)
-    if (e < n) w[e >> 1] |= uint32_t(__ldg(ptr + e)) << (16 * (e & 1));
-  return make_uint4(w[0], w[1], w[2], w[3]);
-}
-
 // Keys visible to head index bh = b·H + h: all Nk, or the key-padding length
 // kv_len[b] clamped to [0, Nk].
 __device__ __forceinline__ int keys_of(const int* kv_len, int bh, int H, int Nk) {

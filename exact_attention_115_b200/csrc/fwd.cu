@@ -47,7 +47,7 @@ constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entr
 // d = 128 kernels come with either count; see fwd_tiles_for).
 constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 1 : 2; }
 
-template <typename T, int D, int NT = fwd_tiles(ElemTraits<T>::tf32, D)>
+template <typename T, int D, int NT = fwd_tiles(ElemTraits<T>::tf32, D), bool BIAS = false>
 struct FwdTraits {
   static constexpr int ES = sizeof(T);
   static constexpr int BN = 128;                 // keys of a K/V tile
@@ -68,10 +68,16 @@ struct FwdTraits {
   // epilogue are then spread over more tiles.  d = 64: two tiles (+5 %).
   static constexpr int TILES = NT;
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
-  static constexpr int SMEM_BUDGET = TILES == 1 ? 110 * 1024 : 200 * 1024;  // tiles, per CTA
-  static constexpr int NS_RAW = (SMEM_BUDGET - TILES * TILE) / TILE;
+  // The bias variants (two tiles) stage each K/V step's [128 rows × 128 keys]
+  // bias tile of every Q tile in shared memory: two 128-byte-swizzled halves
+  // of 64 keys, so that a thread's row reads are free of bank conflicts.
+  static constexpr int BIAS_TILE = BIAS ? 128 * BN * ES : 0;
+  static constexpr int SMEM_BUDGET =
+      TILES == 1 ? 110 * 1024 : (BIAS ? 220 : 200) * 1024;  // tiles, per CTA
+  static constexpr int NS_RAW = (SMEM_BUDGET - TILES * (TILE + BIAS_TILE)) / TILE;
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
-  static constexpr int SMEM_BAR = TILES * TILE + NS * TILE;
+  static constexpr int OFF_BIAS = TILES * TILE + NS * TILE;
+  static constexpr int SMEM_BAR = OFF_BIAS + TILES * BIAS_TILE;
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers + alignment slack
   static constexpr int THREADS = 128 * TILES + 128;
   static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES]
@@ -84,11 +90,14 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
   static_assert(NS >= 2, "need at least two K/V slots");
+  static_assert(!BIAS || TILES == 2, "the staged bias needs the two-tile layout");
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
 
 
 struct FwdBarriers {
+  uint64_t bias_full[2];   // BIAS: tile t's bias tile for the current K/V step has landed
+  uint64_t bias_empty[2];  // BIAS: tile t's softmax warps have copied it out
   uint64_t q_full[2];
   uint64_t s_full[2];
   uint64_t p_full[2];
@@ -98,6 +107,7 @@ struct FwdBarriers {
   uint32_t tmem_base;
   int abort_flag;
 };
+static_assert(sizeof(FwdBarriers) <= 256, "barriers must fit the 256 bytes reserved for them");
 
 __device__ __forceinline__ float round_tf32(float x) {
   uint32_t r;
@@ -188,11 +198,13 @@ __device__ __forceinline__ void stage_v_transposed_tf32(const float* V, int bh, 
 // DROP: dropout on P (16-bit types only), masks drawn in the softmax warps.
 // BIAS: an additive bias on the scaled scores (16-bit types only).
 template <typename T, int D, bool CAUSAL, bool GEN, bool DROP, bool BIAS, int NT>
-__global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, NT>::CTAS_PER_SM)
+__global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<T, D, NT, BIAS>::CTAS_PER_SM)
     fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
-               FwdParams p) {
-  using Tr = FwdTraits<T, D, NT>;
+               const __grid_constant__ CUtensorMap tmBias, FwdParams p) {
+  using Tr = FwdTraits<T, D, NT, BIAS && !ElemTraits<T>::tf32>;
+  // staged bias tiles (16-bit types): the two-tile layout
+  constexpr bool SBIAS = BIAS && !ElemTraits<T>::tf32;
   constexpr bool TF32 = ElemTraits<T>::tf32;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -231,6 +243,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
       mbar_init(&bars->kv_full[i], 1);
       mbar_init(&bars->kv_empty[i], 1);
     }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&bars->bias_full[t], 1);
+      mbar_init(&bars->bias_empty[t], 128);
+    }
     bars->abort_flag = 0;
     fence_mbar_init();
   }
@@ -242,6 +258,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
     tma_prefetch_desc(&tmQ);
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
+    if constexpr (SBIAS) tma_prefetch_desc(&tmBias);
   }
   tc_fence_before();
   __syncthreads();
@@ -250,6 +267,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
 
   uint8_t* sQ[2] = {smem, smem + Tr::TILE};  // (the second only with two tiles)
   uint8_t* sKV = smem + Tr::TILES * Tr::TILE;
+  uint8_t* sBias = smem + Tr::OFF_BIAS;  // SBIAS: [TILES][2 halves][rows][128 B], swizzled
 
   if (warp > Tr::PRODUCER_WARP) {
     // idle warps of the producer/MMA warpgroup
@@ -291,17 +309,43 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
       load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
       return true;
     };
+    // SBIAS: K/V tile j's bias tile of each Q tile (two swizzled halves of
+    // 64 keys; one row each when the bias is shared by all query rows, its
+    // halves a swizzle atom apart), once that tile's softmax warps have
+    // copied out tile j − 1's.  Zero past Nq and Nk.
+    auto load_bias = [&](int j) {
+      for (int t = 0; t < Tr::TILES; ++t) {
+        bool ok = j == 0 || MBAR_WAIT(&bars->bias_empty[t], (j - 1) & 1, abort_flag);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) return false;
+        if (lane == 0 && FA_INBOUNDS(bh < p.B * p.H && j * Tr::BN < p.Nk)) {
+          const int rows = p.bias_rows, half = rows > 1 ? rows * 128 : 1024;
+          mbar_arrive_expect_tx(&bars->bias_full[t], 2 * rows * 128);
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tma_load_4d(sBias + t * Tr::BIAS_TILE + h * half, &tmBias, &bars->bias_full[t], j * Tr::BN + 64 * h,
+                        rows > 1 ? q_row0 + 128 * t : 0, (bh % p.H) % p.bias_H, (bh / p.H) % p.bias_B);
+        }
+      }
+      return true;
+    };
     load_tile(0, sQ[0], &bars->q_full[0], q_row0);
+    if constexpr (SBIAS) load_bias(0);
     load_kv(0);
     if constexpr (Tr::TILES == 2) load_tile(0, sQ[1], &bars->q_full[1], q_row0 + 128);
-    for (int i = 1; i < 2 * n_kv; ++i)
+    for (int i = 1; i < 2 * n_kv; ++i) {
+      if constexpr (SBIAS)
+        if ((i & 1) == 0 && !load_bias(i >> 1)) break;
       if (!load_kv(i)) break;
+    }
     if (lane == 0) {
       // Drain: wait until every issued load has landed before the CTA may exit.
       for (int i = max(0, 2 * n_kv - Tr::NS); i < 2 * n_kv; ++i)
         MBAR_WAIT(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       MBAR_WAIT(&bars->q_full[0], 0, abort_flag);
       if constexpr (Tr::TILES == 2) MBAR_WAIT(&bars->q_full[1], 0, abort_flag);
+      if constexpr (SBIAS)
+        for (int t = 0; t < Tr::TILES; ++t) MBAR_WAIT(&bars->bias_full[t], (n_kv - 1) & 1, abort_flag);
     }
   } else if (warp == Tr::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
@@ -433,24 +477,28 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
     float row_sum_p = 0.f;  // Σ of P as rounded for the P·V product: normalises O
     bool ok = true;
 
-    // bias row of this thread's query (batch b = bh / H, head h = bh % H)
-    const uint16_t* brow = nullptr;
-    if constexpr (BIAS && !TF32)
-      if (qi < p.Nq)
-        brow = reinterpret_cast<const uint16_t*>(p.bias) + (bh / p.H) * p.s_bias.b +
-               (bh % p.H) * p.s_bias.h + (long long)qi * p.s_bias.n;
+    // staged bias tile of this Q tile: chunk c (8 keys) of row rr at
+    // half c / 8, position (c % 8) ^ (rr % 8) of the row's 128 bytes
+    const uint8_t* btile = sBias + t * Tr::BIAS_TILE;
     for (int j = 0; j < n_kv; ++j) {
-      // Bias: this row's values for the tile's columns, loaded before S
-      // arrives so the loads overlap the wait (zero past Nk or past Nq).
-      uint4 bv[(BIAS && !TF32) ? Tr::BN / 8 : 1];
-      if constexpr (BIAS && !TF32) {
+      // Bias: this row's 128 values for the tile's columns, copied out of the
+      // staged tile before S arrives (zero past Nk or past Nq), which is then
+      // released for the next K/V tile's.
+      uint4 bv[SBIAS ? Tr::BN / 8 : 1];
+      if constexpr (SBIAS) {
+        ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->bias_full[t], j & 1, abort_flag));
+        if (!ok) break;
+        if (p.bias_rows > 1) {
 #pragma unroll
-        for (int v = 0; v < Tr::BN / 8; ++v) {
-          const int col = j * Tr::BN + 8 * v;
-          bv[v] = brow && FA_INBOUNDS(col < p.Nk || p.Nk - col <= 0)
-                      ? load8_16bit(brow + col, p.Nk - col)
-                      : make_uint4(0u, 0u, 0u, 0u);
+          for (int v = 0; v < Tr::BN / 8; ++v)
+            bv[v] = *reinterpret_cast<const uint4*>(btile + (v >> 3) * (128 * 128) + r * 128 +
+                                                   (((v & 7) ^ (r & 7)) << 4));
+        } else {  // one row shared by all queries
+#pragma unroll
+          for (int v = 0; v < Tr::BN / 8; ++v)
+            bv[v] = *reinterpret_cast<const uint4*>(btile + (v >> 3) * 1024 + ((v & 7) << 4));
         }
+        mbar_arrive(&bars->bias_empty[t]);
       }
       ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
       tc_fence_after();
@@ -671,7 +719,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT>::THREADS, FwdTraits<T, D, 
 template <typename T, int D, bool CAUSAL, bool GEN, bool DROP = false, bool BIAS = false,
           int NT = fwd_tiles(ElemTraits<T>::tf32, D)>
 static cudaError_t launch_fwd_t(const FwdLaunch& a) {
-  using Tr = FwdTraits<T, D, NT>;
+  using Tr = FwdTraits<T, D, NT, BIAS && !ElemTraits<T>::tf32>;
   if (a.params.tiles != NT) return cudaErrorInvalidValue;  // the grid was sized for another count
   auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP, BIAS, NT>;
   cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
@@ -687,15 +735,17 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   }
   if (!regs_ok) return cudaErrorInvalidConfiguration;
   dim3 grid(a.params.n_qblocks * a.params.H * a.params.B);
-  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.params);
+  kern<<<grid, Tr::THREADS, Tr::SMEM_BYTES, a.stream>>>(a.tmQ, a.tmK, a.tmV, a.tmO, a.tmBias, a.params);
   return cudaGetLastError();
 }
 
 int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
 
-int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool plain) {
+int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias) {
   const int dflt = fwd_tiles(dtype == FA_FP32, d);
-  if (dtype == FA_FP32 || d != 128 || !plain) return dflt;
+  if (dtype == FA_FP32 || d != 128) return dflt;
+  if (bias) return 2;  // the staged bias tiles need the two-tile layout
+  if (drop) return dflt;
   // K/V tiles a 128-row query tile sees, on average (bottom-right causal:
   // query tile i sees about i + 1 + (Nk − Nq) / 128 of them)
   const double kv_tiles = (Nk + 127) / 128;
@@ -712,10 +762,10 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
 #define FA_FWD_CASE(TY, DD)                                                                      \
   {                                                                                              \
     if (bias)                                                                                    \
-      return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true>(a)                   \
-                            : launch_fwd_t<TY, DD, true, true, false, true>(a))                 \
-                    : (drop ? launch_fwd_t<TY, DD, false, true, true, true>(a)                  \
-                            : launch_fwd_t<TY, DD, false, true, false, true>(a));               \
+      return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true, 2>(a)                \
+                            : launch_fwd_t<TY, DD, true, true, false, true, 2>(a))              \
+                    : (drop ? launch_fwd_t<TY, DD, false, true, true, true, 2>(a)               \
+                            : launch_fwd_t<TY, DD, false, true, false, true, 2>(a));            \
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \

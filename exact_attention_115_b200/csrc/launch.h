@@ -51,20 +51,22 @@ struct FwdParams {
   const void* bias;   // additive bias on the scaled scores, [B', H', Nq, Nk] input dtype; null = none
   Strides s_bias;     // its element strides (0 broadcasts a batch or head; columns contiguous)
   float bias_mul;     // 1 / scale: the bias in units of the unscaled scores
+  int bias_H, bias_B; // the bias tensor map's head and batch extents (1 where it broadcasts)
+  int bias_rows;      // rows of a staged bias tile: 128, or 1 for a bias shared by all query rows
 };
 
 struct FwdLaunch {
   CUtensorMap tmQ, tmK, tmV;
   CUtensorMap tmO;  // output, written by TMA stores (16-bit types)
+  CUtensorMap tmBias;  // bias: (key, query, head, batch), 128-byte-swizzled boxes of 64 keys
   FwdParams params;
   cudaStream_t stream;
 };
 
 // Elements in one 128-byte swizzled row for the dtype (the TMA box width).
 int fwd_tile_elems(int dtype);
-// 128-row Q tiles per forward CTA for a call (1 or 2); `plain` = no dropout
-// and no bias.
-int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool plain);
+// 128-row Q tiles per forward CTA for a call (1 or 2).
+int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias);
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a);
 
 struct BwdParams {
