@@ -10,8 +10,9 @@ HBM before the timed region; each step touches ~0.4 GB, larger than the
 126 MB L2, so no flush is inserted.  The decode workload (B=32, H=32,
 Nk=32768, d=128) is timed separately and reported under "decode", and the
 other training workloads (B4 H16 N1024 d64, B1 H32 N16384 d128 causal with
-Q×3, and the causal 2K one in fp16) under "other_workloads", each with its
-fwd, bwd and fwd+bwd TFLOPS against both measured bf16 peaks.
+Q×3, the causal 2K one in fp16, and again with a head-shared additive bias)
+under "other_workloads", each with its fwd, bwd and fwd+bwd TFLOPS against
+both measured bf16 peaks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
 
@@ -228,22 +229,28 @@ def peak_fracs(achieved, peaks):
                                                          FALLBACK_PEAKS["bf16_tflops_sustained"]))}
 
 
-def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None):
+def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_shape=None):
     """fwd and bwd of one workload, each launch bracketed by CUDA events on
     the launching stream (the main backward kernel by the library's own
     timing events); with ``flush`` (a buffer larger than L2) L2 is cleared
-    before every timed launch.  Returns the workload's sub-object."""
+    before every timed launch; with ``bias_shape`` an additive N(0, 1) bias
+    of that (broadcastable) shape is added to the scores.  FLOPs are counted
+    without the bias.  Returns the workload's sub-object."""
     q, k, v, do = W.make_inputs(w, device=dev)
-    O, L = fa.forward(q, k, v, causal=w.causal)
+    bias = None
+    if bias_shape is not None:
+        g = torch.Generator(device=dev).manual_seed(w.seed + 1)
+        bias = torch.randn(*bias_shape, generator=g, device=dev).to(q.dtype)
+    O, L = fa.forward(q, k, v, causal=w.causal, bias=bias)
     dq, dk, dv = (torch.empty_like(x) for x in (q, k, v))
     ws = torch.empty(fa.bwd_workspace_bytes(w.B, w.H, w.Nq, w.Nk, w.d, q.dtype), dtype=torch.uint8,
                      device=dev)
 
     def fwd():
-        fa.forward(q, k, v, causal=w.causal, out=O, lse=L)
+        fa.forward(q, k, v, causal=w.causal, out=O, lse=L, bias=bias)
 
     def bwd():
-        fa.backward(q, k, v, O, do, L, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws)
+        fa.backward(q, k, v, O, do, L, causal=w.causal, dq=dq, dk=dk, dv=dv, workspace=ws, bias=bias)
 
     for _ in range(3):
         fwd()
@@ -282,7 +289,11 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None):
         pk = f"{peak_kind} burst bf16 (fp16 runs at the bf16 rate)"
     else:
         pk = f"{peak_kind} burst bf16"
-    return {"workload": w.name, "shape": w.describe(), "iters": iters,
+    name, shape = w.name, w.describe()
+    if bias_shape is not None:
+        name += "_bias" + "x".join(str(x) for x in bias_shape)
+        shape += f", additive bias {list(bias_shape)} (FLOPs counted without it)"
+    return {"workload": name, "shape": shape, "iters": iters,
             "l2": "flushed before every timed launch" if flush is not None
                   else "inputs larger than L2; no flush",
             "fwd": {"ms": f_ms, "tflops": f_tf, **peak_fracs(f_tf, peaks)},
@@ -337,7 +348,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
-                    help="skip the other workloads (B4 H16 N1024 d64, the 16K causal one, fp16)")
+                    help="skip the other workloads (B4 H16 N1024 d64, the 16K causal one, fp16, with a bias)")
     ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode"],
                     help="run one kernel's small profiling case three times and exit "
                          "(the command an ncu capture wraps; nothing is timed)")
@@ -525,7 +536,9 @@ def main():
         iters = max(5, min(K, 20))
         others = [time_workload(fa, W.MEDIUM, dev, stream, iters, peaks, peak_kind, flush=flush),
                   time_workload(fa, W.LONG_16K, dev, stream, iters, peaks, peak_kind),
-                  time_workload(fa, W.CAUSAL_2K_FP16, dev, stream, iters, peaks, peak_kind)]
+                  time_workload(fa, W.CAUSAL_2K_FP16, dev, stream, iters, peaks, peak_kind),
+                  time_workload(fa, W.CAUSAL_2K, dev, stream, iters, peaks, peak_kind,
+                                bias_shape=(1, W.CAUSAL_2K.H, W.CAUSAL_2K.Nq, W.CAUSAL_2K.Nk))]
         del flush
         torch.cuda.empty_cache()
 
