@@ -7,6 +7,8 @@
 #include <cstring>
 #include <mutex>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "fa.h"
 #include "launch.h"
 
@@ -29,6 +31,15 @@ int cuda_fail(int code) {
   return FA_ERR_CUDA;
 }
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : cuda_fail(int(e)); }
+
+// A named NVTX range around each computing entry point, so that profiler
+// timelines show the library's calls (a no-op unless a tool is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
 
 // Tensor-map encoding is a driver call, which needs a current context on the
 // calling thread; a thread that has made no runtime call yet (an autograd
@@ -272,6 +283,7 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
               const fa_layout* lk, const fa_layout* lv, const fa_layout* lo, int B, int H, int Nq,
               int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
               const int* kv_len, const void* bias, const fa_layout* lbias, void* stream) {
+  NvtxRange nvtx_range("fa_fwd_ex");
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (!Q || !K || !V || !O || !L) return FA_ERR_INVALID;
@@ -367,6 +379,7 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
               int Nq, int Nk, int d, int causal, float scale, int dtype, const fa_dropout* dropout,
               const int* kv_len, const void* bias, const fa_layout* lbias, void* workspace,
               size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("fa_bwd_ex");
   int st = check_common(B, H, Nq, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   const void* ptrs[] = {Q, K, V, O, dO, L, dQ, dK, dV};
@@ -493,6 +506,7 @@ size_t fa_decode_workspace_bytes(int B, int H, int Nk, int d, int num_splits) {
 int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
                  int Nk, int d, float scale, int dtype, int num_splits, const int* kv_len,
                  void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_range("fa_decode_ex");
   int st = check_common(B, H, 1, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
@@ -534,6 +548,7 @@ int fa_decode(const void* Q, const void* K, const void* V, void* O, float* L, in
 
 int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, float* L, int B, int H,
                       int Nk, int d, float scale, int dtype, int num_splits, void* stream) {
+  NvtxRange nvtx_range("fa_decode_noalloc");
   int st = check_common(B, H, 1, Nk, d, scale, dtype);
   if (st != FA_OK) return st;
   if (dtype == FA_FP32) return FA_ERR_UNSUPPORTED;
