@@ -115,12 +115,14 @@ __device__ __forceinline__ float round_tf32(float x) {
   return __uint_as_float(r);
 }
 
-#ifndef FA_EXP2_EMU_PERIOD
-#define FA_EXP2_EMU_PERIOD 4
-#endif
-// One pair in every kEmuPeriod evaluates 2^x on the FMA pipe (exp2_pair<true>)
-// instead of the special-function unit, to balance the two pipes.
-constexpr int kEmuPeriod = FA_EXP2_EMU_PERIOD;
+// One pair in every emu_period(TILES) evaluates 2^x on the FMA pipe
+// (exp2_pair<true>) instead of the special-function unit, to balance the two
+// pipes; 0 = none.  Measured (d = 128 bf16 forward, interleaved A/B, periods
+// 4, 5, 6, 8 and none): the one-tile kernel is fastest with none (causal
+// N = 2048: 175.4 us with 1 in 4, 165.3 us with none), the two-tile kernel
+// with 1 in 5 (non-causal N = 8192: 961.5 us with 1 in 4, 945.0 with 1 in 5,
+// 1056.8 with none).
+constexpr int emu_period(int tiles) { return tiles == 1 ? 0 : 5; }
 
 // 2^x for a pair of floats on the FMA/ALU pipes: x = n + f with n = round(x)
 // (via the 1.5·2^23 rounding constant), f in [-1/2, 1/2]; 2^f from a degree-3
@@ -613,8 +615,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           for (int e = 0; e < 32; ++e) {
             const int q = (c + 2 * e) / 32;
             const uint64_t x = ffma2(pk2(s[c + 2 * e], s[c + 2 * e + 1]), c2, negm2);
-            // every kEmuPeriod-th pair of exponentials on the FMA pipe
-            const float2 pe = (e % kEmuPeriod == kEmuPeriod - 1) ? exp2_pair<true>(x)
+            // every emu_period-th pair of exponentials on the FMA pipe
+            constexpr int EP = emu_period(Tr::TILES);
+            const float2 pe = (EP > 0 && e % EP == EP - 1) ? exp2_pair<true>(x)
                                                                   : exp2_pair<false>(x);
             u[e] = ElemTraits<T>::pack2(pe.x, pe.y);
             const float2 pr = ElemTraits<T>::unpack2(u[e]);
