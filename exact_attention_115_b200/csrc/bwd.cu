@@ -89,6 +89,11 @@ struct BwdTraits {
   // d = 128 and no faster at d = 64: the P phase is not shortened by more
   // warps per sub-partition.
   static constexpr int NCW = 2;
+  // One pair of exponentials in EXP2_EMU of the P phase on the FMA pipe (0 =
+  // none).  Measured (interleaved A/B, periods 2, 4, 8 and none): d = 64 is
+  // fastest with 1 in 8 (B4 H16 N1024 backward 84.1 -> 79.2 us), d = 128
+  // with none (causal N = 2048: 463.9 us, 466.1 with 1 in 8).
+  static constexpr int EXP2_EMU = D == 64 ? 8 : 0;
   static constexpr int CWC = BM / NCW;               // query columns per compute warpgroup
   // d = 128: dQᵀ = Kᵀ dSᵀ with d on the TMEM lanes, so that a warp adds one
   // 128-byte line of the accumulator per query row.  (dQ = dS K with rows on
@@ -675,7 +680,15 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
                 nlq = ffma2(pk2(b2.x, b2.y), pk2(p.bias_l2, p.bias_l2), nlq);
               }
               const float2 x = upk2(ffma2(pk2(__uint_as_float(u[q]), __uint_as_float(u[q + 1])), c2, nlq));
-              float p0 = ex2(x.x), p1 = ex2(x.y);
+              float p0, p1;
+              if (Tr::EXP2_EMU > 0 && (q >> 1) % (Tr::EXP2_EMU > 0 ? Tr::EXP2_EMU : 1) == Tr::EXP2_EMU - 1) {
+                const float2 pe = exp2_pair_fma<true>(x);  // exactly 0 for masked entries
+                p0 = pe.x;
+                p1 = pe.y;
+              } else {
+                p0 = ex2(x.x);
+                p1 = ex2(x.y);
+              }
               if (need_mask) {
                 if (!key_live || (CAUSAL && q0 + q < qmin)) p0 = 0.f;
                 if (!key_live || (CAUSAL && q0 + q + 1 < qmin)) p1 = 0.f;

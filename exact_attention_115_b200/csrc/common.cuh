@@ -495,6 +495,35 @@ __device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+
+// 2^x for a pair of floats on the FMA/ALU pipes: x = n + f with n = round(x)
+// (via the 1.5·2^23 rounding constant), f in [-1/2, 1/2]; 2^f from a degree-3
+// polynomial with minimal maximum relative error (1.0e-4; coefficients from
+// gen_exp2_poly.py); 2^n added to the exponent field.  x is clamped at -125
+// so that masked (-inf) arguments cannot wrap the exponent: they give
+// ~2^-125, or exactly 0 with ZERO_BELOW.
+template <bool ZERO_BELOW>
+__device__ __forceinline__ float2 exp2_pair_fma(float2 x) {
+  const bool z0 = x.x < -125.f, z1 = x.y < -125.f;
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const uint64_t magic = pk2(12582912.f, 12582912.f);
+  const uint64_t t = fadd2(pk2(x.x, x.y), magic);
+  const uint64_t n = fadd2(t, pk2(-12582912.f, -12582912.f));
+  const uint64_t f = ffma2(n, pk2(-1.f, -1.f), pk2(x.x, x.y));
+  uint64_t pp = ffma2(pk2(0.05500893f, 0.05500893f), f, pk2(0.24221095f, 0.24221095f));
+  pp = ffma2(pp, f, pk2(0.6932829f, 0.6932829f));
+  pp = ffma2(pp, f, pk2(1.f, 1.f));
+  const float2 pv = upk2(pp), tv = upk2(t);
+  float2 r = make_float2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
+                         __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
+  if constexpr (ZERO_BELOW) {
+    if (z0) r.x = 0.f;
+    if (z1) r.y = 0.f;
+  }
+  return r;
+}
+
 __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
   uint64_t d;
   asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));

@@ -124,31 +124,15 @@ __device__ __forceinline__ float round_tf32(float x) {
 // 1056.8 with none).
 constexpr int emu_period(int tiles) { return tiles == 1 ? 0 : 5; }
 
-// 2^x for a pair of floats on the FMA/ALU pipes: x = n + f with n = round(x)
-// (via the 1.5·2^23 rounding constant), f in [-1/2, 1/2]; 2^f from a degree-3
-// polynomial with minimal maximum relative error (1.0e-4; coefficients from
-// gen_exp2_poly.py); 2^n added to the exponent field.  x is clamped at -125
-// so masked (-inf) scores give ~2^-125 instead of a wrapped exponent.
+// 2^x for a pair of floats: on the special-function unit, or (EMU) on the
+// FMA/ALU pipes (exp2_pair_fma in common.cuh).
 template <bool EMU>
 __device__ __forceinline__ float2 exp2_pair(uint64_t x2) {
-  if constexpr (!EMU) {
-    const float2 x = upk2(x2);
+  const float2 x = upk2(x2);
+  if constexpr (!EMU)
     return make_float2(ex2(x.x), ex2(x.y));
-  } else {
-    float2 x = upk2(x2);
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const uint64_t magic = pk2(12582912.f, 12582912.f);
-    const uint64_t t = fadd2(pk2(x.x, x.y), magic);
-    const uint64_t n = fadd2(t, pk2(-12582912.f, -12582912.f));
-    const uint64_t f = ffma2(n, pk2(-1.f, -1.f), pk2(x.x, x.y));
-    uint64_t pp = ffma2(pk2(0.05500893f, 0.05500893f), f, pk2(0.24221095f, 0.24221095f));
-    pp = ffma2(pp, f, pk2(0.6932829f, 0.6932829f));
-    pp = ffma2(pp, f, pk2(1.f, 1.f));
-    const float2 pv = upk2(pp), tv = upk2(t);
-    return make_float2(__int_as_float(__float_as_int(pv.x) + (__float_as_int(tv.x) << 23)),
-                       __int_as_float(__float_as_int(pv.y) + (__float_as_int(tv.y) << 23)));
-  }
+  else
+    return exp2_pair_fma<false>(x);
 }
 
 // fp32 inputs (TF32 tensor-core products).  The tensor core reads only the

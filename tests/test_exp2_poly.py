@@ -1,5 +1,6 @@
-"""The FMA-pipe exp2 used for part of the forward softmax: its coefficients
-in fwd.cu are the ones the committed fit produces, and the float32 evaluation
+"""The FMA-pipe exp2 used for part of the softmax exponentials (forward and,
+at d = 64, backward): its coefficients in common.cuh are the ones the
+committed fit produces, and the float32 evaluation
 (same steps as the kernel) stays within the fit's relative-error bound of
 numpy's exp2 over the whole range the kernel uses."""
 import importlib.util
@@ -20,8 +21,8 @@ def _gen():
 
 
 def _kernel_coefficients():
-    src = open(os.path.join(CSRC, "fwd.cu")).read()
-    body = src[src.index("__device__ __forceinline__ float2 exp2_pair"):]
+    src = open(os.path.join(CSRC, "common.cuh")).read()
+    body = src[src.index("__device__ __forceinline__ float2 exp2_pair_fma"):]
     body = body[:body.index("\n}\n")]
     c3, c2 = map(float, re.search(r"ffma2\(pk2\(([-0-9.e]+)f, \1f\), f, pk2\(([-0-9.e]+)f", body).groups())
     c1 = float(re.search(r"ffma2\(pp, f, pk2\(([-0-9.e]+)f", body).group(1))
