@@ -147,6 +147,7 @@ class ClockSampler:
         import threading
 
         self.samples = []
+        self._stop.clear()
         self.sample()
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
@@ -229,13 +230,17 @@ def peak_fracs(achieved, peaks):
                                                          FALLBACK_PEAKS["bf16_tflops_sustained"]))}
 
 
-def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_shape=None):
+def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_shape=None,
+                  sampler=None):
     """fwd and bwd of one workload, each launch bracketed by CUDA events on
     the launching stream (the main backward kernel by the library's own
     timing events); with ``flush`` (a buffer larger than L2) L2 is cleared
     before every timed launch; with ``bias_shape`` an additive N(0, 1) bias
     of that (broadcastable) shape is added to the scores.  FLOPs are counted
-    without the bias.  Returns the workload's sub-object."""
+    without the bias.  The timed loop starts after a short pause, so that a
+    workload is not measured at the clock its predecessor left (a long one
+    runs into the power cap), and ``sampler`` records the clocks during it.
+    Returns the workload's sub-object."""
     q, k, v, do = W.make_inputs(w, device=dev)
     bias = None
     if bias_shape is not None:
@@ -260,6 +265,9 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_
         for x in e:
             x.record(stream)
     torch.cuda.synchronize()
+    time.sleep(0.3)
+    if sampler is not None:
+        sampler.start()
     for e in ev:
         if flush is not None:
             flush.zero_()
@@ -273,6 +281,7 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_
         bwd()
         e[3].record(stream)
     torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler is not None else None
     fa.set_bwd_timing_events(None, None)
     st = fa.status()
     if st != fa.FA_OK:
@@ -301,7 +310,8 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_
                     "main_kernel_tflops": main_tf, **peak_fracs(b_tf, peaks)},
             "fwd_bwd": {"ms": f_ms + b_ms, "tflops": fb_tf, **peak_fracs(fb_tf, peaks)},
             "roofline": {"bound": "tensor", "kernel": "bwd_main_kernel", "achieved": main_tf,
-                         "peak": peak, "unit": UNIT, "frac": main_tf / peak, "peak_kind": pk}}
+                         "peak": peak, "unit": UNIT, "frac": main_tf / peak, "peak_kind": pk},
+            "clocks": clocks}
 
 
 # Decode shape for kernel captures: the decode workload with B = 4 instead of
@@ -534,11 +544,14 @@ def main():
         l2 = torch.cuda.get_device_properties(dev).L2_cache_size
         flush = torch.empty(4 * l2, dtype=torch.uint8, device=dev)  # written before each launch
         iters = max(5, min(K, 20))
-        others = [time_workload(fa, W.MEDIUM, dev, stream, iters, peaks, peak_kind, flush=flush),
-                  time_workload(fa, W.LONG_16K, dev, stream, iters, peaks, peak_kind),
-                  time_workload(fa, W.CAUSAL_2K_FP16, dev, stream, iters, peaks, peak_kind),
+        others = [time_workload(fa, W.MEDIUM, dev, stream, iters, peaks, peak_kind, flush=flush,
+                                sampler=sampler),
+                  time_workload(fa, W.LONG_16K, dev, stream, iters, peaks, peak_kind, sampler=sampler),
+                  time_workload(fa, W.CAUSAL_2K_FP16, dev, stream, iters, peaks, peak_kind,
+                                sampler=sampler),
                   time_workload(fa, W.CAUSAL_2K, dev, stream, iters, peaks, peak_kind,
-                                bias_shape=(1, W.CAUSAL_2K.H, W.CAUSAL_2K.Nq, W.CAUSAL_2K.Nk))]
+                                bias_shape=(1, W.CAUSAL_2K.H, W.CAUSAL_2K.Nq, W.CAUSAL_2K.Nk),
+                                sampler=sampler)]
         del flush
         torch.cuda.empty_cache()
 
