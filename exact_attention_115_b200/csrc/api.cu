@@ -395,8 +395,10 @@ int fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const 
       if (!is_contiguous(*lays[i], H, rows[i], d)) return FA_ERR_UNSUPPORTED;
   }
   if (causal && Nq > Nk) return FA_ERR_UNSUPPORTED;
-  // grids: (rows, B·H) for the per-row kernels, one CTA per (K/V block, head)
-  if (int64_t(B) * H > 65535 || int64_t((Nk + 127) / 128) * B * H > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  // 1-D grids: (head, row block) for the per-row kernels, work items per (K/V block, head)
+  if (int64_t((bwd_pad_rows(Nq) + 15) / 16) * B * H > INT32_MAX ||
+      int64_t((Nk + 127) / 128) * B * H > INT32_MAX)
+    return FA_ERR_UNSUPPORTED;
   DropoutParams drop;
   st = dropout_params(dropout, &drop);
   if (st != FA_OK) return st;
@@ -518,7 +520,7 @@ int fa_decode_ex(const void* Q, const void* K, const void* V, void* O, float* L,
   const int BH = B * H;
   int s = num_splits > 0 ? num_splits : decode_auto_splits(BH, Nk);
   s = std::min(s, Nk);
-  if (s > 65535) return FA_ERR_UNSUPPORTED;
+  if (s > 65535 || int64_t(s) * BH > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid of (head, part)
   const int kps = decode_keys_per_split(Nk, s);
   s = (Nk + kps - 1) / kps;
   const size_t need = fa_decode_workspace_bytes(B, H, Nk, d, num_splits);
@@ -566,7 +568,7 @@ int fa_decode_noalloc(const void* Q, const void* K, const void* V, void* O, floa
   s = std::min(s, Nk);
   if (num_splits == 0)
     while (s > 1 && need_for(s) > cap) --s;  // automatic: fewer parts until they fit
-  if (s > 65535) return FA_ERR_UNSUPPORTED;
+  if (s > 65535 || int64_t(s) * BH > INT32_MAX) return FA_ERR_UNSUPPORTED;  // 1-D grid of (head, part)
   const int kps = decode_keys_per_split(Nk, s);
   s = (Nk + kps - 1) / kps;
   if (need_for(s) > cap) return FA_ERR_WORKSPACE;  // beyond the built-in scratch

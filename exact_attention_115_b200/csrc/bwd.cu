@@ -934,16 +934,18 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
 // rows, so their P is 0), stored negated so the main kernel adds them; in
 // mode 1 the fp32 dQ accumulator is cleared.
 // A group of D/8 lanes handles one row (8 elements per lane).  Heads go in
-// the reverse of the main kernel's order (blocks run y-major), so the first
-// heads the main kernel takes are the last ones written here, still in L2.
+// the reverse of the main kernel's order (blocks run in index order, a
+// head's row blocks consecutive), so the first heads the main kernel takes
+// are the last ones written here, still in L2.
 template <typename T, int D, bool GEN>
 __global__ void __launch_bounds__(256) bwd_preprocess_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;  // rows per block
   const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
-  const int bh = int(gridDim.y) - 1 - int(blockIdx.y);
-  const int q = blockIdx.x * RPB + g;
-  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *p.item_ctr = 0;
+  const unsigned nrb = unsigned(p.Nq_pad + RPB - 1) / RPB;  // row blocks per head (1-D grid)
+  const int bh = p.B * p.H - 1 - int(blockIdx.x / nrb);
+  const int q = int(blockIdx.x % nrb) * RPB + g;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.item_ctr = 0;
   if (q >= p.Nq_pad || !FA_INBOUNDS(bh < p.B * p.H)) return;
   float dsum = 0.f;
   float lsc = INFINITY;
@@ -990,9 +992,10 @@ __global__ void __launch_bounds__(256) bwd_dq_finalise_kernel(BwdParams p) {
   constexpr int LPR = D / 8;
   constexpr int RPB = 256 / LPR;
   const int g = threadIdx.x / LPR, sl = threadIdx.x % LPR;
-  const int bh = int(gridDim.y) - 1 - int(blockIdx.y);
-  const int q = blockIdx.x * RPB + g;
-  if (q >= p.Nq || !FA_INBOUNDS(bh < p.B * p.H)) return;
+  const unsigned nrb = unsigned(p.Nq + RPB - 1) / RPB;  // row blocks per head (1-D grid)
+  const int bh = p.B * p.H - 1 - int(blockIdx.x / nrb);
+  const int q = int(blockIdx.x % nrb) * RPB + g;
+  if (q >= p.Nq || !FA_INBOUNDS(bh >= 0 && bh < p.B * p.H)) return;
   float acc[8];
   const size_t row = size_t(bh) * p.Nq_pad + q;
   if (p.dq_mode >= 2) {
@@ -1142,7 +1145,8 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
   const BwdParams& p = a.params;
   constexpr int RPB = 256 / (D / 8);
   const int BH = p.B * p.H;
-  bwd_preprocess_kernel<T, D, GEN><<<dim3((p.Nq_pad + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  // 1-D grids over (head, row block): B·H may exceed a grid's second dimension
+  bwd_preprocess_kernel<T, D, GEN><<<unsigned((p.Nq_pad + RPB - 1) / RPB) * unsigned(BH), 256, 0, a.stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   auto kern = bwd_main_kernel<T, D, CAUSAL, GEN, DROP, BIAS>;
@@ -1172,7 +1176,7 @@ static cudaError_t launch_bwd_t(const BwdLaunch& a) {
     e = cudaEventRecord(a.ev_stop, a.stream);
     if (e != cudaSuccess) return e;
   }
-  bwd_dq_finalise_kernel<T, D, CAUSAL, GEN><<<dim3((p.Nq + RPB - 1) / RPB, BH), 256, 0, a.stream>>>(p);
+  bwd_dq_finalise_kernel<T, D, CAUSAL, GEN><<<unsigned((p.Nq + RPB - 1) / RPB) * unsigned(BH), 256, 0, a.stream>>>(p);
   return cudaGetLastError();
 }
 

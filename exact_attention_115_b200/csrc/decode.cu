@@ -65,7 +65,9 @@ __global__ void __launch_bounds__(kDecodeThreads)
   constexpr int KPW = 32 / LPK;             // key rows per warp per load
   constexpr int NW = kDecodeThreads / 32;   // warps
   constexpr int GROUPS = NW * KPW;          // independent softmax states per CTA
-  const int part = blockIdx.x, bh = blockIdx.y;
+  // one CTA per (head, part), parts of a head consecutive (a 1-D grid: B·H
+  // may exceed the 65535 of a grid's second dimension)
+  const int part = int(blockIdx.x % unsigned(p.splits)), bh = int(blockIdx.x / unsigned(p.splits));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int sub = lane / LPK, sl = lane % LPK;  // key slot in the warp, lane in the group
 
@@ -192,8 +194,7 @@ __global__ void __launch_bounds__(D) decode_combine_kernel(DecodeParams p) {
 
 template <typename T, int D>
 static cudaError_t launch_decode_t(const DecodeParams& p, cudaStream_t s) {
-  dim3 g1(p.splits, p.BH);
-  decode_split_kernel<T, D><<<g1, kDecodeThreads, 0, s>>>(p);
+  decode_split_kernel<T, D><<<unsigned(p.splits) * unsigned(p.BH), kDecodeThreads, 0, s>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   decode_combine_kernel<T, D><<<p.BH, D, 0, s>>>(p);

@@ -55,7 +55,7 @@ typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID = -1,     /* null pointer, size <= 0, non-finite scale, misaligned pointer */
   FA_ERR_UNSUPPORTED = -2, /* d not in {64,128}, fp32 with d=128, causal with Nq > Nk,
-                              backward with B*H > 65535 */
+                              B or H > 65535, a grid of more than 2^31 - 1 blocks */
   FA_ERR_WORKSPACE = -3,   /* workspace pointer null or smaller than the query says */
   FA_ERR_CUDA = -4,        /* a CUDA runtime error at launch or in fa_status */
   FA_ERR_TIMEOUT = -5,     /* a kernel's bounded wait expired (reported by fa_status) */
