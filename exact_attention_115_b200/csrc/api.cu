@@ -324,10 +324,13 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
                                        &a.params.bias_H, &a.params.bias_B, &a.params.bias_rows);
     if (r != CUDA_SUCCESS) return cuda_fail(100000 + int(r));
   }
+  // Q tiles per CTA and K/V tile rows (3: one Q tile over 64-key K/V tiles)
+  a.params.tiles = fwd_tiles_for(dtype, d, Nq, Nk, causal != 0, drop.t4 != 0, bias != nullptr);
+  const int kv_rows = a.params.tiles == 3 ? 64 : 128;
   bool m4[4];
   if (!make_map(&a.tmQ, Q, dtype, d, Nq, H, B, *lq, 128, &m4[0]) ||
-      !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, 128, &m4[1]) ||
-      !make_map(&a.tmV, V, dtype, d, Nk, H, B, *lv, 128, &m4[2]) ||
+      !make_map(&a.tmK, K, dtype, d, Nk, H, B, *lk, kv_rows, &m4[1]) ||
+      !make_map(&a.tmV, V, dtype, d, Nk, H, B, *lv, kv_rows, &m4[2]) ||
       !make_map(&a.tmO, O, dtype, d, Nq, H, B, *lo, 128, &m4[3]))
     return FA_ERR_CUDA;
   for (int i = 0; i < 4; ++i) a.params.map4d |= int(m4[i]) << i;
@@ -341,8 +344,7 @@ int fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* L, co
   a.params.Nq = Nq;
   a.params.Nk = Nk;
   a.params.scale_log2 = scale * 1.4426950408889634f;
-  a.params.tiles = fwd_tiles_for(dtype, d, Nq, Nk, causal != 0, drop.t4 != 0, bias != nullptr);
-  const int rows = 128 * a.params.tiles;
+  const int rows = a.params.tiles == 2 ? 256 : 128;  // query rows per CTA
   a.params.n_qblocks = (Nq + rows - 1) / rows;
   a.params.head_group = head_group_for(size_t(Nk) * d * 2 * elem_size(dtype), BH);
   a.stream = static_cast<cudaStream_t>(stream);

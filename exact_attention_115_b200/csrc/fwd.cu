@@ -12,15 +12,21 @@
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
-// (fwd_tiles_for: two, except one for 16-bit d = 128 when a query tile sees
-// fewer than 12 K/V tiles on average).  With two tiles it ping-pongs them so
-// the tensor core works on one tile while the softmax warps work on the
-// other; with one tile two CTAs share an SM and interleave the same way.  Roles per CTA (128 threads per tile + 128):
+// (fwd_tiles_for: two, except for 16-bit d = 128 when a query tile sees
+// fewer than 24 K/V tiles of 128 keys on average, or 48 under the causal
+// mask).  With two tiles it ping-pongs them over 128-key K/V tiles so the
+// tensor core works on one tile while the softmax warps work on the other.
+// With one tile (NT = 3) the K/V tiles have 64 keys and the score tile is
+// double-buffered in TMEM, so the scores of K/V tile j + 1 are computed
+// while the softmax of tile j runs; two such CTAs share an SM.  (NT = 1, one
+// tile over 128-key K/V tiles with one score buffer, serves the dropout
+// variants.)  Roles per CTA (128 threads per tile + 128):
 //   warpgroup t (warps 4t..4t+3)  softmax + correction + epilogue of Q tile t
 //                                 (thread = row), 200 registers
 //   last warpgroup: warp 4·TILES issues the tcgen05 MMAs (one thread) and
 //                   owns TMEM, the next warp is the TMA producer, the rest idle
-// TMEM: S[tiles] | O[tiles] (256 or 512 columns).  P overwrites S in place
+// TMEM: S[tiles] | O[tiles] (256 or 512 columns), or S0 | S1 | O (64, 64 and
+// d columns) with double-buffered scores.  P overwrites S in place
 // (bf16 pairs or tf32) and is read by the P·V MMA straight from TMEM.  The
 // running max is only moved when it grows by more than kRescaleThreshold
 // (log2 units), so the O accumulator is rescaled rarely; the result is exact
@@ -47,26 +53,30 @@ constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entr
 // d = 128 kernels come with either count; see fwd_tiles_for).
 constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 1 : 2; }
 
+// NT: 1 or 2 Q tiles of 128 rows per CTA over K/V tiles of 128 keys, or 3:
+// one Q tile over K/V tiles of 64 keys with its score tile double-buffered
+// in TMEM (S0 | S1 | O = 64 + 64 + d columns), so that the next score tile
+// is computed while the softmax of the current one runs.
 template <typename T, int D, int NT = fwd_tiles(ElemTraits<T>::tf32, D), bool BIAS = false>
 struct FwdTraits {
   static constexpr int ES = sizeof(T);
-  static constexpr int BN = 128;                 // keys of a K/V tile
+  static constexpr int BN = NT == 3 ? 64 : 128;  // keys of a K/V tile
+  static constexpr int SBUF = NT == 3 ? 2 : 1;   // score buffers per Q tile
   static constexpr int AW = 128 / ES;            // elements per 128-byte swizzled row
   static constexpr int DC = D / AW;              // 128-byte column blocks in a row
-  static constexpr int CHUNK = 128 * 128;        // bytes of one column block (128 rows)
-  static constexpr int TILE = 128 * D * ES;      // bytes of one 128-row tile
+  static constexpr int CHUNK = 128 * 128;        // bytes of one column block of a Q (or O) tile
+  static constexpr int TILE = 128 * D * ES;      // bytes of one 128-row Q (or O) tile
+  static constexpr int KV_CHUNK = BN * 128;      // bytes of one column block of a K/V tile
+  static constexpr int KV_TILE = BN * D * ES;    // bytes of one K/V tile
   static constexpr int KSTEP = 32 / ES;          // K extent of one MMA instruction
   // 128-row Q tiles per CTA.  With one tile a CTA needs 256 TMEM columns and
   // under half of shared memory, so two CTAs share an SM: one's softmax runs
   // while the other's products run, and one's set-up and epilogue overlap the
   // other's main loop, at the price of loading each K/V tile twice per SM.
   // With two tiles the CTA ping-pongs its own tiles over one K/V stream.
-  // Measured (d = 128, bf16): one tile is faster when a query tile sees few
-  // K/V tiles (causal N = 1024: 113 vs 121 us; causal N = 2048: 174 vs
-  // 176 us), two when it sees many (causal N = 4096, 8192, 16384 and
-  // non-causal N = 2048, 8192: 6-10 % faster), as the CTA's set-up and
-  // epilogue are then spread over more tiles.  d = 64: two tiles (+5 %).
-  static constexpr int TILES = NT;
+  // Which count is faster depends on how many K/V tiles a query tile sees
+  // (measurements at fwd_tiles_for).  d = 64: two tiles (+5 %).
+  static constexpr int TILES = NT == 2 ? 2 : 1;
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
   // The bias variants (two tiles) stage each K/V step's [128 rows × 128 keys]
   // bias tile of every Q tile in shared memory: two 128-byte-swizzled halves
@@ -74,13 +84,14 @@ struct FwdTraits {
   static constexpr int BIAS_TILE = BIAS ? 128 * BN * ES : 0;
   static constexpr int SMEM_BUDGET =
       TILES == 1 ? 110 * 1024 : (BIAS ? 220 : 200) * 1024;  // tiles, per CTA
-  static constexpr int NS_RAW = (SMEM_BUDGET - TILES * (TILE + BIAS_TILE)) / TILE;
+  static constexpr int NS_RAW = (SMEM_BUDGET - TILES * (TILE + BIAS_TILE)) / KV_TILE;
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
-  static constexpr int OFF_BIAS = TILES * TILE + NS * TILE;
+  static constexpr int OFF_BIAS = TILES * TILE + NS * KV_TILE;
   static constexpr int SMEM_BAR = OFF_BIAS + TILES * BIAS_TILE;
   static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers + alignment slack
   static constexpr int THREADS = 128 * TILES + 128;
-  static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES]
+  static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES], or S0 | S1 | O
+  static constexpr int COL_O = TILES * SBUF * BN;            // first O column
   static constexpr int MMA_WARP = 4 * TILES;                // then the TMA producer
   static constexpr int PRODUCER_WARP = MMA_WARP + 1;
   // setmaxnreg split of the registers a CTA launches with (65536 / CTAS_PER_SM)
@@ -89,7 +100,9 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
-  static_assert(NS >= 2, "need at least two K/V slots");
+  static_assert(NS >= 2 * SBUF, "K/V slots for the products in flight");
+  static_assert(NT != 3 || (!BIAS && !ElemTraits<T>::tf32), "64-key tiles: 16-bit, no bias");
+  static_assert(COL_O + TILES * D <= TMEM_COLS, "TMEM budget");
   static_assert(!BIAS || TILES == 2, "the staged bias needs the two-tile layout");
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
@@ -279,10 +292,11 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         // (a tile may start past the end only by the CTA's second Q tile:
         // TMA fills its rows with zeros)
         if (!FA_INBOUNDS(bh < p.B * p.H && row >= 0 && row < (which == 0 ? p.Nq + 128 : p.Nk))) return;
-        mbar_arrive_expect_tx(bar, Tr::TILE);
+        const int bytes = which == 0 ? Tr::TILE : Tr::KV_TILE, chunk = which == 0 ? Tr::CHUNK : Tr::KV_CHUNK;
+        mbar_arrive_expect_tx(bar, bytes);
 #pragma unroll
         for (int c = 0; c < Tr::DC; ++c)
-          tma_load_bh(dst + c * Tr::CHUNK, map, GEN && ((p.map4d >> which) & 1), bar, c * Tr::AW, row, bh, p.H);
+          tma_load_bh(dst + c * chunk, map, GEN && ((p.map4d >> which) & 1), bar, c * Tr::AW, row, bh, p.H);
       }
     };
     auto load_kv = [&](int i) {  // i-th K/V tile in consumption order: K0 V0 K1 V1 ...
@@ -292,7 +306,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         ok = MBAR_WAIT(&bars->kv_empty[slot], ((i / Tr::NS) - 1) & 1, abort_flag);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
-      load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
+      load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::KV_TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
       return true;
     };
     // SBIAS: K/V tile j's bias tile of each Q tile (two swizzled halves of
@@ -340,8 +354,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
     // arithmetic); the elected lane issues the MMAs and commits.
     {
       const bool leader = elect_one();
-      const uint32_t tS[2] = {tmem, tmem + 128};
-      const uint32_t tO[2] = {tmem + 128 * Tr::TILES, tmem + 128 * Tr::TILES + D};
+      // score buffers: tile t (two tiles), or buffer b of the one tile (NT = 3)
+      const uint32_t tS[2] = {tmem, tmem + Tr::BN};
+      const uint32_t tO[2] = {tmem + Tr::COL_O, tmem + Tr::COL_O + D};
       const uint32_t aQ[2] = {smem_u32(sQ[0]), smem_u32(sQ[1])};
       const uint32_t aKV = smem_u32(sKV);
 
@@ -349,26 +364,28 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
       // loops each MMA only adds a compile-time offset (in 16-byte units), so
       // the issuing thread keeps ahead of the tensor core.
       const uint64_t descQ[2] = {sw128_desc(aQ[0], 16, 1024), sw128_desc(aQ[1], 16, 1024)};
-      auto issue_qk = [&](int t, int slot) {
+      // S of Q tile t (or into score buffer b: sb) = Q_t · K(slot)ᵀ
+      auto issue_qk = [&](int t, int slot, int sb) {
         const uint64_t da = descQ[t];
-        const uint64_t db = sw128_desc(aKV + slot * Tr::TILE, 16, 1024);
+        const uint64_t db = sw128_desc(aKV + slot * Tr::KV_TILE, 16, 1024);
 #pragma unroll
         for (int ks = 0; ks < D / Tr::KSTEP; ++ks) {
-          constexpr int kChunk16 = Tr::CHUNK / 16;
-          const uint64_t o = uint64_t((ks >> 2) * kChunk16 + (ks & 3) * 2);
-          if (leader) mma_ss<TF32>(tS[t], da + o, db + o, Tr::IDESC_QK, ks > 0);
+          const uint64_t oa = uint64_t((ks >> 2) * (Tr::CHUNK / 16) + (ks & 3) * 2);
+          const uint64_t ob = uint64_t((ks >> 2) * (Tr::KV_CHUNK / 16) + (ks & 3) * 2);
+          if (leader) mma_ss<TF32>(tS[sb], da + oa, db + ob, Tr::IDESC_QK, ks > 0);
         }
       };
-      auto issue_pv = [&](int t, int slot, bool acc) {
-        const uint32_t vb = aKV + slot * Tr::TILE;
+      // O of Q tile t += P (score buffer sb) · V(slot)
+      auto issue_pv = [&](int t, int slot, bool acc, int sb) {
+        const uint32_t vb = aKV + slot * Tr::KV_TILE;
         // 16-bit: V tile [key][d] is an MN-major B operand; step = KSTEP key rows.
         // TF32: V tile was stored transposed ([d][key], K-major); step = 32 bytes.
-        const uint64_t db = TF32 ? sw128_desc(vb, 16, 1024) : sw128_desc(vb, Tr::CHUNK, 1024);
+        const uint64_t db = TF32 ? sw128_desc(vb, 16, 1024) : sw128_desc(vb, Tr::KV_CHUNK, 1024);
 #pragma unroll
         for (int ks = 0; ks < Tr::BN / Tr::KSTEP; ++ks) {
           const uint64_t o = TF32 ? uint64_t((ks >> 2) * (D * 8) + (ks & 3) * 2)
                                   : uint64_t(ks * Tr::KSTEP * 8);
-          if (leader) mma_ts<TF32>(tO[t], tS[t] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
+          if (leader) mma_ts<TF32>(tO[t], tS[sb] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
         }
       };
       auto commit = [&](uint64_t* bar) {
@@ -378,12 +395,49 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         return MBAR_WAIT_WARP(&bars->kv_full[i % Tr::NS], (i / Tr::NS) & 1, abort_flag);
       };
 
-      if constexpr (Tr::TILES == 1) {
+      if constexpr (Tr::SBUF == 2) {
+        // One tile, two score buffers: S(0) and S(1) first; then for each j,
+        // once the softmax has written P(j) into buffer j % 2, P(j)·V(j) and
+        // S(j+2) into the same buffer (in issue order after P·V read P).  The
+        // softmax of tile j+1 runs while these products do.  K/V come in the
+        // producer's order K0 V0 K1 V1 …: K(j+1) is taken before V(j).
+        bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
+        tc_fence_after();
+        if (ok) issue_qk(0, 0, 0);
+        commit(&bars->s_full[0]);
+        commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
+        if (ok && n_kv > 1) {
+          ok = kv_wait(2);
+          tc_fence_after();
+          if (ok) issue_qk(0, 2 % Tr::NS, 1);
+          commit(&bars->s_full[1]);
+          commit(&bars->kv_empty[2 % Tr::NS]);
+        }
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int b = j & 1, iv = 2 * j + 1, ik = 2 * j + 4;
+          const int sv = iv % Tr::NS, sk = ik % Tr::NS;
+          ok = kv_wait(iv) && MBAR_WAIT_WARP(&bars->p_full[b], (j >> 1) & 1, abort_flag);
+          tc_fence_after();
+          if (!ok) break;
+          issue_pv(0, sv, j > 0, b);
+          commit(&bars->o_full[0]);
+          if (j + 1 == n_kv) commit(&bars->o_full[1]);  // the tile's last product, for the epilogue
+          commit(&bars->kv_empty[sv]);
+          if (j + 2 < n_kv) {
+            ok = kv_wait(ik);
+            tc_fence_after();
+            if (!ok) break;
+            issue_qk(0, sk, b);
+            commit(&bars->s_full[b]);
+            commit(&bars->kv_empty[sk]);
+          }
+        }
+      } else if constexpr (Tr::TILES == 1) {
         // One tile: S(j), then (once the softmax has written P(j)) P(j)·V(j)
         // and S(j+1) into the same columns, in issue order after P·V read P.
         bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
         tc_fence_after();
-        if (ok) issue_qk(0, 0);
+        if (ok) issue_qk(0, 0, 0);
         commit(&bars->s_full[0]);
         commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
         for (int j = 0; j < n_kv && ok; ++j) {
@@ -392,14 +446,14 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           ok = kv_wait(iv) && MBAR_WAIT_WARP(&bars->p_full[0], j & 1, abort_flag);
           tc_fence_after();
           if (!ok) break;
-          issue_pv(0, sv, j > 0);
+          issue_pv(0, sv, j > 0, 0);
           commit(&bars->o_full[0]);
           commit(&bars->kv_empty[sv]);
           if (j + 1 < n_kv) {
             ok = kv_wait(ik);
             tc_fence_after();
             if (!ok) break;
-            issue_qk(0, sk);
+            issue_qk(0, sk, 0);
             commit(&bars->s_full[0]);
             commit(&bars->kv_empty[sk]);
           }
@@ -407,11 +461,11 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
       } else {
       bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
       tc_fence_after();
-      if (ok) issue_qk(0, 0);
+      if (ok) issue_qk(0, 0, 0);
       commit(&bars->s_full[0]);
       ok = ok && MBAR_WAIT_WARP(&bars->q_full[1], 0, abort_flag);
       tc_fence_after();
-      if (ok) issue_qk(1, 0);
+      if (ok) issue_qk(1, 0, 1);
       commit(&bars->s_full[1]);
       commit(&bars->kv_empty[0]);
       for (int j = 0; j < n_kv && ok; ++j) {
@@ -421,24 +475,24 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         ok = ok && MBAR_WAIT_WARP(&bars->p_full[0], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
-        issue_pv(0, sv, j > 0);
+        issue_pv(0, sv, j > 0, 0);
         commit(&bars->o_full[0]);
         const bool more = j + 1 < n_kv;
         if (more) {
           ok = kv_wait(ik);
           tc_fence_after();
           if (!ok) break;
-          issue_qk(0, sk);
+          issue_qk(0, sk, 0);
           commit(&bars->s_full[0]);
         }
         ok = MBAR_WAIT_WARP(&bars->p_full[1], j & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
-        issue_pv(1, sv, j > 0);
+        issue_pv(1, sv, j > 0, 1);
         commit(&bars->o_full[1]);
         commit(&bars->kv_empty[sv]);
         if (more) {
-          issue_qk(1, sk);
+          issue_qk(1, sk, 1);
           commit(&bars->s_full[1]);
           commit(&bars->kv_empty[sk]);
         }
@@ -453,8 +507,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
     const int r = quad * 32 + lane;  // row in the tile = TMEM lane
     const int qi = q_row0 + t * 128 + r;
     const uint32_t lane_off = uint32_t(quad * 32) << 16;
-    const uint32_t tS = tmem + lane_off + t * 128;
-    const uint32_t tO = tmem + lane_off + 128 * Tr::TILES + t * D;
+    const uint32_t tS0 = tmem + lane_off + t * 128;  // S of tile t (or score buffer 0)
+    const uint32_t tO = tmem + lane_off + Tr::COL_O + t * D;
     const float sl2 = p.scale_log2;
     const int tile_first_row = q_row0 + t * 128;
 
@@ -486,10 +540,14 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         }
         mbar_arrive(&bars->bias_empty[t]);
       }
-      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[t], j & 1, abort_flag));
+      // score buffer of K/V tile j: the tile's own, or j % 2 of two
+      const int sb = Tr::SBUF == 2 ? (j & 1) : t;
+      const uint32_t sph = Tr::SBUF == 2 ? ((j >> 1) & 1) : (j & 1);
+      const uint32_t tS = tS0 + (Tr::SBUF == 2 ? (j & 1) * Tr::BN : 0);
+      ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->s_full[sb], sph, abort_flag));
       tc_fence_after();
       if (!ok) break;
-      uint32_t su[4][32];
+      uint32_t su[Tr::BN / 32][32];
       if constexpr (BIAS && !TF32) {
         // 32 columns at a time, each plus its bias / scale (so the bias
         // registers free up as the scores arrive)
@@ -508,9 +566,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           }
         }
       } else {
-        // All four 32-column loads in flight, one wait.
+        // All 32-column loads in flight, one wait.
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, su[q]);
+        for (int q = 0; q < Tr::BN / 32; ++q) tmem_ld32(tS + 32 * q, su[q]);
         tmem_ld_wait();
       }
       float* s = reinterpret_cast<float*>(&su[0][0]);
@@ -524,17 +582,19 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         for (int c = 0; c < Tr::BN; ++c)
           if (c >= lim) s[c] = -INFINITY;
       }
-      // Row maximum: four independent chains of 3-input max.
-      float mq[4];
+      // Row maximum: independent chains of 3-input max, one per 32 columns.
+      float mq[Tr::BN / 32];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
+      for (int q = 0; q < Tr::BN / 32; ++q) {
         const float* v = s + 32 * q;
         float a = fmax3(v[0], v[1], v[2]);
 #pragma unroll
         for (int i = 3; i < 31; i += 2) a = fmax3(a, v[i], v[i + 1]);
         mq[q] = fmaxf(a, v[31]);
       }
-      const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      float mx = fmaxf(mq[0], mq[1]);
+#pragma unroll
+      for (int q = 2; q < Tr::BN / 32; q += 2) mx = fmax3(mx, mq[q], mq[q + 1]);
       const float m_tile = mx * sl2;
       const bool upd = m_tile > m_ref + kRescaleThreshold;
       float alpha = 1.f;
@@ -621,11 +681,15 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
       }
       tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&bars->p_full[t]);
+      mbar_arrive(&bars->p_full[sb]);
     }
 
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
+    // the tile's last product (with two score buffers the per-product
+    // barrier may be two phases behind here, so the last product has its own)
+    if (ok)
+      ok = __all_sync(0xffffffffu, Tr::SBUF == 2 ? MBAR_WAIT(&bars->o_full[1], 0, abort_flag)
+                                                 : MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
     tc_fence_after();
     if (ok) {
       // A row whose every score was masked (m_ref still -inf) has O = 0: the
@@ -733,12 +797,18 @@ int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool
   if (dtype == FA_FP32 || d != 128) return dflt;
   if (bias) return 2;  // the staged bias tiles need the two-tile layout
   if (drop) return dflt;
-  // K/V tiles a 128-row query tile sees, on average (bottom-right causal:
-  // query tile i sees about i + 1 + (Nk − Nq) / 128 of them)
+  // 128-key K/V tiles a 128-row query tile sees, on average (bottom-right
+  // causal: query tile i sees about i + 1 + (Nk − Nq) / 128 of them).  One Q
+  // tile over 64-key K/V tiles with double-buffered scores, against two Q
+  // tiles over one K/V stream (forward µs, d = 128 bf16, interleaved A/B,
+  // both orders): causal N = 1024 104.6 vs 120.8, N = 2048 160.8 vs 177.6,
+  // N = 4096 275–276 vs 281–282, N = 8192 506–510 vs 506–523, N = 16384 ×3
+  // even; non-causal N = 2048 289 vs 296, N = 4096 508–509 vs 491–492,
+  // N = 8192 972–1050 vs 937–1044.
   const double kv_tiles = (Nk + 127) / 128;
   const double q_tiles = (Nq + 127) / 128;
   const double avg = causal ? std::min(kv_tiles, (q_tiles + 1) / 2 + double(Nk - Nq) / 128) : kv_tiles;
-  return avg >= 12.0 ? 2 : 1;
+  return avg >= (causal ? 48.0 : 24.0) ? 2 : 3;
 }
 
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
@@ -756,6 +826,11 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \
+    if (DD == 128 && a.params.tiles == 3)                                                        \
+      return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 3>(a)                \
+                           : launch_fwd_t<TY, DD, true, false, false, false, 3>(a))              \
+                    : (gen ? launch_fwd_t<TY, DD, false, true, false, false, 3>(a)               \
+                           : launch_fwd_t<TY, DD, false, false, false, false, 3>(a));            \
     if (DD == 128 && a.params.tiles == 2)                                                        \
       return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 2>(a)                \
                            : launch_fwd_t<TY, DD, true, false, false, false, 2>(a))              \

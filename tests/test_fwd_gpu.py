@@ -56,23 +56,25 @@ def test_rectangular(fa, Nq, Nk, causal):
 
 
 @pytest.mark.parametrize("Nq,Nk,causal,dtype", [
-    (1600, 1600, False, "bf16"),   # 13 K/V tiles per query tile, 12.5 Q tiles: a half-empty last CTA
-    (3000, 3000, True, "bf16"),    # causal, 12.5 K/V tiles on average, ragged ends
-    (1000, 2000, True, "fp16"),    # bottom-right causal with Nk − Nq = 1000
-    (129, 1700, False, "bf16"),    # two Q tiles, the second with one row
+    (3100, 3100, False, "bf16"),   # 25 K/V tiles per query tile; the last CTA holds 28 rows
+    (300, 6500, True, "bf16"),     # bottom-right causal, ~50 K/V tiles on average, ragged ends
+    (1000, 7000, True, "fp16"),    # bottom-right causal with Nk − Nq = 6000
+    (129, 3200, False, "bf16"),    # two Q tiles, the second with one row
 ])
 def test_two_tile_d128_kernel(fa, Nq, Nk, causal, dtype):
-    """Shapes whose query tiles see 12 or more K/V tiles on average run the
-    16-bit d = 128 forward with two Q tiles per CTA."""
+    """Shapes whose query tiles see 24 or more 128-key K/V tiles on average
+    (48 or more with the causal mask) run the 16-bit d = 128 forward with two
+    Q tiles per CTA; the shorter ones (every other test here at d = 128) run
+    one Q tile over 64-key K/V tiles."""
     run_full(fa, 1, 2, Nq, Nk, 128, causal, dtype, seed=Nq + 3 * Nk)
 
 
 def test_two_tile_d128_kernel_strided_with_padding(fa):
     """The two-tile d = 128 forward on a [B, N, H, d] layout with key padding."""
-    B, H, N, d = 2, 2, 1700, 128
+    B, H, N, d = 2, 2, 3200, 128
     q, k, v, _ = W.make_tensors(B, H, N, N, d, "bf16", seed=8, device="cuda", with_grad=False)
     bshd = lambda t: t.transpose(1, 2).contiguous().transpose(1, 2)  # noqa: E731
-    kv_len = torch.tensor([1700, 900], dtype=torch.int32, device="cuda")
+    kv_len = torch.tensor([3200, 900], dtype=torch.int32, device="cuda")
     scale = 1 / math.sqrt(d)
     O, L = fa.forward(bshd(q), bshd(k), bshd(v), causal=False, scale=scale, kv_len=kv_len)
     assert fa.status() == fa.FA_OK
