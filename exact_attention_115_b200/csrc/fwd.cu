@@ -14,14 +14,15 @@
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
 // (fwd_tiles_for: two, except for 16-bit d = 128 when a query tile sees
 // fewer than 24 K/V tiles of 128 keys on average, or 48 under the causal
-// mask).  With two tiles it ping-pongs them over 128-key K/V tiles so the
-// tensor core works on one tile while the softmax warps work on the other.
-// With one tile (NT = 3) the K/V tiles have 64 keys and the score tile is
-// double-buffered in TMEM, so the scores of K/V tile j + 1 are computed
-// while the softmax of tile j runs; two such CTAs share an SM (the dropout
-// variants too: causal B8 H16 N2048 with p = 0.1, 257.3 -> 227.0 us against
-// one tile over 128-key K/V tiles with one score buffer, NT = 1, which
-// remains as a variant).  Roles per CTA (128 threads per tile + 128):
+// mask).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
+// so the tensor core works on one tile while the softmax warps work on the
+// other.  With one tile (NT = 3) the K/V tiles have 64 keys and the score
+// tile is double-buffered in TMEM, so the scores of K/V tile j + 1 are
+// computed while the softmax of tile j runs; two such CTAs share an SM.
+// Against one tile over 128-key K/V tiles with a single score buffer (the
+// design it replaced) causal B8 H16 N2048 d128 went 168.1 -> 159.1 us, and
+// with dropout p = 0.1 257.3 -> 227.0 us.  Roles per CTA (128 threads per
+// tile + 128):
 //   warpgroup t (warps 4t..4t+3)  softmax + correction + epilogue of Q tile t
 //                                 (thread = row), 200 registers
 //   last warpgroup: warp 4·TILES issues the tcgen05 MMAs (one thread) and
@@ -50,9 +51,10 @@ namespace {
 #endif
 constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entries stay <= 2^8
 
-// Q tiles per CTA of the dropout, bias and fp32 variants (the plain 16-bit
-// d = 128 kernels come with either count; see fwd_tiles_for).
-constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 1 : 2; }
+// Kernel shape of the dropout and fp32 variants: 3 (one Q tile over 64-key
+// K/V tiles) for 16-bit d = 128, else 2 (two Q tiles over 128-key K/V
+// tiles); the plain 16-bit d = 128 kernels come in both (fwd_tiles_for).
+constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 3 : 2; }
 
 // NT: 1 or 2 Q tiles of 128 rows per CTA over K/V tiles of 128 keys, or 3:
 // one Q tile over K/V tiles of 64 keys with its score tile double-buffered
@@ -102,6 +104,7 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
   static_assert(NS >= 2 * SBUF, "K/V slots for the products in flight");
+  static_assert(NT == 2 || NT == 3, "two Q tiles, or one over 64-key K/V tiles");
   static_assert(NT != 3 || (!BIAS && !ElemTraits<T>::tf32), "64-key tiles: 16-bit, no bias");
   static_assert(COL_O + TILES * D <= TMEM_COLS, "TMEM budget");
   static_assert(!BIAS || TILES == 2, "the staged bias needs the two-tile layout");
@@ -430,32 +433,6 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
             if (!ok) break;
             issue_qk(0, sk, b);
             commit(&bars->s_full[b]);
-            commit(&bars->kv_empty[sk]);
-          }
-        }
-      } else if constexpr (Tr::TILES == 1) {
-        // One tile: S(j), then (once the softmax has written P(j)) P(j)·V(j)
-        // and S(j+1) into the same columns, in issue order after P·V read P.
-        bool ok = MBAR_WAIT_WARP(&bars->q_full[0], 0, abort_flag) && kv_wait(0);
-        tc_fence_after();
-        if (ok) issue_qk(0, 0, 0);
-        commit(&bars->s_full[0]);
-        commit(&bars->kv_empty[0]);  // K_0's slot, once S(0) has read it
-        for (int j = 0; j < n_kv && ok; ++j) {
-          const int iv = 2 * j + 1, ik = 2 * j + 2;
-          const int sv = iv % Tr::NS, sk = ik % Tr::NS;
-          ok = kv_wait(iv) && MBAR_WAIT_WARP(&bars->p_full[0], j & 1, abort_flag);
-          tc_fence_after();
-          if (!ok) break;
-          issue_pv(0, sv, j > 0, 0);
-          commit(&bars->o_full[0]);
-          commit(&bars->kv_empty[sv]);
-          if (j + 1 < n_kv) {
-            ok = kv_wait(ik);
-            tc_fence_after();
-            if (!ok) break;
-            issue_qk(0, sk, 0);
-            commit(&bars->s_full[0]);
             commit(&bars->kv_empty[sk]);
           }
         }
@@ -824,17 +801,9 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
                             : launch_fwd_t<TY, DD, true, true, false, true, 2>(a))              \
                     : (drop ? launch_fwd_t<TY, DD, false, true, true, true, 2>(a)               \
                             : launch_fwd_t<TY, DD, false, true, false, true, 2>(a));            \
-    if (drop && DD == 128)                                                                       \
-      return causal ? launch_fwd_t<TY, DD, true, true, true, false, 3>(a)                        \
-                    : launch_fwd_t<TY, DD, false, true, true, false, 3>(a);                      \
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \
-    if (DD == 128 && a.params.tiles == 3)                                                        \
-      return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 3>(a)                \
-                           : launch_fwd_t<TY, DD, true, false, false, false, 3>(a))              \
-                    : (gen ? launch_fwd_t<TY, DD, false, true, false, false, 3>(a)               \
-                           : launch_fwd_t<TY, DD, false, false, false, false, 3>(a));            \
     if (DD == 128 && a.params.tiles == 2)                                                        \
       return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 2>(a)                \
                            : launch_fwd_t<TY, DD, true, false, false, false, 2>(a))              \
