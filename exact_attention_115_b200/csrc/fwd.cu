@@ -12,9 +12,9 @@
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
-// (fwd_tiles_for: two, except for 16-bit d = 128 when a query tile sees
-// fewer than 24 K/V tiles of 128 keys on average, or 48 under the causal
-// mask).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
+// (fwd_tiles_for: one for 16-bit types, except two for the bias and for
+// d = 128 when a query tile sees 24 or more K/V tiles of 128 keys on
+// average, 48 under the causal mask; two for fp32).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
 // so the tensor core works on one tile while the softmax warps work on the
 // other.  With one tile (NT = 3) the K/V tiles have 64 keys and the score
 // tile is double-buffered in TMEM, so the scores of K/V tile j + 1 are
@@ -52,9 +52,10 @@ namespace {
 constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entries stay <= 2^8
 
 // Kernel shape of the dropout and fp32 variants: 3 (one Q tile over 64-key
-// K/V tiles) for 16-bit d = 128, else 2 (two Q tiles over 128-key K/V
-// tiles); the plain 16-bit d = 128 kernels come in both (fwd_tiles_for).
-constexpr int fwd_tiles(bool tf32, int d) { return (!tf32 && d == 128) ? 3 : 2; }
+// K/V tiles) for 16-bit types, 2 (two Q tiles over 128-key K/V tiles) for
+// fp32; the plain 16-bit d = 128 kernels come in both (fwd_tiles_for), the
+// bias variants in shape 2.
+constexpr int fwd_tiles(bool tf32, int d) { return (void)d, tf32 ? 2 : 3; }
 
 // NT: 1 or 2 Q tiles of 128 rows per CTA over K/V tiles of 128 keys, or 3:
 // one Q tile over K/V tiles of 64 keys with its score tile double-buffered
@@ -78,7 +79,7 @@ struct FwdTraits {
   // other's main loop, at the price of loading each K/V tile twice per SM.
   // With two tiles the CTA ping-pongs its own tiles over one K/V stream.
   // Which count is faster depends on how many K/V tiles a query tile sees
-  // (measurements at fwd_tiles_for).  d = 64: two tiles (+5 %).
+  // (measurements at fwd_tiles_for).
   static constexpr int TILES = NT == 2 ? 2 : 1;
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
   // The bias variants (two tiles) stage each K/V step's [128 rows × 128 keys]
@@ -772,9 +773,14 @@ int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
 
 int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias) {
   const int dflt = fwd_tiles(dtype == FA_FP32, d);
-  if (dtype == FA_FP32 || d != 128) return dflt;
+  if (dtype == FA_FP32) return dflt;
   if (bias) return 2;  // the staged bias tiles need the two-tile layout
-  if (drop) return 3;
+  // d = 64: one tile over 64-key K/V tiles at every length measured (µs,
+  // interleaved A/B, both orders, against two tiles): B4 H16 N1024 41.3–42.2
+  // vs 43.0–43.1, causal N = 1024 90.3 vs 108.6, N = 2048 142 vs 163,
+  // N = 4096 244 vs 270, N = 8192 448–453 vs 485–489, B1 H32 N16384 1671 vs
+  // 1813; non-causal N = 4096 450 vs 466, N = 8192 857 vs 888.
+  if (d != 128 || drop) return 3;
   // 128-key K/V tiles a 128-row query tile sees, on average (bottom-right
   // causal: query tile i sees about i + 1 + (Nk − Nq) / 128 of them).  One Q
   // tile over 64-key K/V tiles with double-buffered scores, against two Q
@@ -804,7 +810,7 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \
-    if (DD == 128 && a.params.tiles == 2)                                                        \
+    if (a.params.tiles == 2)                                                                     \
       return causal ? (gen ? launch_fwd_t<TY, DD, true, true, false, false, 2>(a)                \
                            : launch_fwd_t<TY, DD, true, false, false, false, 2>(a))              \
                     : (gen ? launch_fwd_t<TY, DD, false, true, false, false, 2>(a)               \
