@@ -54,7 +54,7 @@
 // MMA order is dV, next Sᵀ, dQ, dK, next dPᵀ: dQ lands in the dPᵀ columns
 // (read by then), warpgroup 2 drains it while dK runs, and the next dPᵀ
 // waits until warpgroup 2 has the dQ values in registers.  Q (with −L·log2e
-// and −D) is double buffered, dO single buffered.
+// and −D) has two stages at d = 128 and three at d = 64, dO one.
 #define FA_SITE_BASE 20000
 #include <algorithm>
 
@@ -112,23 +112,26 @@ struct BwdTraits {
   // d = 128 reduces dQᵀ from registers and needs no staging.
   static constexpr int DQ_STAGE = DQ_STAGED ? BM * D * 4 : 0;
   // shared-memory offsets (all 1024-aligned).  K is double buffered (the
-  // next work item's K loads while this item runs); Q is double buffered
-  // (the next step's Sᵀ needs it while this step's dK still reads the
-  // current one); V and dO are single buffered.
+  // next work item's K loads while this item runs); Q has QS stages (the
+  // next step's Sᵀ needs one while this step's dK still reads the current
+  // one); V and dO are single buffered.
   // The bias variants stage each step's [BM queries × BN keys] bias tile in
   // shared memory (one TMA load).  At d = 128 its 32 KB take the second K
   // buffer (K is then single buffered); at d = 64 there is room after the rest.
   static constexpr int BIAS_TILE = BIAS ? BM * BN * ES : 0;
   static constexpr bool K_SINGLE = BIAS && D == 128;
   static constexpr int KBUF = K_SINGLE ? 1 : 2;      // K buffers
+  // Q stages: three at d = 64 (room to spare), so a stage is reloaded two
+  // steps after its dK product released it; two at d = 128.
+  static constexpr int QS = D == 64 ? 3 : 2;
   static constexpr int OFF_K = 0;                    // 2 buffers
   static constexpr int OFF_V = OFF_K + 2 * KV_TILE;
-  static constexpr int OFF_Q = OFF_V + KV_TILE;      // 2 stages
-  static constexpr int OFF_DO = OFF_Q + 2 * Q_TILE;
+  static constexpr int OFF_Q = OFF_V + KV_TILE;      // QS stages
+  static constexpr int OFF_DO = OFF_Q + QS * Q_TILE;
   static constexpr int OFF_DS = OFF_DO + Q_TILE;
   static constexpr int OFF_DQ = OFF_DS + DS_TILE;
   static constexpr int OFF_LD = OFF_DQ + DQ_STAGE;   // L·log2e and D per Q stage
-  static constexpr int OFF_BAR = OFF_LD + 2 * 2 * BM * 4;
+  static constexpr int OFF_BAR = OFF_LD + QS * 2 * BM * 4;
   static constexpr int OFF_BIAS = K_SINGLE ? OFF_K + KV_TILE : (OFF_BAR + 512 + 1023) / 1024 * 1024;
   // the base is checked to be 1024-aligned
   static constexpr int SMEM_BYTES = (BIAS && !K_SINGLE) ? OFF_BIAS + BIAS_TILE : OFF_BAR + 512;
@@ -163,7 +166,7 @@ struct BwdTraits {
 
 // The kernel is persistent: a CTA takes work items (K/V block, head) in turn
 // and numbers its steps across items (g).  The per-step barriers complete
-// once per step except q_full / q_empty (one per Q stage, every other
+// once per step except q_full / q_empty (one per Q stage, every QS-th
 // step); v_full, v_free, dkv_done and dkv_free complete once per work item,
 // k_full[b] / k_free[b] once per item that uses K buffer b (every other
 // item), item_full[s] once per item published in ring slot s.  A producer
@@ -175,8 +178,8 @@ struct BwdBarriers {
   uint64_t k_free[2];
   uint64_t v_full;
   uint64_t v_free;
-  uint64_t q_full[2];
-  uint64_t q_empty[2];
+  uint64_t q_full[3];     // Q stage s (of QS) holds its step's Q, −L·log2e and −D
+  uint64_t q_empty[3];
   uint64_t do_full;
   uint64_t do_empty;
   uint64_t s_full;
@@ -266,6 +269,8 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(&bars->k_full[b], 1);
       mbar_init(&bars->k_free[b], 1);
+    }
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&bars->q_full[b], 1);
       mbar_init(&bars->q_empty[b], 1);
     }
@@ -379,7 +384,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
         int bh, kb, i0, n_q;
         item(j, bh, kb, i0, n_q);
         for (int i = 0; i < n_q && ok; ++i) {
-          const int gs = g + i, s = gs & 1;
+          const int gs = g + i, s = gs % Tr::QS;
           const int q0 = (i0 + i) * BM;
           if constexpr (BIAS) {
             // the step's [BM queries × BN keys] bias tile (zero past Nq and
@@ -397,7 +402,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
                         (bh % p.H) % p.bias_H, (bh / p.H) % p.bias_B);
           }
           // Q (with −L·log2e and −D) into stage s, once step gs-2 has released it
-          if (gs >= 2 && !MBAR_WAIT(&bars->q_empty[s], ((gs >> 1) - 1) & 1, abort_flag)) {
+          if (gs >= Tr::QS && !MBAR_WAIT(&bars->q_empty[s], ((gs / Tr::QS) - 1) & 1, abort_flag)) {
             ok = false;
             break;
           }
@@ -428,8 +433,8 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
         g += n_q;
       }
       // Drain every issued load before the CTA may exit.
-      for (int gs = max(0, g - 2); gs < g; ++gs)
-        MBAR_WAIT(&bars->q_full[gs & 1], (gs >> 1) & 1, abort_flag);
+      for (int gs = max(0, g - Tr::QS); gs < g; ++gs)
+        MBAR_WAIT(&bars->q_full[gs % Tr::QS], (gs / Tr::QS) & 1, abort_flag);
       if (g > 0) MBAR_WAIT(&bars->do_full, (g - 1) & 1, abort_flag);
       if (BIAS && g > 0) MBAR_WAIT(&bars->bias_full, (g - 1) & 1, abort_flag);
     }
@@ -519,12 +524,12 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
         const uint64_t dK_k = kbuf(dK_k0, b), dK_mn = kbuf(dK_mn0, b);
         ok = MBAR_WAIT_WARP(&bars->k_full[b], (it / Tr::KBUF) & 1, abort_flag);
         if (ok && n_q > 0)
-          ok = MBAR_WAIT_WARP(&bars->q_full[g & 1], (g >> 1) & 1, abort_flag) &&
+          ok = MBAR_WAIT_WARP(&bars->q_full[g % Tr::QS], (g / Tr::QS) & 1, abort_flag) &&
                MBAR_WAIT_WARP(&bars->do_full, g & 1, abort_flag);
         tc_fence_after();
         if (!ok) break;
         if (n_q > 0) {
-          mma_st(colS, dK_k, stg(dQ_k0, g & 1));
+          mma_st(colS, dK_k, stg(dQ_k0, g % Tr::QS));
           commit(&bars->s_full);
           // dPᵀ(0) needs V, and the previous item's last dQ out of the dPᵀ columns
           ok = MBAR_WAIT_WARP(&bars->v_full, it & 1, abort_flag);
@@ -552,7 +557,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
         // the compute warpgroups by then), dK, and last the next dPᵀ, once
         // warpgroup 2 has drained dQ from those columns.
         for (int i = 0; i < n_q; ++i) {
-          const int gs = g + i, s = gs & 1;
+          const int gs = g + i, s = gs % Tr::QS, sn = (gs + 1) % Tr::QS;
           const bool more = i + 1 < n_q;
           ok = MBAR_WAIT_WARP(&bars->p_ready, gs & 1, abort_flag);
           tc_fence_after();
@@ -560,10 +565,10 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
           mma_dv(i > 0);
           commit(&bars->do_empty);
           if (more) {
-            ok = MBAR_WAIT_WARP(&bars->q_full[s ^ 1], ((gs + 1) >> 1) & 1, abort_flag);
+            ok = MBAR_WAIT_WARP(&bars->q_full[sn], ((gs + 1) / Tr::QS) & 1, abort_flag);
             tc_fence_after();
             if (!ok) break;
-            mma_st(colS, dK_k, stg(dQ_k0, s ^ 1));
+            mma_st(colS, dK_k, stg(dQ_k0, sn));
             commit(&bars->s_full);
           }
           ok = MBAR_WAIT_WARP(&bars->ds_ready, gs & 1, abort_flag);
@@ -614,7 +619,7 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
       const bool key_live = key < keys_of(p.kv_len, bh, p.H, p.Nk);
       const int qmin = key - off;  // first query row that sees this key
       for (int i = 0; i < n_q; ++i) {
-        const int gs = g + i, s = gs & 1;
+        const int gs = g + i, s = gs % Tr::QS;
         const int q0 = (i0 + i) * BM + cw * CWC;  // first query column of this warpgroup
         // −L·log2e and −D of this warpgroup's query columns (16-byte aligned)
         const float4* sL4 = reinterpret_cast<const float4*>(sLD + (s * 2 + 0) * BM + cw * CWC);
