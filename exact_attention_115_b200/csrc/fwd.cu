@@ -769,8 +769,6 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   return cudaGetLastError();
 }
 
-int fwd_tile_elems(int dtype) { return dtype == FA_FP32 ? 32 : 64; }
-
 int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias) {
   const int dflt = fwd_tiles(dtype == FA_FP32, d);
   if (dtype == FA_FP32) return dflt;

@@ -42,7 +42,7 @@ struct FwdParams {
   float* L;
   int B, H, Nq, Nk;
   float scale_log2;  // scale * log2(e)
-  int tiles;         // 1 or 2 128-row Q tiles per CTA, or 3: one over 64-key K/V tiles (fwd_tiles_for)
+  int tiles;         // kernel shape (fwd_tiles_for): 2 = two 128-row Q tiles per CTA, 3 = one over 64-key K/V tiles
   int n_qblocks;     // ceil(Nq / query rows per CTA): one CTA per block of query rows
   int head_group;    // heads per launch-order group (see head_group_for)
   int map4d;         // bit per tensor map (Q 0, K 1, V 2, O 3): 4-D (d, N, H, B), else 3-D (d, N, B·H)
@@ -63,10 +63,8 @@ struct FwdLaunch {
   cudaStream_t stream;
 };
 
-// Elements in one 128-byte swizzled row for the dtype (the TMA box width).
-int fwd_tile_elems(int dtype);
-// Forward kernel for a call: 1 or 2 128-row Q tiles per CTA over 128-key K/V
-// tiles, or 3: one Q tile over 64-key K/V tiles with double-buffered scores.
+// Forward kernel for a call: 2 (two 128-row Q tiles per CTA over 128-key K/V
+// tiles) or 3 (one Q tile over 64-key K/V tiles with double-buffered scores).
 int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias);
 cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a);
 
