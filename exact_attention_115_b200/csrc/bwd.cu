@@ -652,6 +652,9 @@ __global__ void __launch_bounds__(BwdTraits<T, D, BIAS>::THREADS, 1)
 #pragma unroll
             for (int c = 0; c < CWC; c += 2) bpk[c >> 1] = v | (v << 16);
           }
+          // (the next tile is written by TMA, another proxy: a proxy fence
+          // orders these reads before that write, as in the forward)
+          fence_async_smem();
           mbar_arrive(&bars->bias_empty);
         }
         // ---- P = exp2(S·c − L·log2e), causal / ragged masking

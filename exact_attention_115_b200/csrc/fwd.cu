@@ -12,9 +12,9 @@
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
-// (fwd_tiles_for: one for 16-bit types, except two for the bias and for
-// d = 128 when a query tile sees 24 or more K/V tiles of 128 keys on
-// average, 48 under the causal mask; two for fp32).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
+// (fwd_tiles_for: one for 16-bit types, except two for d = 128 when a
+// query tile sees 24 or more K/V tiles of 128 keys on average, 48 under the
+// causal mask; two for fp32).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
 // so the tensor core works on one tile while the softmax warps work on the
 // other.  With one tile (NT = 3) the K/V tiles have 64 keys and the score
 // tile is double-buffered in TMEM, so the scores of K/V tile j + 1 are
@@ -53,8 +53,8 @@ constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entr
 
 // Kernel shape of the dropout and fp32 variants: 3 (one Q tile over 64-key
 // K/V tiles) for 16-bit types, 2 (two Q tiles over 128-key K/V tiles) for
-// fp32; the plain 16-bit d = 128 kernels come in both (fwd_tiles_for), the
-// bias variants in shape 2.
+// fp32; the plain and bias 16-bit d = 128 kernels come in both
+// (fwd_tiles_for).
 constexpr int fwd_tiles(bool tf32, int d) { return (void)d, tf32 ? 2 : 3; }
 
 // NT: 1 or 2 Q tiles of 128 rows per CTA over K/V tiles of 128 keys, or 3:
@@ -82,9 +82,10 @@ struct FwdTraits {
   // (measurements at fwd_tiles_for).
   static constexpr int TILES = NT == 2 ? 2 : 1;
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
-  // The bias variants (two tiles) stage each K/V step's [128 rows × 128 keys]
-  // bias tile of every Q tile in shared memory: two 128-byte-swizzled halves
-  // of 64 keys, so that a thread's row reads are free of bank conflicts.
+  // The bias variants stage each K/V step's [128 rows × BN keys] bias tile
+  // of every Q tile in shared memory: 128-byte-swizzled blocks of 64 keys,
+  // so that a thread's row reads are free of bank conflicts.  With one tile
+  // the 16 KB bias tile leaves room for three K/V slots at d = 128.
   static constexpr int BIAS_TILE = BIAS ? 128 * BN * ES : 0;
   static constexpr int SMEM_BUDGET =
       TILES == 1 ? 110 * 1024 : (BIAS ? 220 : 200) * 1024;  // tiles, per CTA
@@ -104,11 +105,12 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
-  static_assert(NS >= 2 * SBUF, "K/V slots for the products in flight");
+  // K/V slots: two per score buffer, or (bias, one tile) three, so that K of
+  // tile j + 2 loads once P(j)·V(j) has read V(j)
+  static_assert(NS >= (BIAS && SBUF == 2 ? 3 : 2 * SBUF), "K/V slots for the products in flight");
   static_assert(NT == 2 || NT == 3, "two Q tiles, or one over 64-key K/V tiles");
-  static_assert(NT != 3 || (!BIAS && !ElemTraits<T>::tf32), "64-key tiles: 16-bit, no bias");
+  static_assert(NT != 3 || !ElemTraits<T>::tf32, "64-key tiles: 16-bit types");
   static_assert(COL_O + TILES * D <= TMEM_COLS, "TMEM budget");
-  static_assert(!BIAS || TILES == 2, "the staged bias needs the two-tile layout");
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
 
@@ -207,7 +209,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
                const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                const __grid_constant__ CUtensorMap tmBias, FwdParams p) {
   using Tr = FwdTraits<T, D, NT, BIAS && !ElemTraits<T>::tf32>;
-  // staged bias tiles (16-bit types): the two-tile layout
+  // staged bias tiles (16-bit types)
   constexpr bool SBIAS = BIAS && !ElemTraits<T>::tf32;
   constexpr bool TF32 = ElemTraits<T>::tf32;
   extern __shared__ uint8_t smem_raw[];
@@ -271,7 +273,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
 
   uint8_t* sQ[2] = {smem, smem + Tr::TILE};  // (the second only with two tiles)
   uint8_t* sKV = smem + Tr::TILES * Tr::TILE;
-  uint8_t* sBias = smem + Tr::OFF_BIAS;  // SBIAS: [TILES][2 halves][rows][128 B], swizzled
+  uint8_t* sBias = smem + Tr::OFF_BIAS;  // SBIAS: [TILES][BN / 64 blocks][rows][128 B], swizzled
 
   if (warp > Tr::PRODUCER_WARP) {
     // idle warps of the producer/MMA warpgroup
@@ -314,9 +316,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
       load_tile((i & 1) ? 2 : 1, sKV + slot * Tr::KV_TILE, &bars->kv_full[slot], (i >> 1) * Tr::BN);
       return true;
     };
-    // SBIAS: K/V tile j's bias tile of each Q tile (two swizzled halves of
-    // 64 keys; one row each when the bias is shared by all query rows, its
-    // halves a swizzle atom apart), once that tile's softmax warps have
+    // SBIAS: K/V tile j's bias tile of each Q tile (BN / 64 swizzled blocks
+    // of 64 keys; one row each when the bias is shared by all query rows, the
+    // blocks a swizzle atom apart), once that tile's softmax warps have
     // copied out tile j − 1's.  Zero past Nq and Nk.
     auto load_bias = [&](int j) {
       for (int t = 0; t < Tr::TILES; ++t) {
@@ -325,9 +327,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         if (!ok) return false;
         if (lane == 0 && FA_INBOUNDS(bh < p.B * p.H && j * Tr::BN < p.Nk)) {
           const int rows = p.bias_rows, half = rows > 1 ? rows * 128 : 1024;
-          mbar_arrive_expect_tx(&bars->bias_full[t], 2 * rows * 128);
+          mbar_arrive_expect_tx(&bars->bias_full[t], (Tr::BN / 64) * rows * 128);
 #pragma unroll
-          for (int h = 0; h < 2; ++h)
+          for (int h = 0; h < Tr::BN / 64; ++h)
             tma_load_4d(sBias + t * Tr::BIAS_TILE + h * half, &tmBias, &bars->bias_full[t], j * Tr::BN + 64 * h,
                         rows > 1 ? q_row0 + 128 * t : 0, (bh % p.H) % p.bias_H, (bh / p.H) % p.bias_B);
         }
@@ -496,11 +498,11 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
     float row_sum_p = 0.f;  // Σ of P as rounded for the P·V product: normalises O
     bool ok = true;
 
-    // staged bias tile of this Q tile: chunk c (8 keys) of row rr at
-    // half c / 8, position (c % 8) ^ (rr % 8) of the row's 128 bytes
+    // staged bias tile of this Q tile: chunk c (8 keys) of row rr in the
+    // 64-key block c / 8, position (c % 8) ^ (rr % 8) of the row's 128 bytes
     const uint8_t* btile = sBias + t * Tr::BIAS_TILE;
     for (int j = 0; j < n_kv; ++j) {
-      // Bias: this row's 128 values for the tile's columns, copied out of the
+      // Bias: this row's BN values for the tile's columns, copied out of the
       // staged tile before S arrives (zero past Nk or past Nq), which is then
       // released for the next K/V tile's.
       uint4 bv[SBIAS ? Tr::BN / 8 : 1];
@@ -517,6 +519,11 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           for (int v = 0; v < Tr::BN / 8; ++v)
             bv[v] = *reinterpret_cast<const uint4*>(btile + (v >> 3) * 1024 + ((v & 7) << 4));
         }
+        // The values are still in flight when the tile is released, and the
+        // next tile is written by TMA (the async proxy): without a proxy
+        // fence that write overtook these reads now and then (seen as rows of
+        // L and O that changed from run to run).
+        fence_async_smem();
         mbar_arrive(&bars->bias_empty[t]);
       }
       // score buffer of K/V tile j: the tile's own, or j % 2 of two
@@ -531,7 +538,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         // 32 columns at a time, each plus its bias / scale (so the bias
         // registers free up as the scores arrive)
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
+        for (int q = 0; q < Tr::BN / 32; ++q) {
           tmem_ld32(tS + 32 * q, su[q]);
           tmem_ld_wait();
 #pragma unroll
@@ -772,7 +779,6 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
 int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool bias) {
   const int dflt = fwd_tiles(dtype == FA_FP32, d);
   if (dtype == FA_FP32) return dflt;
-  if (bias) return 2;  // the staged bias tiles need the two-tile layout
   // d = 64: one tile over 64-key K/V tiles at every length measured (µs,
   // interleaved A/B, both orders, against two tiles): B4 H16 N1024 41.3–42.2
   // vs 43.0–43.1, causal N = 1024 90.3 vs 108.6, N = 2048 142 vs 163,
@@ -786,7 +792,12 @@ int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool
   // both orders): causal N = 1024 104.6 vs 120.8, N = 2048 160.8 vs 177.6,
   // N = 4096 275–276 vs 281–282, N = 8192 506–510 vs 506–523, N = 16384 ×3
   // even; non-causal N = 2048 289 vs 296, N = 4096 508–509 vs 491–492,
-  // N = 8192 972–1050 vs 937–1044.
+  // N = 8192 972–1050 vs 937–1044.  With a bias the same rule holds (one
+  // tile with a 3-slot ring, against two tiles with staged 128-key bias
+  // tiles, µs): causal N = 2048 head-shared [1, H, N, N] 240–253 vs
+  // 259–274, full 256–267 vs 277–289, query-broadcast 225–227 vs 248–249,
+  // causal N = 8192 495–513 vs 534–548; non-causal N = 4096 451–470 vs
+  // 462–480 (before the proxy fence on the bias tile, which costs ~3 %).
   const double kv_tiles = (Nk + 127) / 128;
   const double q_tiles = (Nq + 127) / 128;
   const double avg = causal ? std::min(kv_tiles, (q_tiles + 1) / 2 + double(Nk - Nq) / 128) : kv_tiles;
@@ -800,11 +811,16 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
   // dropout and bias run in general-layout variants only
 #define FA_FWD_CASE(TY, DD)                                                                      \
   {                                                                                              \
-    if (bias)                                                                                    \
+    if (bias && a.params.tiles == 2)                                                             \
       return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true, 2>(a)                \
                             : launch_fwd_t<TY, DD, true, true, false, true, 2>(a))              \
                     : (drop ? launch_fwd_t<TY, DD, false, true, true, true, 2>(a)               \
                             : launch_fwd_t<TY, DD, false, true, false, true, 2>(a));            \
+    if (bias)                                                                                    \
+      return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true, 3>(a)                \
+                            : launch_fwd_t<TY, DD, true, true, false, true, 3>(a))              \
+                    : (drop ? launch_fwd_t<TY, DD, false, true, true, true, 3>(a)               \
+                            : launch_fwd_t<TY, DD, false, true, false, true, 3>(a));            \
     if (drop)                                                                                    \
       return causal ? launch_fwd_t<TY, DD, true, true, true>(a)                                  \
                     : launch_fwd_t<TY, DD, false, true, true>(a);                                \

@@ -83,6 +83,18 @@ def test_bias_rectangular_causal(fa):
     _run(fa, q, k, v, do, bias, True, "bias Nq130 Nk300 causal")
 
 
+@pytest.mark.parametrize("bshape", ["full", "query_bcast"])
+def test_bias_long_rows(fa, bshape):
+    """Rows of 3100 keys at d = 128 (25 K/V tiles of 128 keys per query
+    tile) take the two-tile forward with its 128-key bias tiles; the shorter
+    rows above take the one-tile form with 64-key ones."""
+    B, H, Nq, Nk = 1, 2, 200, 3100
+    q, k, v, do = W.make_tensors(B, H, Nq, Nk, 128, "bf16", seed=94, device="cuda")
+    shape = (B, H, Nq) if bshape == "full" else (B, H, 1)
+    bias = _bias(shape + (Nk,), Nk, torch.bfloat16, seed=12, ninf=0.05)
+    _run(fa, q, k, v, do, bias, False, f"bias {bshape} Nq{Nq} Nk{Nk}")
+
+
 def test_bias_with_dropout_padding_fp16_strided(fa):
     B, H, N, d = 2, 2, 256, 64
     q, k, v, do = W.make_tensors(B, H, N, N, d, "fp16", seed=91, device="cuda")
@@ -135,3 +147,28 @@ def test_bias_autograd(fa):
     assert fa.status() == fa.FA_OK
     assert torch.equal(O.detach(), O0)
     assert torch.equal(ka.grad, dk0) and torch.equal(va.grad, dv0)
+
+
+def test_bias_repeatable(fa):
+    """The same call gives the same bits every time: O and L of the forward,
+    dK and dV of the backward (dQ is summed by atomics, in no fixed order).
+    The staged bias tile is refilled by TMA right after the softmax threads
+    read it; a missing proxy fence there showed as rows of L and O that
+    changed from run to run, most often on long rows (here 46 steps of 64
+    keys per query tile, one-tile kernel)."""
+    B, H, N, d = 4, 16, 2944, 128
+    q, k, v, do = W.make_tensors(B, H, N, N, d, "bf16", seed=95, device="cuda")
+    g = torch.Generator(device="cuda").manual_seed(13)
+    bias = torch.randn(1, H, N, N, generator=g, device="cuda").to(torch.bfloat16)
+    outs = [fa.forward(q, k, v, bias=bias) for _ in range(20)]
+    torch.cuda.synchronize()
+    assert fa.status() == fa.FA_OK
+    O0, L0 = outs[0]
+    differ = [i for i, (O, L) in enumerate(outs) if not (torch.equal(O, O0) and torch.equal(L, L0))]
+    assert not differ, f"forward runs {differ} differ from the first"
+    del outs
+    grads = [fa.backward(q, k, v, O0, do, L0, bias=bias)[1:] for _ in range(4)]
+    torch.cuda.synchronize()
+    assert fa.status() == fa.FA_OK
+    for i, (dk, dv) in enumerate(grads[1:], 1):
+        assert torch.equal(dk, grads[0][0]) and torch.equal(dv, grads[0][1]), f"backward run {i} differs"
