@@ -323,23 +323,28 @@ DECODE_PROFILE = W.Workload("decode_b4h32nk32768d128", 4, 32, 1, 32768, 128, Fal
 
 def profile_case(name: str):
     """Three launches of one kernel's case: the causal B8 H16 N2048 d128
-    forward or backward, or the reduced decode shape.  A capture skips the
-    first two launches of the kernel (``-s 2 -c 1``)."""
+    forward (``fwd_bias``: with the bench's head-shared [1, 16, 2048, 2048]
+    additive bias) or backward, or the reduced decode shape.  A capture
+    skips the first two launches of the kernel (``-s 2 -c 1``)."""
     import exact_attention_115_b200 as fa
 
     dev = torch.device("cuda", 0)
     w = DECODE_PROFILE if name == "decode" else W.CAUSAL_2K
     q, k, v, do = W.make_inputs(w, device=dev, with_grad=name == "bwd")
+    bias = None
+    if name == "fwd_bias":
+        g = torch.Generator(device=dev).manual_seed(w.seed + 1)
+        bias = torch.randn(1, w.H, w.Nq, w.Nk, generator=g, device=dev).to(q.dtype)
     if name == "decode":
         for _ in range(3):
             fa.decode(q, k, v)
     else:
-        O, L = fa.forward(q, k, v, causal=w.causal)
+        O, L = fa.forward(q, k, v, causal=w.causal, bias=bias)
         for _ in range(3 if name == "bwd" else 2):
             if name == "bwd":
                 fa.backward(q, k, v, O, do, L, causal=w.causal)
             else:
-                fa.forward(q, k, v, causal=w.causal, out=O, lse=L)
+                fa.forward(q, k, v, causal=w.causal, out=O, lse=L, bias=bias)
     torch.cuda.synchronize(dev)
     st = fa.status()
     print(f"profile case {name}: {w.describe()} status {fa.STATUS_NAMES.get(st, st)}")
@@ -359,7 +364,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the other workloads (B4 H16 N1024 d64, the 16K causal one, fp16, with a bias)")
-    ap.add_argument("--profile-case", choices=["fwd", "bwd", "decode"],
+    ap.add_argument("--profile-case", choices=["fwd", "fwd_bias", "bwd", "decode"],
                     help="run one kernel's small profiling case three times and exit "
                          "(the command an ncu capture wraps; nothing is timed)")
     args = ap.parse_args()

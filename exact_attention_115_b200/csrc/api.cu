@@ -214,7 +214,7 @@ int decode_keys_per_split(int Nk, int splits) {
 
 }  // namespace
 
-cudaError_t set_smem_once(const void* kernel, int bytes) {
+cudaError_t set_smem_once(const void* kernel, int bytes, bool max_carveout) {
   static std::mutex mu;
   static int done_n[kMaxDevices] = {0};
   constexpr int kTracked = 128;  // more than the kernel variants of the library
@@ -228,6 +228,9 @@ cudaError_t set_smem_once(const void* kernel, int bytes) {
     for (int i = 0; i < done_n[dev]; ++i)
       if (done_k[dev][i] == kernel) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && max_carveout)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess && track && done_n[dev] < kTracked) done_k[dev][done_n[dev]++] = kernel;
   return e;
 }

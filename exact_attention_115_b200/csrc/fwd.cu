@@ -12,9 +12,9 @@
 // exp2 with scale·log2(e) folded into one FFMA per score.
 //
 // B200 design (not the pages'): a CTA owns one or two 128-row Q tiles
-// (fwd_tiles_for: one for 16-bit types, except two for d = 128 when a
-// query tile sees 24 or more K/V tiles of 128 keys on average, 48 under the
-// causal mask; two for fp32).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
+// (fwd_tiles_for: one for 16-bit types, except two for d = 128 without a
+// bias or dropout when a query tile sees 24 or more K/V tiles of 128 keys
+// on average, 48 under the causal mask; two for fp32).  With two tiles (NT = 2) it ping-pongs them over 128-key K/V tiles
 // so the tensor core works on one tile while the softmax warps work on the
 // other.  With one tile (NT = 3) the K/V tiles have 64 keys and the score
 // tile is double-buffered in TMEM, so the scores of K/V tile j + 1 are
@@ -53,8 +53,8 @@ constexpr float kRescaleThreshold = FA_RESCALE_THRESHOLD;  // log2 units: P entr
 
 // Kernel shape of the dropout and fp32 variants: 3 (one Q tile over 64-key
 // K/V tiles) for 16-bit types, 2 (two Q tiles over 128-key K/V tiles) for
-// fp32; the plain and bias 16-bit d = 128 kernels come in both
-// (fwd_tiles_for).
+// fp32; the plain 16-bit d = 128 kernels come in both (fwd_tiles_for), the
+// bias variants in shape 3.
 constexpr int fwd_tiles(bool tf32, int d) { return (void)d, tf32 ? 2 : 3; }
 
 // NT: 1 or 2 Q tiles of 128 rows per CTA over K/V tiles of 128 keys, or 3:
@@ -84,16 +84,26 @@ struct FwdTraits {
   static constexpr int CTAS_PER_SM = TILES == 1 ? 2 : 1;
   // The bias variants stage each K/V step's [128 rows × BN keys] bias tile
   // of every Q tile in shared memory: 128-byte-swizzled blocks of 64 keys,
-  // so that a thread's row reads are free of bank conflicts.  With one tile
-  // the 16 KB bias tile leaves room for three K/V slots at d = 128.
+  // so that a thread's row reads are free of bank conflicts.  They are built
+  // in the one-tile form only: with the four K/V slots below it measured
+  // faster than two tiles with 128-key bias tiles at every length.
   static constexpr int BIAS_TILE = BIAS ? 128 * BN * ES : 0;
-  static constexpr int SMEM_BUDGET =
-      TILES == 1 ? 110 * 1024 : (BIAS ? 220 : 200) * 1024;  // tiles, per CTA
+  static constexpr int SMEM_BUDGET = TILES == 1 ? (BIAS ? 112 : 110) * 1024 : 200 * 1024;  // tiles, per CTA
   static constexpr int NS_RAW = (SMEM_BUDGET - TILES * (TILE + BIAS_TILE)) / KV_TILE;
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
   static constexpr int OFF_BIAS = TILES * TILE + NS * KV_TILE;
-  static constexpr int SMEM_BAR = OFF_BIAS + TILES * BIAS_TILE;
-  static constexpr int SMEM_BYTES = SMEM_BAR + 256 + 1024;  // barriers + alignment slack
+  static constexpr int SMEM_BAR = OFF_BIAS + TILES * BIAS_TILE;  // the tiles' extent
+  // Dynamic shared memory a CTA may take with two per SM: 228 KB, less
+  // 1 KB the system reserves per CTA, halved.
+  static constexpr int SMEM_2CTA = (228 * 1024 - 2 * 1024) / 2;
+  // The barriers (256 bytes) go after the tiles, plus up to 1 KB of slack to
+  // align the tiles to 1024 bytes.  With one tile, a bias and d = 128 (Q,
+  // four K/V slots and the bias tile: 112 KB) that is 256 bytes too many for
+  // two CTAs per SM; there (TIGHT) the barriers take the alignment gap when
+  // it is 256 bytes or more, and follow the tiles otherwise (the gap is then
+  // under 256 bytes, so they still end within the 1 KB of slack).
+  static constexpr bool TIGHT = TILES == 1 && SMEM_BAR + 256 + 1024 > SMEM_2CTA;
+  static constexpr int SMEM_BYTES = SMEM_BAR + (TIGHT ? 0 : 256) + 1024;
   static constexpr int THREADS = 128 * TILES + 128;
   static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES], or S0 | S1 | O
   static constexpr int COL_O = TILES * SBUF * BN;            // first O column
@@ -105,9 +115,9 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
-  // K/V slots: two per score buffer, or (bias, one tile) three, so that K of
-  // tile j + 2 loads once P(j)·V(j) has read V(j)
-  static_assert(NS >= (BIAS && SBUF == 2 ? 3 : 2 * SBUF), "K/V slots for the products in flight");
+  static_assert(NS >= 2 * SBUF, "K/V slots for the products in flight");
+  static_assert(TILES == 2 || SMEM_BYTES <= SMEM_2CTA, "two one-tile CTAs per SM");
+  static_assert(!BIAS || TILES == 1, "the bias variants are one-tile kernels (fwd_tiles_for)");
   static_assert(NT == 2 || NT == 3, "two Q tiles, or one over 64-key K/V tiles");
   static_assert(NT != 3 || !ElemTraits<T>::tf32, "64-key tiles: 16-bit types");
   static_assert(COL_O + TILES * D <= TMEM_COLS, "TMEM budget");
@@ -215,7 +225,8 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-  FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(smem + Tr::SMEM_BAR);
+  FwdBarriers* bars = reinterpret_cast<FwdBarriers*>(
+      Tr::TIGHT && smem - smem_raw >= 256 ? smem_raw : smem + Tr::SMEM_BAR);
   volatile int* abort_flag = &bars->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -547,8 +558,10 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
             const uint32_t w = (c & 7) < 2 ? bv[c >> 3].x : (c & 7) < 4 ? bv[c >> 3].y
                              : (c & 7) < 6 ? bv[c >> 3].z : bv[c >> 3].w;
             const float2 b2 = ElemTraits<T>::unpack2(w);
-            su[q][e] = __float_as_uint(fmaf(b2.x, p.bias_mul, __uint_as_float(su[q][e])));
-            su[q][e + 1] = __float_as_uint(fmaf(b2.y, p.bias_mul, __uint_as_float(su[q][e + 1])));
+            const float2 r2 = upk2(ffma2(pk2(b2.x, b2.y), pk2(p.bias_mul, p.bias_mul),
+                                         pk2(__uint_as_float(su[q][e]), __uint_as_float(su[q][e + 1]))));
+            su[q][e] = __float_as_uint(r2.x);
+            su[q][e + 1] = __float_as_uint(r2.y);
           }
         }
       } else {
@@ -759,7 +772,7 @@ static cudaError_t launch_fwd_t(const FwdLaunch& a) {
   using Tr = FwdTraits<T, D, NT, BIAS && !ElemTraits<T>::tf32>;
   if (a.params.tiles != NT) return cudaErrorInvalidValue;  // the grid was sized for another count
   auto kern = fwd_kernel<T, D, CAUSAL, GEN, DROP, BIAS, NT>;
-  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES);
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(kern), Tr::SMEM_BYTES, Tr::TIGHT);
   if (e != cudaSuccess) return e;
   // setmaxnreg redistributes the registers the CTA was launched with; refuse
   // to launch if the compiled register count cannot cover the split.
@@ -784,7 +797,14 @@ int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool
   // vs 43.0–43.1, causal N = 1024 90.3 vs 108.6, N = 2048 142 vs 163,
   // N = 4096 244 vs 270, N = 8192 448–453 vs 485–489, B1 H32 N16384 1671 vs
   // 1813; non-causal N = 4096 450 vs 466, N = 8192 857 vs 888.
-  if (d != 128 || drop) return 3;
+  // With a bias: one tile with 64-key bias tiles and four K/V slots, against
+  // two tiles with 128-key bias tiles and two K/V slots (forward µs, d = 128
+  // bf16, head-shared [1, H, N, N] bias unless noted, interleaved A/B, both
+  // orders): non-causal N = 4096 406–432 vs 456–498, N = 8192 834–869 vs
+  // 1004–1046, N = 3072 (full bias) 244–261 vs 280–305; causal N = 2048
+  // 225–239 vs 259–274, N = 12288 1891–1948 vs 2100–2175, N = 16384
+  // 1631–1735 vs 1847–1917.
+  if (bias || d != 128 || drop) return 3;
   // 128-key K/V tiles a 128-row query tile sees, on average (bottom-right
   // causal: query tile i sees about i + 1 + (Nk − Nq) / 128 of them).  One Q
   // tile over 64-key K/V tiles with double-buffered scores, against two Q
@@ -792,12 +812,7 @@ int fwd_tiles_for(int dtype, int d, int Nq, int Nk, bool causal, bool drop, bool
   // both orders): causal N = 1024 104.6 vs 120.8, N = 2048 160.8 vs 177.6,
   // N = 4096 275–276 vs 281–282, N = 8192 506–510 vs 506–523, N = 16384 ×3
   // even; non-causal N = 2048 289 vs 296, N = 4096 508–509 vs 491–492,
-  // N = 8192 972–1050 vs 937–1044.  With a bias the same rule holds (one
-  // tile with a 3-slot ring, against two tiles with staged 128-key bias
-  // tiles, µs): causal N = 2048 head-shared [1, H, N, N] 240–253 vs
-  // 259–274, full 256–267 vs 277–289, query-broadcast 225–227 vs 248–249,
-  // causal N = 8192 495–513 vs 534–548; non-causal N = 4096 451–470 vs
-  // 462–480 (before the proxy fence on the bias tile, which costs ~3 %).
+  // N = 8192 972–1050 vs 937–1044.
   const double kv_tiles = (Nk + 127) / 128;
   const double q_tiles = (Nq + 127) / 128;
   const double avg = causal ? std::min(kv_tiles, (q_tiles + 1) / 2 + double(Nk - Nq) / 128) : kv_tiles;
@@ -811,11 +826,6 @@ cudaError_t launch_fwd(int dtype, int d, bool causal, const FwdLaunch& a) {
   // dropout and bias run in general-layout variants only
 #define FA_FWD_CASE(TY, DD)                                                                      \
   {                                                                                              \
-    if (bias && a.params.tiles == 2)                                                             \
-      return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true, 2>(a)                \
-                            : launch_fwd_t<TY, DD, true, true, false, true, 2>(a))              \
-                    : (drop ? launch_fwd_t<TY, DD, false, true, true, true, 2>(a)               \
-                            : launch_fwd_t<TY, DD, false, true, false, true, 2>(a));            \
     if (bias)                                                                                    \
       return causal ? (drop ? launch_fwd_t<TY, DD, true, true, true, true, 3>(a)                \
                             : launch_fwd_t<TY, DD, true, true, false, true, 3>(a))              \

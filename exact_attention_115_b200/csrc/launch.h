@@ -157,6 +157,8 @@ cudaError_t take_error_decode(int* word, int* site);
 cudaError_t launch_selftest_wait(unsigned long long limit_ns, cudaStream_t stream);
 
 // Sets the dynamic shared-memory limit of `kernel` on the current device once.
-cudaError_t set_smem_once(const void* kernel, int bytes);
+// Sets a kernel's dynamic shared-memory size once per device (and, with
+// max_carveout, asks for the largest shared-memory carveout of the SM).
+cudaError_t set_smem_once(const void* kernel, int bytes, bool max_carveout = false);
 
 }  // namespace fa

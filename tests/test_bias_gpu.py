@@ -85,9 +85,9 @@ def test_bias_rectangular_causal(fa):
 
 @pytest.mark.parametrize("bshape", ["full", "query_bcast"])
 def test_bias_long_rows(fa, bshape):
-    """Rows of 3100 keys at d = 128 (25 K/V tiles of 128 keys per query
-    tile) take the two-tile forward with its 128-key bias tiles; the shorter
-    rows above take the one-tile form with 64-key ones."""
+    """Rows of 3100 keys at d = 128: without a bias such rows take the
+    two-tile forward; with one they stay on the one-tile kernel and its
+    64-key bias tiles, here over 49 K/V steps (the ring wraps many times)."""
     B, H, Nq, Nk = 1, 2, 200, 3100
     q, k, v, do = W.make_tensors(B, H, Nq, Nk, 128, "bf16", seed=94, device="cuda")
     shape = (B, H, Nq) if bshape == "full" else (B, H, 1)
