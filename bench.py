@@ -230,6 +230,15 @@ def peak_fracs(achieved, peaks):
                                                          FALLBACK_PEAKS["bf16_tflops_sustained"]))}
 
 
+def fill_queue():
+    """Keep the device busy for ~10 ms (a bounded spin of torch's own) before
+    a timed region starts, so that the host has queued the region's launches
+    by the time the device reaches them: a short region (20 steps of the
+    causal 2K workload are ~13 ms of device work) then measures the device,
+    not the Python launch path and the clock-sampling thread."""
+    torch.cuda._sleep(20_000_000)
+
+
 def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_shape=None,
                   sampler=None):
     """fwd and bwd of one workload, each launch bracketed by CUDA events on
@@ -268,6 +277,7 @@ def time_workload(fa, w, dev, stream, iters, peaks, peak_kind, flush=None, bias_
     time.sleep(0.3)
     if sampler is not None:
         sampler.start()
+    fill_queue()
     for e in ev:
         if flush is not None:
             flush.zero_()
@@ -422,6 +432,7 @@ def main():
     sampler.start()
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
+    fill_queue()
     t_start.record(stream)
     for _ in range(K):
         step()
