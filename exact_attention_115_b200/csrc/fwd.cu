@@ -28,7 +28,8 @@
 //   last warpgroup: warp 4·TILES issues the tcgen05 MMAs (one thread) and
 //                   owns TMEM, the next warp is the TMA producer, the rest idle
 // TMEM: S[tiles] | O[tiles] (256 or 512 columns), or S0 | S1 | O (64, 64 and
-// d columns) with double-buffered scores.  P overwrites S in place
+// d columns) with double-buffered scores, at d = 64 followed by 16 columns
+// of row sums of the rounded P (a P · ones product; see FwdTraits::ONES).  P overwrites S in place
 // (bf16 pairs or tf32) and is read by the P·V MMA straight from TMEM.  The
 // running max is only moved when it grows by more than kRescaleThreshold
 // (log2 units), so the O accumulator is rescaled rarely; the result is exact
@@ -92,7 +93,13 @@ struct FwdTraits {
   static constexpr int NS_RAW = (SMEM_BUDGET - TILES * (TILE + BIAS_TILE)) / KV_TILE;
   static constexpr int NS = NS_RAW > 8 ? 8 : NS_RAW;  // K/V ring slots
   static constexpr int OFF_BIAS = TILES * TILE + NS * KV_TILE;
-  static constexpr int SMEM_BAR = OFF_BIAS + TILES * BIAS_TILE;  // the tiles' extent
+  // d = 64, one tile: the row sums of P as rounded for the P·V product come
+  // from the tensor core, P · ones[64 keys × 16] into 16 TMEM columns after
+  // O, with the B operand a constant [16 × 64] K-major tile of ones.
+  static constexpr bool ONES = SBUF == 2 && D == 64;
+  static constexpr int ONES_TILE = ONES ? 16 * 128 : 0;
+  static constexpr int OFF_ONES = OFF_BIAS + TILES * BIAS_TILE;
+  static constexpr int SMEM_BAR = OFF_ONES + ONES_TILE;  // the tiles' extent
   // Dynamic shared memory a CTA may take with two per SM: 228 KB, less
   // 1 KB the system reserves per CTA, halved.
   static constexpr int SMEM_2CTA = (228 * 1024 - 2 * 1024) / 2;
@@ -107,6 +114,7 @@ struct FwdTraits {
   static constexpr int THREADS = 128 * TILES + 128;
   static constexpr int TMEM_COLS = TILES == 1 ? 256 : 512;  // S[TILES] | O[TILES], or S0 | S1 | O
   static constexpr int COL_O = TILES * SBUF * BN;            // first O column
+  static constexpr int COL_R = COL_O + TILES * D;            // ONES: the row sums (16 columns)
   static constexpr int MMA_WARP = 4 * TILES;                // then the TMA producer
   static constexpr int PRODUCER_WARP = MMA_WARP + 1;
   // setmaxnreg split of the registers a CTA launches with (65536 / CTAS_PER_SM)
@@ -115,12 +123,13 @@ struct FwdTraits {
   static constexpr uint32_t IDESC_QK = make_idesc(ElemTraits<T>::fmt, 128, BN, 0, 0);
   static constexpr uint32_t IDESC_PV =
       make_idesc(ElemTraits<T>::fmt, 128, D, 0, ElemTraits<T>::tf32 ? 0 : 1);
+  static constexpr uint32_t IDESC_R = make_idesc(ElemTraits<T>::fmt, 128, 16, 0, 0);
   static_assert(NS >= 2 * SBUF, "K/V slots for the products in flight");
   static_assert(TILES == 2 || SMEM_BYTES <= SMEM_2CTA, "two one-tile CTAs per SM");
   static_assert(!BIAS || TILES == 1, "the bias variants are one-tile kernels (fwd_tiles_for)");
   static_assert(NT == 2 || NT == 3, "two Q tiles, or one over 64-key K/V tiles");
   static_assert(NT != 3 || !ElemTraits<T>::tf32, "64-key tiles: 16-bit types");
-  static_assert(COL_O + TILES * D <= TMEM_COLS, "TMEM budget");
+  static_assert(COL_O + TILES * D + (ONES ? 32 : 0) <= TMEM_COLS, "TMEM budget");
   static_assert(D % AW == 0, "head dim must fill whole swizzle rows");
 };
 
@@ -222,6 +231,9 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
   // staged bias tiles (16-bit types)
   constexpr bool SBIAS = BIAS && !ElemTraits<T>::tf32;
   constexpr bool TF32 = ElemTraits<T>::tf32;
+  // the rounded-P row sums by the tensor core (with dropout the product sees
+  // the dropped weights, so the sums stay in the softmax threads)
+  constexpr bool RSUM = Tr::ONES && !DROP;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -276,6 +288,14 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
     tma_prefetch_desc(&tmK);
     tma_prefetch_desc(&tmV);
     if constexpr (SBIAS) tma_prefetch_desc(&tmBias);
+  }
+  if constexpr (RSUM) {
+    if (warp == Tr::PRODUCER_WARP) {
+      const uint32_t one2 = ElemTraits<T>::pack2(1.f, 1.f);
+      for (int i = lane; i < Tr::ONES_TILE / 16; i += 32)
+        reinterpret_cast<uint4*>(smem + Tr::OFF_ONES)[i] = make_uint4(one2, one2, one2, one2);
+      fence_async_smem();  // the tensor core reads it
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -406,6 +426,15 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           if (leader) mma_ts<TF32>(tO[t], tS[sb] + ks * 8, db + o, Tr::IDESC_PV, (acc || ks > 0) ? 1u : 0u);
         }
       };
+      // RSUM: the row sums of P (score buffer sb) += P · ones
+      auto issue_rsum = [&](int sb, bool acc) {
+        const uint64_t db = sw128_desc(smem_u32(smem + Tr::OFF_ONES), 16, 1024);
+#pragma unroll
+        for (int ks = 0; ks < Tr::BN / Tr::KSTEP; ++ks)
+          if (leader)
+            mma_ts<false>(tmem + Tr::COL_R, tS[sb] + ks * 8, db + uint64_t(ks * 2), Tr::IDESC_R,
+                          (acc || ks > 0) ? 1u : 0u);
+      };
       auto commit = [&](uint64_t* bar) {
         if (leader) tc_commit(bar);
       };
@@ -438,6 +467,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
           tc_fence_after();
           if (!ok) break;
           issue_pv(0, sv, j > 0, b);
+          if constexpr (RSUM) issue_rsum(b, j > 0);
           commit(&bars->o_full[0]);
           if (j + 1 == n_kv) commit(&bars->o_full[1]);  // the tile's last product, for the epilogue
           commit(&bars->kv_empty[sv]);
@@ -609,7 +639,7 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
         tc_fence_after();
         if (!ok) break;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
+        for (int c = 0; c < D + (RSUM ? 32 : 0); c += 32) {  // (RSUM: the row sums follow O)
           uint32_t u[32];
           tmem_ld32(tO + c, u);
           tmem_ld_wait();
@@ -663,9 +693,11 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
             const float2 pe = (EP > 0 && e % EP == EP - 1) ? exp2_pair<true>(x)
                                                                   : exp2_pair<false>(x);
             u[e] = ElemTraits<T>::pack2(pe.x, pe.y);
-            const float2 pr = ElemTraits<T>::unpack2(u[e]);
             sum2[q] = fadd2(sum2[q], pk2(pe.x, pe.y));
-            sum2_p[q] = fadd2(sum2_p[q], pk2(pr.x, pr.y));
+            if constexpr (!RSUM) {
+              const float2 pr = ElemTraits<T>::unpack2(u[e]);
+              sum2_p[q] = fadd2(sum2_p[q], pk2(pr.x, pr.y));
+            }
             // the product sees the dropped weights; the sums above do not
             if constexpr (DROP) u[e] &= keep_pair_mask(keep[e / 2], (2 * e) & 3);
           }
@@ -691,6 +723,12 @@ __global__ void __launch_bounds__(FwdTraits<T, D, NT, BIAS>::THREADS, FwdTraits<
                                                  : MBAR_WAIT(&bars->o_full[t], (n_kv - 1) & 1, abort_flag));
     tc_fence_after();
     if (ok) {
+      if constexpr (RSUM) {  // the row sum of the rounded P, after O in TMEM
+        uint32_t u[32];
+        tmem_ld32(tO + D, u);
+        tmem_ld_wait();
+        row_sum_p = __uint_as_float(u[0]);
+      }
       // A row whose every score was masked (m_ref still -inf) has O = 0: the
       // FMA-pipe exponentials leave it tiny but nonzero weights otherwise.
       float inv = (row_sum_p > 0.f && m_ref != -INFINITY) ? 1.f / row_sum_p : 0.f;
